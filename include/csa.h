@@ -1,0 +1,225 @@
+/*
+ * csa.h -- C ABI of the CSA / HCA hot path (B200, sm_100a).
+ *
+ * The method is DeepSeek-V4's Compressed Sparse Attention (CSA) and Heavily
+ * Compressed Attention (HCA), as restated on the pages "DeepSeek-V4: Towards
+ * Highly Efficient Million-Token Context Intelligence" (ai-papers-daily notes,
+ * Modules B, C, D, F) and "DeepSeek V4 大模型算法解析" (section 二 核心算法).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor pointers are DEVICE pointers to dense, row-major, contiguous
+ *    buffers that the caller owns and allocates. The library allocates no
+ *    memory and keeps no state between calls except one device error word
+ *    per GPU (see csa_get_error).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). Every call only enqueues work on it and returns; results are
+ *    ready when the stream reaches that point.
+ *  - Positions: q_pos[b][t] is the absolute position of a query in its
+ *    sequence (prefill: 0 .. n-1; decode: the context length minus one).
+ *    The compressed entries visible to a query at position t are
+ *    V_t = min(E, floor((t + 1) / m)): entry i covers tokens m*i .. m*i+m-1
+ *    and is visible once its last token is at or before t.
+ *  - Validation: each call checks its arguments on the host (null pointers,
+ *    sizes, 16-byte alignment of every vector-loaded buffer, supported
+ *    dtype/shape combinations) before launching anything. On failure it
+ *    returns CSA_ERR_INVALID_ARG or CSA_ERR_UNSUPPORTED, launches nothing and
+ *    writes nothing; csa_last_message() then describes the failure.
+ *  - Device-side checks (a selection index outside [0, V_t), a window
+ *    position outside the window buffer) never trap: the offending key is
+ *    skipped and the device error word records CSA_ERR_BOUNDS, which
+ *    csa_get_error reports.
+ *  - A launch failure returns CSA_ERR_CUDA.
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CSA_F32 = 0,   /* IEEE binary32 */
+    CSA_BF16 = 1,  /* bfloat16 */
+    CSA_E4M3 = 2   /* 8-bit float e4m3 (finite, max 448), always with scales */
+} csa_dtype;
+
+typedef enum {
+    CSA_OK = 0,
+    CSA_ERR_INVALID_ARG = -1,
+    CSA_ERR_UNSUPPORTED = -2,
+    CSA_ERR_CUDA = -3,
+    CSA_ERR_TIMEOUT = -4,
+    CSA_ERR_BOUNDS = -5
+} csa_status;
+
+/*
+ * A table of KV entries of width c, `rows` rows (compressed entries, or
+ * indexer keys of width c_I).
+ *   plain layout: dt = CSA_F32 or CSA_BF16, rope_dims = 0, scale = rope =
+ *     NULL; body is [rows, c].
+ *   fp8 layout (low-precision KV storage, Module F): dt = CSA_E4M3;
+ *     body is [rows, c - rope_dims] e4m3 codes; scale is
+ *     [rows, (c - rope_dims) / scale_group] float32 (> 0); the value of
+ *     body[r][j] is code * scale[r][j / scale_group]; when rope_dims > 0 the
+ *     trailing rope_dims channels are stored unscaled as bfloat16 in rope
+ *     [rows, rope_dims].
+ * The same struct describes inputs (read) and outputs (written); `body`,
+ * `scale` and `rope` are cast to const by readers.
+ */
+typedef struct {
+    void *body;
+    float *scale;
+    void *rope;
+    int c;
+    int rope_dims;
+    int scale_group;
+    csa_dtype dt;
+} csa_entries;
+
+/* ABI version: bumped on any incompatible change of this header. */
+int csa_abi_version(void);
+
+/* Human-readable text of a status code (static storage). */
+const char *csa_status_string(csa_status s);
+
+/* Text of the last host-side validation failure of this thread (static,
+ * thread-local storage; empty when none). */
+const char *csa_last_message(void);
+
+/*
+ * csa_compress_kv -- token-level compressor.
+ *   CSA (overlap = 1), Eq. 9-12 (Module B step 1; the overlapping windows of
+ *   "第一阶段"): entry i, channel j pools rows m*i .. m*i+m-1 of Ca and rows
+ *   m*(i-1) .. m*i-1 of Cb with the softmax (over those 2m token positions,
+ *   per channel) of the logits Za + Ba and Zb + Bb. Entry 0 has no previous
+ *   block: its Cb half is left out of the softmax.
+ *   HCA (overlap = 0), Eq. 20-23 (Module C): m = m' rows of Ca with logits
+ *   Za + Ba; Cb, Zb and Bb must be NULL.
+ * Arguments:
+ *   Ca, Cb, Za, Zb  [n, c] of in_dt (F32 or BF16), rows = tokens.
+ *   Ba, Bb          [m, c] float32 position biases.
+ *   n               tokens; n % m == 0 (an incomplete tail block is not an
+ *                   entry); E = n / m entries are written.
+ *   out             [E, c] entries: plain F32/BF16, or the fp8 layout with
+ *                   scale_group dividing c - rope_dims (per-group scale =
+ *                   max(amax / 448, 2^-126), codes rounded to nearest even
+ *                   and saturated; rope channels stored as bf16).
+ * Requirements: c % 8 == 0 (bf16) or c % 4 == 0 (f32), 1 <= m <= 1024,
+ *   all buffers 16-byte aligned.
+ */
+csa_status csa_compress_kv(const void *Ca, const void *Cb, const void *Za, const void *Zb,
+                           const float *Ba, const float *Bb, int64_t n, int c, int m,
+                           int overlap, csa_dtype in_dt, csa_entries out, void *stream);
+
+/*
+ * csa_indexer_scores -- lightning-indexer scores, Eq. 16 (Module B step 2):
+ *   I[b][t][s] = sum_h wI[b][t][h] * ReLU(qI[b][t][h] . kI[b][s])
+ * for every visible entry s < V_t. There is no softmax and no scale factor.
+ * Entries s >= V_t of a score row are NOT written (the selection never
+ * reads them).
+ * Arguments:
+ *   qI        [B, n_q, hI, cI] of dt; dt = CSA_E4M3 requires qI_scale
+ *             [B, n_q, hI] float32 > 0 (one scale per query head), else NULL.
+ *   wI        [B, n_q, hI] float32 head weights.
+ *   kI        keys, rows = B * E (batch b owns rows b*E .. b*E+E-1), c = cI;
+ *             kI.dt must equal dt; for CSA_E4M3, scale_group == cI (one
+ *             positive scale per key) and rope_dims == 0.
+ *   q_pos     [B, n_q] int64 query positions.
+ *   m         compression ratio used for visibility.
+ *   scores    [B, n_q, ld] float32, ld >= E.
+ * Requirements: cI % 16 == 0, cI <= 256, 1 <= hI <= 128.
+ */
+csa_status csa_indexer_scores(const void *qI, const float *qI_scale, const float *wI,
+                              csa_entries kI, const int64_t *q_pos, int B, int64_t n_q,
+                              int64_t E, int hI, int cI, int m, csa_dtype dt, float *scores,
+                              int64_t ld, void *stream);
+
+/*
+ * csa_topk -- top-k selector, Eq. 17 (Module B step 2):
+ * for each row r, the min(k, V_r) visible entries (s < V_r, V_r from
+ * q_pos[r] and m) with the largest scores. Equal scores prefer the lower
+ * index (+0 and -0 are equal). The row of idx lists the chosen indices in
+ * ascending order, then -1 up to k. Scores must not be NaN.
+ * Arguments:
+ *   scores    [rows, ld] float32 (only s < V_r is read).
+ *   q_pos     [rows] int64.
+ *   idx       [rows, k] int32 output.
+ *   workspace, ws_bytes   device scratch of at least
+ *             csa_topk_workspace_size(rows, E, k) bytes (may be NULL when that
+ *             size is 0).
+ * Requirements: 1 <= k <= 4096.
+ */
+csa_status csa_topk(const float *scores, int64_t rows, int64_t E, int64_t ld,
+                    const int64_t *q_pos, int m, int k, int32_t *idx, void *workspace,
+                    size_t ws_bytes, void *stream);
+size_t csa_topk_workspace_size(int64_t rows, int64_t E, int k);
+
+/*
+ * csa_sparse_mqa -- shared-KV multi-query attention over the selected
+ * compressed entries, Eq. 18-19 (Module B step 3), joined by the sliding-window
+ * branch and the attention sink (Module D). Every key is also its own value.
+ * For query (b, t) and head i the key set is
+ *   { kv[b][idx[b*n_q+t][j]] : idx >= 0 }  (entries, each must be < V_t)
+ *   U { kwin[b][p - win_pos0[b]] : max(0, t - n_win + 1) <= p <= t }
+ * and, with z_j = scale * q . key_j, M = max(max_j z_j, sink[i]),
+ *   out = sum_j e^{z_j - M} key_j / (sum_j e^{z_j - M} + e^{sink[i] - M})
+ *   lse = M + log(sum_j e^{z_j - M} + e^{sink[i] - M}).
+ * Arguments:
+ *   q         [B, n_q, h, c] of q_dt (F32 or BF16); out has the same shape
+ *             and dtype.
+ *   kv        entries, rows = B * E (batch b owns rows b*E ..), width c;
+ *             plain (dt == q_dt) or the fp8 layout (bf16 queries only).
+ *   E, m      entries per batch and the compression ratio that fixes
+ *             V_t = min(E, floor((t + 1) / m)); a listed index outside
+ *             [0, V_t) is skipped and recorded as CSA_ERR_BOUNDS.
+ *   idx       [B * n_q, k] int32 (ascending or not; -1 = empty slot).
+ *   kwin      [B, win_rows, c] of q_dt: raw KV rows; row r of batch b holds
+ *             position win_pos0[b] + r (win_pos0 NULL means 0).
+ *   sink      [h] float32 per-head sink logits (-inf disables the sink).
+ *   lse       [B, n_q, h] float32 or NULL.
+ *   workspace csa_mqa_workspace_size(...) bytes of device scratch, or NULL
+ *             when that size is 0.
+ * Requirements: c a power of two from 64 to 1024, 1 <= h <= 128,
+ *   0 <= k <= 4096, n_win >= 0; q, out, kwin and entry buffers 16-byte
+ *   aligned.
+ */
+csa_status csa_sparse_mqa(const void *q, csa_dtype q_dt, csa_entries kv, int64_t E, int m,
+                          const int32_t *idx, int k, const void *kwin, int64_t win_rows,
+                          const int64_t *win_pos0, int n_win, const int64_t *q_pos,
+                          const float *sink, int B, int64_t n_q, int h, float scale,
+                          void *out, float *lse, void *workspace, size_t ws_bytes,
+                          void *stream);
+
+/*
+ * hca_dense_mqa -- HCA core attention, Eq. 24-26 (Module C): as
+ * csa_sparse_mqa, but every visible entry s < V_t (V_t from m = m') is a key
+ * instead of a selection.
+ */
+csa_status hca_dense_mqa(const void *q, csa_dtype q_dt, csa_entries kv, int64_t E, int m,
+                         const void *kwin, int64_t win_rows, const int64_t *win_pos0,
+                         int n_win, const int64_t *q_pos, const float *sink, int B,
+                         int64_t n_q, int h, float scale, void *out, float *lse,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/* Device scratch bytes that csa_sparse_mqa / hca_dense_mqa need for this
+ * shape (split-KV partial results for small query counts); 0 when none. */
+size_t csa_mqa_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys);
+
+/*
+ * csa_get_error -- synchronises the current device, reads and clears its
+ * device error word, and returns the status it held (CSA_OK if none). When
+ * buf is not NULL, a description (at most len bytes, NUL-terminated) is
+ * written to it. Call it after a batch of work to confirm that no device-side
+ * check fired.
+ */
+csa_status csa_get_error(char *buf, size_t len);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H */

@@ -1,0 +1,298 @@
+// api.cu -- the C ABI of csa.h: argument validation, device error word and
+// dispatch to the kernel launchers. No call allocates device memory.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+__device__ unsigned g_err[4];
+
+thread_local char g_msg[512];
+
+csa_status fail(csa_status st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+constexpr int kMaxDevices = 64;
+unsigned *g_err_ptr[kMaxDevices];
+
+// Device address of this GPU's error word (looked up once per device).
+unsigned *err_word()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return nullptr;
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_err) != cudaSuccess)
+            return nullptr;
+        g_err_ptr[dev] = (unsigned *)p;
+    }
+    return g_err_ptr[dev];
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+bool pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+csa_status launched(cudaError_t e, const char *what)
+{
+    if (e != cudaSuccess)
+        return fail(CSA_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+    g_msg[0] = 0;
+    return CSA_OK;
+}
+
+#define REQUIRE(cond, st, ...)                                                           \
+    do {                                                                                 \
+        if (!(cond))                                                                     \
+            return fail(st, __VA_ARGS__);                                                \
+    } while (0)
+
+csa_status check_entries(const csa_entries &t, int c, bool allow_fp8, const char *what)
+{
+    REQUIRE(t.body, CSA_ERR_INVALID_ARG, "%s: body is NULL", what);
+    REQUIRE(t.c == c, CSA_ERR_INVALID_ARG, "%s: c = %d, expected %d", what, t.c, c);
+    REQUIRE(aligned16(t.body), CSA_ERR_INVALID_ARG, "%s: body not 16-byte aligned", what);
+    if (t.dt == CSA_E4M3) {
+        REQUIRE(allow_fp8, CSA_ERR_UNSUPPORTED, "%s: e4m3 entries not supported here", what);
+        REQUIRE(t.scale && aligned16(t.scale), CSA_ERR_INVALID_ARG,
+                "%s: e4m3 entries need 16-byte aligned scales", what);
+        REQUIRE(t.rope_dims >= 0 && t.rope_dims < c, CSA_ERR_INVALID_ARG,
+                "%s: rope_dims = %d out of range", what, t.rope_dims);
+        REQUIRE((t.rope_dims > 0) == (t.rope != nullptr), CSA_ERR_INVALID_ARG,
+                "%s: rope pointer must be given exactly when rope_dims > 0", what);
+        REQUIRE(!t.rope || aligned16(t.rope), CSA_ERR_INVALID_ARG,
+                "%s: rope not 16-byte aligned", what);
+        REQUIRE(t.scale_group > 0 && (c - t.rope_dims) % t.scale_group == 0,
+                CSA_ERR_INVALID_ARG, "%s: scale_group %d must divide c - rope_dims = %d", what,
+                t.scale_group, c - t.rope_dims);
+        REQUIRE((c - t.rope_dims) % 16 == 0 && t.rope_dims % 8 == 0, CSA_ERR_UNSUPPORTED,
+                "%s: c - rope_dims must be a multiple of 16 and rope_dims of 8", what);
+    } else {
+        REQUIRE(t.dt == CSA_F32 || t.dt == CSA_BF16, CSA_ERR_INVALID_ARG,
+                "%s: unknown dtype %d", what, (int)t.dt);
+        REQUIRE(t.rope_dims == 0, CSA_ERR_INVALID_ARG,
+                "%s: rope_dims must be 0 for plain entries", what);
+    }
+    return CSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int csa_abi_version(void) { return 1; }
+
+const char *csa_status_string(csa_status s)
+{
+    switch (s) {
+    case CSA_OK: return "ok";
+    case CSA_ERR_INVALID_ARG: return "invalid argument";
+    case CSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case CSA_ERR_CUDA: return "CUDA error";
+    case CSA_ERR_TIMEOUT: return "device wait timed out";
+    case CSA_ERR_BOUNDS: return "index out of bounds on the device";
+    }
+    return "unknown status";
+}
+
+const char *csa_last_message(void) { return g_msg; }
+
+csa_status csa_compress_kv(const void *Ca, const void *Cb, const void *Za, const void *Zb,
+                           const float *Ba, const float *Bb, int64_t n, int c, int m,
+                           int overlap, csa_dtype in_dt, csa_entries out, void *stream)
+{
+    const char *w = "csa_compress_kv";
+    REQUIRE(Ca && Za && Ba, CSA_ERR_INVALID_ARG, "%s: Ca, Za and Ba are required", w);
+    if (overlap)
+        REQUIRE(Cb && Zb && Bb, CSA_ERR_INVALID_ARG, "%s: overlap needs Cb, Zb and Bb", w);
+    else
+        REQUIRE(!Cb && !Zb && !Bb, CSA_ERR_INVALID_ARG,
+                "%s: without overlap Cb, Zb and Bb must be NULL", w);
+    REQUIRE(m >= 1 && m <= 1024, CSA_ERR_INVALID_ARG, "%s: m = %d out of [1, 1024]", w, m);
+    REQUIRE(n >= 0 && n % m == 0, CSA_ERR_INVALID_ARG, "%s: n = %lld must be a multiple of m",
+            w, (long long)n);
+    REQUIRE(in_dt == CSA_F32 || in_dt == CSA_BF16, CSA_ERR_UNSUPPORTED,
+            "%s: input dtype must be F32 or BF16", w);
+    const int vec = in_dt == CSA_BF16 ? 8 : 4;
+    REQUIRE(c > 0 && c % vec == 0 && pow2(c / vec) && c / vec <= 256, CSA_ERR_UNSUPPORTED,
+            "%s: c = %d unsupported (c / %d must be a power of two <= 256)", w, c, vec);
+    REQUIRE(aligned16(Ca) && aligned16(Za) && aligned16(Ba) && (!overlap ||
+            (aligned16(Cb) && aligned16(Zb) && aligned16(Bb))), CSA_ERR_INVALID_ARG,
+            "%s: inputs must be 16-byte aligned", w);
+    csa_status st = check_entries(out, c, true, "csa_compress_kv(out)");
+    if (st != CSA_OK)
+        return st;
+    if (out.dt == CSA_E4M3) {
+        REQUIRE(out.scale_group % vec == 0 && pow2(out.scale_group / vec) &&
+                out.scale_group / vec <= 32, CSA_ERR_UNSUPPORTED,
+                "%s: scale_group %d unsupported for this input dtype", w, out.scale_group);
+    }
+    unsigned *err = err_word();
+    REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
+    csa::CompressArgs a{Ca, Cb, Za, Zb, Ba, Bb, n, c, m, overlap ? 1 : 0, in_dt, out};
+    return launched(csa::launch_compress(a, err, (cudaStream_t)stream), w);
+}
+
+csa_status csa_indexer_scores(const void *qI, const float *qI_scale, const float *wI,
+                              csa_entries kI, const int64_t *q_pos, int B, int64_t n_q,
+                              int64_t E, int hI, int cI, int m, csa_dtype dt, float *scores,
+                              int64_t ld, void *stream)
+{
+    const char *w = "csa_indexer_scores";
+    REQUIRE(qI && wI && q_pos && scores, CSA_ERR_INVALID_ARG,
+            "%s: qI, wI, q_pos and scores are required", w);
+    REQUIRE(B >= 0 && n_q >= 0 && E >= 0 && E <= INT32_MAX, CSA_ERR_INVALID_ARG,
+            "%s: bad B / n_q / E", w);
+    REQUIRE(hI >= 1 && hI <= 128, CSA_ERR_UNSUPPORTED, "%s: hI = %d out of [1, 128]", w, hI);
+    REQUIRE(cI >= 16 && cI <= 256 && cI % 16 == 0, CSA_ERR_UNSUPPORTED,
+            "%s: cI = %d unsupported", w, cI);
+    REQUIRE(m >= 1, CSA_ERR_INVALID_ARG, "%s: m must be >= 1", w);
+    REQUIRE(ld >= E, CSA_ERR_INVALID_ARG, "%s: ld < E", w);
+    REQUIRE(dt == CSA_F32 || dt == CSA_BF16 || dt == CSA_E4M3, CSA_ERR_INVALID_ARG,
+            "%s: unknown dtype", w);
+    REQUIRE(kI.dt == dt, CSA_ERR_INVALID_ARG, "%s: kI dtype differs from qI dtype", w);
+    csa_status st = check_entries(kI, cI, true, "csa_indexer_scores(kI)");
+    if (st != CSA_OK)
+        return st;
+    if (dt == CSA_E4M3) {
+        REQUIRE(qI_scale, CSA_ERR_INVALID_ARG, "%s: e4m3 queries need qI_scale", w);
+        REQUIRE(kI.scale_group == cI && kI.rope_dims == 0, CSA_ERR_UNSUPPORTED,
+                "%s: e4m3 keys need one scale per key and no rope part", w);
+    }
+    REQUIRE(aligned16(qI), CSA_ERR_INVALID_ARG, "%s: qI not 16-byte aligned", w);
+    unsigned *err = err_word();
+    REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
+    csa::IndexerArgs a{qI, qI_scale, wI, kI, q_pos, B, n_q, E, hI, cI, m, dt, scores, ld};
+    if ((int64_t)B * n_q == 0 || E == 0)
+        return CSA_OK;
+    return launched(csa::launch_indexer(a, err, (cudaStream_t)stream), w);
+}
+
+size_t csa_topk_workspace_size(int64_t rows, int64_t E, int k)
+{
+    (void)rows; (void)E; (void)k;
+    return 0;
+}
+
+csa_status csa_topk(const float *scores, int64_t rows, int64_t E, int64_t ld,
+                    const int64_t *q_pos, int m, int k, int32_t *idx, void *workspace,
+                    size_t ws_bytes, void *stream)
+{
+    const char *w = "csa_topk";
+    (void)workspace; (void)ws_bytes;
+    REQUIRE(scores && q_pos && idx, CSA_ERR_INVALID_ARG, "%s: scores, q_pos and idx required", w);
+    REQUIRE(rows >= 0 && rows <= INT32_MAX && E >= 0 && E <= INT32_MAX && ld >= E,
+            CSA_ERR_INVALID_ARG, "%s: bad rows / E / ld", w);
+    REQUIRE(k >= 1 && k <= 4096, CSA_ERR_UNSUPPORTED, "%s: k = %d out of [1, 4096]", w, k);
+    REQUIRE(m >= 1, CSA_ERR_INVALID_ARG, "%s: m must be >= 1", w);
+    unsigned *err = err_word();
+    REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
+    csa::TopkArgs a{scores, rows, E, ld, q_pos, m, k, idx};
+    return launched(csa::launch_topk(a, err, (cudaStream_t)stream), w);
+}
+
+size_t csa_mqa_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys)
+{
+    return csa::attend_workspace_size(B, n_q, h, c, max_keys);
+}
+
+static csa_status attend_common(const char *w, const void *q, csa_dtype q_dt, csa_entries kv,
+                                int64_t E, const int32_t *idx, int k, int m, const void *kwin,
+                                int64_t win_rows, const int64_t *win_pos0, int n_win,
+                                const int64_t *q_pos, const float *sink, int B, int64_t n_q,
+                                int h, float scale, void *out, float *lse, void *workspace,
+                                size_t ws_bytes, void *stream)
+{
+    REQUIRE(q && out && q_pos && sink, CSA_ERR_INVALID_ARG,
+            "%s: q, out, q_pos and sink are required", w);
+    REQUIRE(q_dt == CSA_F32 || q_dt == CSA_BF16, CSA_ERR_UNSUPPORTED,
+            "%s: q dtype must be F32 or BF16", w);
+    const int c = kv.c;
+    REQUIRE(c >= 64 && c <= 1024 && pow2(c), CSA_ERR_UNSUPPORTED,
+            "%s: c = %d unsupported (a power of two from 64 to 1024)", w, c);
+    csa_status st = check_entries(kv, c, q_dt == CSA_BF16, w);
+    if (st != CSA_OK)
+        return st;
+    REQUIRE(kv.dt == q_dt || kv.dt == CSA_E4M3, CSA_ERR_UNSUPPORTED,
+            "%s: entries dtype must match q (or be e4m3 with bf16 q)", w);
+    REQUIRE(h >= 1 && h <= 128, CSA_ERR_UNSUPPORTED, "%s: h = %d out of [1, 128]", w, h);
+    REQUIRE(B >= 0 && n_q >= 0 && (int64_t)B * n_q <= INT32_MAX && E >= 0 && E <= INT32_MAX,
+            CSA_ERR_INVALID_ARG, "%s: bad B / n_q / E", w);
+    REQUIRE(m >= 1, CSA_ERR_INVALID_ARG, "%s: m must be >= 1", w);
+    REQUIRE(k >= 0 && k <= 4096, CSA_ERR_UNSUPPORTED, "%s: k = %d out of [0, 4096]", w, k);
+    REQUIRE(k == 0 || idx, CSA_ERR_INVALID_ARG, "%s: idx required when k > 0", w);
+    REQUIRE(n_win >= 0, CSA_ERR_INVALID_ARG, "%s: n_win < 0", w);
+    REQUIRE(n_win == 0 || (kwin && win_rows >= 1 && aligned16(kwin)), CSA_ERR_INVALID_ARG,
+            "%s: a window needs a 16-byte aligned kwin with win_rows >= 1", w);
+    REQUIRE(aligned16(q) && aligned16(out), CSA_ERR_INVALID_ARG,
+            "%s: q and out must be 16-byte aligned", w);
+    const size_t need = csa::attend_workspace_size(B, n_q, h, c, (idx ? k : E) + n_win);
+    REQUIRE(ws_bytes >= need && (need == 0 || workspace), CSA_ERR_INVALID_ARG,
+            "%s: workspace of %zu bytes required", w, need);
+    unsigned *err = err_word();
+    REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
+    if ((int64_t)B * n_q == 0)
+        return CSA_OK;
+    csa::AttendArgs a{q, q_dt, kv, E, idx, k, m, kwin, n_win > 0 ? win_rows : 0, win_pos0,
+                      n_win, q_pos, sink, B, n_q, h, scale, out, lse, workspace, ws_bytes};
+    return launched(csa::launch_attend(a, err, (cudaStream_t)stream), w);
+}
+
+csa_status csa_sparse_mqa(const void *q, csa_dtype q_dt, csa_entries kv, int64_t E, int m,
+                          const int32_t *idx, int k, const void *kwin, int64_t win_rows,
+                          const int64_t *win_pos0, int n_win, const int64_t *q_pos,
+                          const float *sink, int B, int64_t n_q, int h, float scale,
+                          void *out, float *lse, void *workspace, size_t ws_bytes,
+                          void *stream)
+{
+    return attend_common("csa_sparse_mqa", q, q_dt, kv, E, idx, k, m, kwin, win_rows,
+                         win_pos0, n_win, q_pos, sink, B, n_q, h, scale, out, lse, workspace,
+                         ws_bytes, stream);
+}
+
+csa_status hca_dense_mqa(const void *q, csa_dtype q_dt, csa_entries kv, int64_t E, int m,
+                         const void *kwin, int64_t win_rows, const int64_t *win_pos0,
+                         int n_win, const int64_t *q_pos, const float *sink, int B,
+                         int64_t n_q, int h, float scale, void *out, float *lse,
+                         void *workspace, size_t ws_bytes, void *stream)
+{
+    return attend_common("hca_dense_mqa", q, q_dt, kv, E, nullptr, 0, m, kwin, win_rows,
+                         win_pos0, n_win, q_pos, sink, B, n_q, h, scale, out, lse, workspace,
+                         ws_bytes, stream);
+}
+
+csa_status csa_get_error(char *buf, size_t len)
+{
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        if (buf && len)
+            snprintf(buf, len, "CUDA error: %s", cudaGetErrorString(cudaGetLastError()));
+        return CSA_ERR_CUDA;
+    }
+    unsigned h[4] = {0, 0, 0, 0};
+    if (cudaMemcpyFromSymbol(h, g_err, sizeof h) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    const unsigned zero[4] = {0, 0, 0, 0};
+    if (cudaMemcpyToSymbol(g_err, zero, sizeof zero) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    const csa_status st = (csa_status)(-(int)h[0]);
+    if (buf && len) {
+        if (h[0])
+            snprintf(buf, len, "%s (kernel %u, detail %u %u)", csa_status_string(st), h[1], h[2],
+                     h[3]);
+        else
+            snprintf(buf, len, "%s", "ok");
+    }
+    return st;
+}
+
+}  // extern "C"

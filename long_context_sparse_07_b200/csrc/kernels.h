@@ -1,0 +1,69 @@
+// kernels.h -- host-side launchers of the device kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "csa.h"
+
+namespace csa {
+
+struct CompressArgs {
+    const void *Ca, *Cb, *Za, *Zb;
+    const float *Ba, *Bb;
+    int64_t n;
+    int c, m, overlap;
+    csa_dtype in_dt;
+    csa_entries out;
+};
+cudaError_t launch_compress(const CompressArgs &a, unsigned *err, cudaStream_t s);
+
+struct IndexerArgs {
+    const void *qI;
+    const float *qI_scale, *wI;
+    csa_entries kI;
+    const int64_t *q_pos;
+    int B;
+    int64_t n_q, E;
+    int hI, cI, m;
+    csa_dtype dt;
+    float *scores;
+    int64_t ld;
+};
+cudaError_t launch_indexer(const IndexerArgs &a, unsigned *err, cudaStream_t s);
+
+struct TopkArgs {
+    const float *scores;
+    int64_t rows, E, ld;
+    const int64_t *q_pos;
+    int m, k;
+    int32_t *idx;
+};
+cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s);
+
+struct AttendArgs {
+    const void *q;
+    csa_dtype q_dt;
+    csa_entries kv;
+    int64_t E;
+    const int32_t *idx;   // NULL = dense (every visible entry)
+    int k, m;
+    const void *kwin;
+    int64_t win_rows;
+    const int64_t *win_pos0;
+    int n_win;
+    const int64_t *q_pos;
+    const float *sink;
+    int B;
+    int64_t n_q;
+    int h;
+    float scale;
+    void *out;
+    float *lse;
+    void *ws;
+    size_t ws_bytes;
+};
+cudaError_t launch_attend(const AttendArgs &a, unsigned *err, cudaStream_t s);
+size_t attend_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys);
+
+}  // namespace csa

@@ -1,0 +1,216 @@
+"""Device-resident steps of the hot path, built on the C ABI.
+
+``CsaPrefill``, ``HcaPrefill`` and ``Decode`` hold one workload's operands and
+outputs in device memory and run one pass of the path per ``step()``:
+
+* CSA prefill: compress KV entries -> compress indexer keys -> indexer scores
+  -> top-k -> sparse shared-KV attention (window + sink);
+* HCA prefill: compress (m' = 128, no overlap) -> dense shared-KV attention;
+* decode: indexer scores -> top-k -> sparse attention, and HCA dense
+  attention, for a batch of single-token queries over long caches.
+
+Only buffer management and argument marshalling live here; every step runs
+in ``libcsa.so``. The raw window KV of a prefill is the pre-compression KV
+(C^a for CSA, C for HCA).
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional
+
+import torch
+
+from . import abi
+from .abi import Entries
+
+DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def _dev(ops: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tensor]:
+    return {k: v.to(device, non_blocking=False).contiguous() for k, v in ops.items()}
+
+
+class CsaPrefill:
+    """One causal CSA prefill of a single sequence (batch 1)."""
+
+    launches_per_step = 5
+    kind = "csa"
+
+    def __init__(self, w, ops: Dict[str, torch.Tensor], device="cuda"):
+        self.w = w
+        d = self.d = _dev(ops, device)
+        n, c, E = w.n, w.c, w.E
+        self.q_pos = torch.arange(n, device=device, dtype=torch.int64)
+        self.win_pos0 = torch.zeros(1, device=device, dtype=torch.int64)
+        self.entries = Entries(torch.empty(E, c, device=device, dtype=DT[w.dtype]), c)
+        if w.idx_dtype == "e4m3":
+            self.kI = Entries(torch.empty(E, w.cI, device=device, dtype=torch.float8_e4m3fn),
+                              w.cI, scale=torch.empty(E, device=device, dtype=torch.float32),
+                              scale_group=w.cI)
+        else:
+            self.kI = Entries(torch.empty(E, w.cI, device=device, dtype=DT[w.idx_dtype]), w.cI)
+        self.scores = torch.empty(1, n, E, device=device, dtype=torch.float32)
+        self.idx = torch.empty(n, w.k, device=device, dtype=torch.int32)
+        self.out = torch.empty(1, n, w.h, c, device=device, dtype=DT[w.dtype])
+        self.lse = torch.empty(1, n, w.h, device=device, dtype=torch.float32)
+        self.scale = 1.0 / math.sqrt(c)
+
+    def compress_kv(self, stream=None):
+        d, w = self.d, self.w
+        abi.csa_compress_kv(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"], w.m, True,
+                            self.entries, stream)
+
+    def compress_index(self, stream=None):
+        d, w = self.d, self.w
+        abi.csa_compress_kv(d["CIa"], d["CIb"], d["ZIa"], d["ZIb"], d["BIa"], d["BIb"], w.m,
+                            True, self.kI, stream)
+
+    def index(self, stream=None):
+        d, w = self.d, self.w
+        qs = d.get("qI_scale")
+        abi.csa_indexer_scores(d["qI"][None], qs[None] if qs is not None else None,
+                               d["wI"][None], self.kI, self.q_pos[None], w.m, self.scores,
+                               w.E, stream)
+
+    def select(self, stream=None):
+        w = self.w
+        abi.csa_topk(self.scores[0], self.q_pos, w.m, w.k, self.idx, w.E, stream=stream)
+
+    def attend(self, stream=None):
+        d, w = self.d, self.w
+        abi.csa_sparse_mqa(d["q"][None], self.entries, w.E, w.m, self.idx, w.k, d["Ca"][None],
+                           self.win_pos0, w.n_win, self.q_pos[None], d["sink"], self.scale,
+                           self.out, self.lse, stream=stream)
+
+    def phases(self):
+        """The kernels of one step, in order: (name, launch)."""
+        return [("compress_kv", self.compress_kv), ("compress_index", self.compress_index),
+                ("indexer", self.index), ("topk", self.select), ("attend", self.attend)]
+
+    def inputs(self):
+        """Device operands a step reads (copied from the host in end-to-end runs)."""
+        return {k: v for k, v in self.d.items()}
+
+    def result(self):
+        return self.out
+
+    def step(self, stream=None):
+        for _, f in self.phases():
+            f(stream)
+
+
+class HcaPrefill:
+    """One causal HCA prefill of a single sequence (batch 1)."""
+
+    launches_per_step = 2
+    kind = "hca"
+
+    def __init__(self, w, ops: Dict[str, torch.Tensor], device="cuda"):
+        self.w = w
+        self.d = _dev(ops, device)
+        n, c, E = w.n, w.c, w.E
+        self.q_pos = torch.arange(n, device=device, dtype=torch.int64)
+        self.win_pos0 = torch.zeros(1, device=device, dtype=torch.int64)
+        self.entries = Entries(torch.empty(E, c, device=device, dtype=DT[w.dtype]), c)
+        self.out = torch.empty(1, n, w.h, c, device=device, dtype=DT[w.dtype])
+        self.lse = torch.empty(1, n, w.h, device=device, dtype=torch.float32)
+        self.scale = 1.0 / math.sqrt(c)
+
+    def compress(self, stream=None):
+        d, w = self.d, self.w
+        abi.csa_compress_kv(d["C"], None, d["Z"], None, d["B"], None, w.m, False,
+                            self.entries, stream)
+
+    def attend(self, stream=None):
+        d, w = self.d, self.w
+        abi.hca_dense_mqa(d["q"][None], self.entries, w.E, w.m, d["C"][None], self.win_pos0,
+                          w.n_win, self.q_pos[None], d["sink"], self.scale, self.out, self.lse,
+                          stream=stream)
+
+    def phases(self):
+        return [("compress_kv", self.compress), ("attend", self.attend)]
+
+    def inputs(self):
+        return {k: v for k, v in self.d.items()}
+
+    def result(self):
+        return self.out
+
+    def step(self, stream=None):
+        for _, f in self.phases():
+            f(stream)
+
+
+class Decode:
+    """One batched decode step over long CSA and HCA caches."""
+
+    launches_per_step = 4
+    kind = "decode"
+
+    def __init__(self, w, ops: Dict[str, torch.Tensor], device="cuda"):
+        self.w = w
+        d = self.d = _dev(ops, device)
+        B = w.batch
+        self.E = d["kI"].shape[1]
+        self.E_hca = d["hca_nope"].shape[1]
+        self.kI = Entries(d["kI"].view(B * self.E, w.cI), w.cI,
+                          scale=d["kI_scale"].view(B * self.E), scale_group=w.cI)
+        self.kv = Entries(d["kv_nope"].view(B * self.E, -1), w.c,
+                          scale=d["kv_scale"].view(B * self.E, -1),
+                          rope=d["kv_rope"].view(B * self.E, -1), rope_dims=w.rope_dims,
+                          scale_group=w.scale_group)
+        self.hkv = Entries(d["hca_nope"].view(B * self.E_hca, -1), w.c,
+                           scale=d["hca_scale"].view(B * self.E_hca, -1),
+                           rope=d["hca_rope"].view(B * self.E_hca, -1), rope_dims=w.rope_dims,
+                           scale_group=w.scale_group)
+        self.scores = torch.empty(B, 1, self.E, device=device, dtype=torch.float32)
+        self.idx = torch.empty(B, w.k, device=device, dtype=torch.int32)
+        self.out = torch.empty(B, 1, w.h, w.c, device=device, dtype=torch.bfloat16)
+        self.lse = torch.empty(B, 1, w.h, device=device, dtype=torch.float32)
+        self.hout = torch.empty_like(self.out)
+        self.hlse = torch.empty_like(self.lse)
+        self.scale = 1.0 / math.sqrt(w.c)
+        maxk = w.k + w.n_win
+        self.ws = self._workspace(B, w, maxk, device)
+        self.hws = self._workspace(B, w, self.E_hca + w.n_win, device)
+
+    @staticmethod
+    def _workspace(B, w, keys, device) -> Optional[torch.Tensor]:
+        n = abi.csa_mqa_workspace_size(B, 1, w.h, w.c, keys)
+        return torch.empty(max(n, 1), device=device, dtype=torch.uint8) if n else None
+
+    def index(self, stream=None):
+        d, w = self.d, self.w
+        abi.csa_indexer_scores(d["qI"], d["qI_scale"], d["wI"], self.kI, d["q_pos"], w.m,
+                               self.scores, self.E, stream)
+
+    def select(self, stream=None):
+        w = self.w
+        abi.csa_topk(self.scores.view(w.batch, self.E), self.d["q_pos"].view(-1), w.m, w.k,
+                     self.idx, self.E, stream=stream)
+
+    def attend(self, stream=None):
+        d, w = self.d, self.w
+        abi.csa_sparse_mqa(d["q"], self.kv, self.E, w.m, self.idx, w.k, d["kwin"],
+                           d["win_pos0"], w.n_win, d["q_pos"], d["sink"], self.scale,
+                           self.out, self.lse, workspace=self.ws, stream=stream)
+
+    def attend_hca(self, stream=None):
+        d, w = self.d, self.w
+        abi.hca_dense_mqa(d["q"], self.hkv, self.E_hca, w.m_hca, d["kwin"], d["win_pos0"],
+                          w.n_win, d["q_pos"], d["sink"], self.scale, self.hout, self.hlse,
+                          workspace=self.hws, stream=stream)
+
+    def phases(self):
+        return [("indexer", self.index), ("topk", self.select), ("attend", self.attend),
+                ("attend_hca", self.attend_hca)]
+
+    def inputs(self):
+        return {k: v for k, v in self.d.items()}
+
+    def result(self):
+        return self.out
+
+    def step(self, stream=None):
+        for _, f in self.phases():
+            f(stream)
