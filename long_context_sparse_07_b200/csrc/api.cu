@@ -207,7 +207,8 @@ size_t csa_mqa_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys
 }
 
 static csa_status attend_common(const char *w, const void *q, csa_dtype q_dt, csa_entries kv,
-                                int64_t E, const int32_t *idx, int k, int m, const void *kwin,
+                                int64_t E, int dense, const int32_t *idx, int k, int m,
+                                const void *kwin,
                                 int64_t win_rows, const int64_t *win_pos0, int n_win,
                                 const int64_t *q_pos, const float *sink, int B, int64_t n_q,
                                 int h, float scale, void *out, float *lse, void *workspace,
@@ -236,14 +237,14 @@ static csa_status attend_common(const char *w, const void *q, csa_dtype q_dt, cs
             "%s: a window needs a 16-byte aligned kwin with win_rows >= 1", w);
     REQUIRE(aligned16(q) && aligned16(out), CSA_ERR_INVALID_ARG,
             "%s: q and out must be 16-byte aligned", w);
-    const size_t need = csa::attend_workspace_size(B, n_q, h, c, (idx ? k : E) + n_win);
+    const size_t need = csa::attend_workspace_size(B, n_q, h, c, (dense ? E : k) + n_win);
     REQUIRE(ws_bytes >= need && (need == 0 || workspace), CSA_ERR_INVALID_ARG,
             "%s: workspace of %zu bytes required", w, need);
     unsigned *err = err_word();
     REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
     if ((int64_t)B * n_q == 0)
         return CSA_OK;
-    csa::AttendArgs a{q, q_dt, kv, E, idx, k, m, kwin, n_win > 0 ? win_rows : 0, win_pos0,
+    csa::AttendArgs a{q, q_dt, kv, E, idx, dense, k, m, kwin, n_win > 0 ? win_rows : 0, win_pos0,
                       n_win, q_pos, sink, B, n_q, h, scale, out, lse, workspace, ws_bytes};
     return launched(csa::launch_attend(a, err, (cudaStream_t)stream), w);
 }
@@ -255,7 +256,7 @@ csa_status csa_sparse_mqa(const void *q, csa_dtype q_dt, csa_entries kv, int64_t
                           void *out, float *lse, void *workspace, size_t ws_bytes,
                           void *stream)
 {
-    return attend_common("csa_sparse_mqa", q, q_dt, kv, E, idx, k, m, kwin, win_rows,
+    return attend_common("csa_sparse_mqa", q, q_dt, kv, E, 0, idx, k, m, kwin, win_rows,
                          win_pos0, n_win, q_pos, sink, B, n_q, h, scale, out, lse, workspace,
                          ws_bytes, stream);
 }
@@ -266,7 +267,7 @@ csa_status hca_dense_mqa(const void *q, csa_dtype q_dt, csa_entries kv, int64_t 
                          int64_t n_q, int h, float scale, void *out, float *lse,
                          void *workspace, size_t ws_bytes, void *stream)
 {
-    return attend_common("hca_dense_mqa", q, q_dt, kv, E, nullptr, 0, m, kwin, win_rows,
+    return attend_common("hca_dense_mqa", q, q_dt, kv, E, 1, nullptr, 0, m, kwin, win_rows,
                          win_pos0, n_win, q_pos, sink, B, n_q, h, scale, out, lse, workspace,
                          ws_bytes, stream);
 }

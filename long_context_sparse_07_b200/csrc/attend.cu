@@ -31,6 +31,7 @@ struct Dev {
     csa_dtype kv_dt;
     int64_t E;
     const int32_t *idx;
+    int dense;
     int k, m;
     const void *kwin;
     int64_t win_rows;
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(Dev d)
     const int h0 = blockIdx.y * HG;
     const int64_t t = d.q_pos[bt];
     const int64_t V = visible(t, d.m, d.E);
-    const int64_t nsel = d.idx ? d.k : V;
+    const int64_t nsel = d.dense ? V : d.k;
     const int64_t w0 = t - d.n_win + 1 < 0 ? 0 : t - d.n_win + 1;
     const int64_t nwin = d.n_win > 0 ? t - w0 + 1 : 0;
     const int64_t NK = nsel + nwin;
@@ -111,7 +112,7 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(Dev d)
             int src = 0;
             if (j < NK) {
                 if (j < nsel) {
-                    const int64_t s = d.idx ? (int64_t)d.idx[bt * d.k + j] : j;
+                    const int64_t s = d.dense ? j : (int64_t)d.idx[bt * d.k + j];
                     if (s >= 0) {
                         if (s < V)
                             r = b * d.E + s;
@@ -260,6 +261,7 @@ cudaError_t launch_attend(const AttendArgs &a, unsigned *err, cudaStream_t s)
     d.group = a.kv.dt == CSA_E4M3 ? a.kv.scale_group : 1;
     d.E = a.E;
     d.idx = a.idx;
+    d.dense = a.dense;
     d.k = a.k;
     d.m = a.m;
     d.kwin = a.kwin;

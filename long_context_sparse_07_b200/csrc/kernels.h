@@ -46,7 +46,8 @@ struct AttendArgs {
     csa_dtype q_dt;
     csa_entries kv;
     int64_t E;
-    const int32_t *idx;   // NULL = dense (every visible entry)
+    const int32_t *idx;   // selection lists [B * n_q, k] (sparse only)
+    int dense;            // 1: every visible entry is a key (HCA); 0: idx lists them
     int k, m;
     const void *kwin;
     int64_t win_rows;

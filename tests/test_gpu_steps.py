@@ -58,9 +58,10 @@ def test_compress_plain(name, n, c, m, overlap, dtype):
     abi.csa_get_error()
     assert_close_out(to_np(out), ref, dtype, name)
     if dtype == "bf16":
-        # storage rounding is the only difference: at most one bf16 ulp
+        # storage rounding is the main difference: at most one bf16 ulp, plus
+        # the float32 accumulation error (absolute: results near zero cancel)
         refb = torch.from_numpy(ref).float().to(torch.bfloat16).float().numpy()
-        ulp = np.abs(refb) * 2.0 ** -7 + 1e-30
+        ulp = np.abs(refb) * 2.0 ** -7 + 4e-6
         assert (np.abs(to_np(out) - refb) <= ulp).all()
 
 
