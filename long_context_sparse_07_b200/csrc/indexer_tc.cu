@@ -1,14 +1,342 @@
-// indexer_tc.cu -- tensor-core (tcgen05) path of the lightning indexer.
+// indexer_tc.cu -- lightning-indexer scores (Eq. 16) on the 5th-generation
+// tensor cores (tcgen05 + TMEM), fed by TMA.
+//
+// The contraction q^I . k^I is the one dense GEMM of the path. Operands are
+// swapped so that each TMEM lane holds one compressed key: the MMA computes
+//   D[key][(token, head)] = sum_x kI[key][x] * qI[token][head][x]
+// with M = 128 keys (A, streamed), N = NT tokens x HI heads (B, resident),
+// K = c_I (bf16: kind::f16, 16 per MMA; e4m3: kind::f8f6f4, 32 per MMA).
+// The epilogue thread that owns a key lane then reduces over heads inside
+// its registers: I[t][s] = kscale[s] * sum_h w'[t][h] * ReLU(D[s][(t, h)]),
+// with w' = wI * qI_scale (scales are positive, so they commute with ReLU).
+//
+// Warp roles (192 threads): warp 0 issues TMA loads (query tile once, then a
+// ring of key-tile stages), warp 1 owns TMEM and issues the MMAs into two
+// accumulator buffers, warps 2-5 drain the accumulators (one lane quarter
+// each) and write score rows, overlapping the next tile's MMAs. Key tiles
+// past the causal bound of every token of the tile are never loaded; score
+// entries s >= V_t are not written. Every wait is bounded; on expiry the
+// block records CSA_ERR_TIMEOUT, drains its own copies and returns.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
+#include "tma_host.h"
 
 namespace csa {
 
+namespace {
+
+struct TcArgs {
+    const float *wI, *qI_scale, *kI_scale;
+    const int64_t *q_pos;
+    int64_t n_q, E;
+    int m, kb;            // kb: 128-byte blocks per row of c_I
+    int nchunks;
+    int64_t key_chunk;
+    float *scores;
+    int64_t ld;
+    unsigned *err;
+};
+
+constexpr int kThreads = 192;
+
+template <bool FP8, int HI, int NT>
+struct Cfg {
+    static constexpr int N = NT * HI;
+    static constexpr int STAGES = FP8 ? 6 : 4;
+    static constexpr int TMEM_COLS = (2 * N) < 32 ? 32 : 2 * N;
+    static constexpr uint32_t IDESC = FP8 ? tc::idesc_e4m3(128, N) : tc::idesc_bf16(128, N);
+    static size_t smem_bytes(int kb)
+    {
+        return 1024 + (size_t)kb * N * 128 + (size_t)STAGES * kb * 16384 + 256 + N * 4 + NT * 8;
+    }
+};
+
+template <bool FP8, int HI, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmq,
+                  const TcArgs a)
+{
+    using C = Cfg<FP8, HI, NT>;
+    constexpr int N = C::N;
+    constexpr int S = C::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int KB = a.kb;
+    uint8_t *sB = smem;
+    uint8_t *sA = sB + (size_t)KB * N * 128;
+    uint64_t *bars = (uint64_t *)(sA + (size_t)S * KB * 16384);
+    uint64_t *full = bars, *empty = bars + S, *bfull = bars + 2 * S;
+    uint64_t *accf = bfull + 1, *acce = accf + 2, *done = acce + 2;
+    uint32_t *tmem_slot = (uint32_t *)(done + 1);
+    int *abort_flag = (int *)(tmem_slot + 1);
+    float *wsm = (float *)(bars + 32);
+    int64_t *vt = (int64_t *)(wsm + N);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.y;
+    const int64_t tile = blockIdx.x / a.nchunks;
+    const int chunk = blockIdx.x % a.nchunks;
+    const int64_t t0 = tile * NT;
+
+    if (threadIdx.x < NT) {
+        const int64_t t = t0 + threadIdx.x;
+        vt[threadIdx.x] = t < a.n_q ? visible(a.q_pos[(int64_t)b * a.n_q + t], a.m, a.E) : 0;
+    }
+    if (threadIdx.x == 0)
+        *abort_flag = 0;
+    __syncthreads();
+    int64_t vmax = 0;
+#pragma unroll
+    for (int tt = 0; tt < NT; tt++)
+        vmax = vt[tt] > vmax ? vt[tt] : vmax;
+    const int64_t s_begin = (int64_t)chunk * a.key_chunk;
+    int64_t s_end = s_begin + a.key_chunk;
+    if (s_end > vmax)
+        s_end = vmax;
+    if (s_end <= s_begin)
+        return;                                   // uniform: nothing visible here
+    const int ntiles = (int)((s_end - s_begin + 127) / 128);
+
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < S; i++) {
+            tc::mbar_init(&full[i], 1);
+            tc::mbar_init(&empty[i], 1);
+        }
+        tc::mbar_init(bfull, 1);
+        for (int i = 0; i < 2; i++) {
+            tc::mbar_init(&accf[i], 1);
+            tc::mbar_init(&acce[i], 4);
+        }
+        tc::mbar_init(done, 1);
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&tmk);
+        tc::tma_prefetch_desc(&tmq);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    if (warp >= 2) {
+        for (int col = threadIdx.x - 64; col < N; col += 128) {
+            const int tt = col / HI, hh = col % HI;
+            const int64_t t = t0 + tt;
+            float wv = 0.f;
+            if (t < a.n_q) {
+                const int64_t r = ((int64_t)b * a.n_q + t) * HI + hh;
+                wv = a.wI[r];
+                if (FP8)
+                    wv *= a.qI_scale[r];
+            }
+            wsm[col] = wv;
+        }
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- producer
+            const int xstep = FP8 ? 128 : 64;    // elements per 128-byte block
+            int issued = 0;
+            bool ok = true;
+            tc::mbar_arrive_expect_tx(bfull, (uint32_t)(KB * N * 128));
+            for (int kb = 0; kb < KB; kb++)
+                tc::tma_load_2d(sB + (size_t)kb * N * 128, &tmq, bfull, kb * xstep,
+                                (int)(((int64_t)b * a.n_q + t0) * HI));
+            for (int i = 0; i < ntiles && ok; i++) {
+                const int st = i % S;
+                if (i >= S && !tc::mbar_wait(&empty[st], ((i / S) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::mbar_arrive_expect_tx(&full[st], (uint32_t)(KB * 16384));
+                for (int kb = 0; kb < KB; kb++)
+                    tc::tma_load_2d(sA + (size_t)(st * KB + kb) * 16384, &tmk, &full[st],
+                                    kb * xstep, (int)((int64_t)b * a.E + s_begin + (int64_t)i * 128));
+                issued = i + 1;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report(a.err, CSA_ERR_TIMEOUT, K_INDEXER_TC, blockIdx.x, 0);
+                // let the copies already in flight land before the block exits
+                volatile int never = 0;
+                static_cast<void>(tc::mbar_wait(bfull, 0, &never, 200000000ull));
+                for (int i = issued - S < 0 ? 0 : issued - S; i < issued; i++)
+                    static_cast<void>(tc::mbar_wait(&full[i % S], (i / S) & 1, &never, 200000000ull));
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            bool ok = tc::mbar_wait(bfull, 0, abort_flag);
+            const uint32_t sBa = tc::smem_u32(sB);
+            for (int i = 0; i < ntiles && ok; i++) {
+                const int st = i % S, buf = i & 1;
+                if (i >= 2 && !tc::mbar_wait(&acce[buf], ((i / 2) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (!tc::mbar_wait(&full[st], (i / S) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after();
+                const uint32_t d = tmem + (uint32_t)(buf * N);
+                const uint32_t sAa = tc::smem_u32(sA + (size_t)st * KB * 16384);
+#pragma unroll 1
+                for (int kb = 0; kb < KB; kb++) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; kk++) {
+                        const uint64_t ad = tc::sdesc_sw128(sAa + kb * 16384 + kk * 32);
+                        const uint64_t bd = tc::sdesc_sw128(sBa + kb * N * 128 + kk * 32);
+                        if (FP8)
+                            tc::mma_f8(d, ad, bd, C::IDESC, (kb | kk) != 0);
+                        else
+                            tc::mma_f16(d, ad, bd, C::IDESC, (kb | kk) != 0);
+                    }
+                }
+                tc::mma_commit(&empty[st]);
+                tc::mma_commit(&accf[buf]);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report(a.err, CSA_ERR_TIMEOUT, K_INDEXER_TC, blockIdx.x, 1);
+            }
+            // every MMA issued above has completed once `done` flips
+            tc::mma_commit(done);
+            volatile int never = 0;
+            static_cast<void>(tc::mbar_wait(done, 0, &never, 200000000ull));
+        }
+    } else {
+        // ---------------- epilogue: warps 2..5, lane quarter = warp % 4
+        const int q4 = warp & 3;
+        const int row = q4 * 32 + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+        for (int i = 0; i < ntiles; i++) {
+            const int buf = i & 1;
+            if (!tc::mbar_wait(&accf[buf], (i / 2) & 1, abort_flag)) {
+                *abort_flag = 1;
+                report(a.err, CSA_ERR_TIMEOUT, K_INDEXER_TC, blockIdx.x, 2);
+                break;
+            }
+            tc::fence_after();
+            const int64_t s = s_begin + (int64_t)i * 128 + row;
+            float ks = 1.f;
+            if (FP8)
+                ks = s < a.E ? a.kI_scale[(int64_t)b * a.E + s] : 0.f;
+            const uint32_t base = lane_addr + (uint32_t)(buf * N);
+#pragma unroll
+            for (int tt = 0; tt < NT; tt++) {
+                float sacc = 0.f;
+                if constexpr (HI >= 32) {
+#pragma unroll
+                    for (int cc = 0; cc < HI / 32; cc++) {
+                        uint32_t r[32];
+                        tc::tmem_ld32(base + (uint32_t)(tt * HI + cc * 32), r);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; j++)
+                            sacc += wsm[tt * HI + cc * 32 + j] * fmaxf(__uint_as_float(r[j]), 0.f);
+                    }
+                } else {
+                    uint32_t r[16];
+                    tc::tmem_ld16(base + (uint32_t)(tt * HI), r);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 16; j++)
+                        sacc += wsm[tt * HI + j] * fmaxf(__uint_as_float(r[j]), 0.f);
+                }
+                const int64_t t = t0 + tt;
+                if (t < a.n_q && s < vt[tt])
+                    a.scores[((int64_t)b * a.n_q + t) * a.ld + s] = sacc * ks;
+            }
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0)
+                tc::mbar_arrive(&acce[buf]);
+        }
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after();
+        tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <bool FP8, int HI, int NT>
+cudaError_t launch_one(const IndexerArgs &a, unsigned *err, cudaStream_t s)
+{
+    using C = Cfg<FP8, HI, NT>;
+    const int esize = FP8 ? 1 : 2;
+    CUtensorMap tmk, tmq;
+    const CUtensorMapDataType dt =
+        FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_tmap_2d(&tmk, a.kI.body, dt, esize, (uint64_t)a.B * a.E, a.cI, 128) ||
+        !make_tmap_2d(&tmq, a.qI, dt, esize, (uint64_t)a.B * a.n_q * HI, a.cI, C::N))
+        return cudaErrorInvalidValue;
+    TcArgs t;
+    t.wI = a.wI;
+    t.qI_scale = a.qI_scale;
+    t.kI_scale = a.kI.scale;
+    t.q_pos = a.q_pos;
+    t.n_q = a.n_q;
+    t.E = a.E;
+    t.m = a.m;
+    t.kb = a.cI * esize / 128;
+    const int64_t ttiles = (a.n_q + NT - 1) / NT;
+    // few token tiles: split the keys of each tile over several blocks
+    t.key_chunk = a.E;
+    t.nchunks = 1;
+    if (ttiles * a.B < 296) {
+        t.key_chunk = 2048;
+        t.nchunks = (int)((a.E + t.key_chunk - 1) / t.key_chunk);
+    }
+    t.scores = a.scores;
+    t.ld = a.ld;
+    t.err = err;
+    const size_t smem = C::smem_bytes(t.kb);
+    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<FP8, HI, NT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    dim3 grid((unsigned)(ttiles * t.nchunks), (unsigned)a.B);
+    indexer_tc_kernel<FP8, HI, NT><<<grid, kThreads, smem, s>>>(tmk, tmq, t);
+    return cudaGetLastError();
+}
+
+template <bool FP8>
+cudaError_t dispatch_heads(const IndexerArgs &a, unsigned *err, cudaStream_t s, bool few)
+{
+    switch (a.hI) {
+    case 16: return few ? launch_one<FP8, 16, 1>(a, err, s) : launch_one<FP8, 16, 16>(a, err, s);
+    case 32: return few ? launch_one<FP8, 32, 1>(a, err, s) : launch_one<FP8, 32, 8>(a, err, s);
+    case 64: return few ? launch_one<FP8, 64, 1>(a, err, s) : launch_one<FP8, 64, 4>(a, err, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
 cudaError_t launch_indexer_tc(const IndexerArgs &a, unsigned *err, cudaStream_t s, bool *taken)
 {
-    (void)a; (void)err; (void)s;
     *taken = false;
-    return cudaSuccess;
+    if (a.dt == CSA_F32)
+        return cudaSuccess;
+    if (a.hI != 16 && a.hI != 32 && a.hI != 64)
+        return cudaSuccess;
+    const int esize = a.dt == CSA_E4M3 ? 1 : 2;
+    if ((a.cI * esize) % 128 != 0 || a.cI * esize > 256)
+        return cudaSuccess;
+    if (((uintptr_t)a.qI & 15) || ((uintptr_t)a.kI.body & 15))
+        return cudaSuccess;
+    *taken = true;
+    const bool few = a.n_q <= 8;
+    return a.dt == CSA_E4M3 ? dispatch_heads<true>(a, err, s, few)
+                            : dispatch_heads<false>(a, err, s, few);
 }
 
 }  // namespace csa
