@@ -5,43 +5,53 @@
 // value. Keys therefore go on the M axis of both contractions:
 //   S^T[key][head]  = sum_d K[key][d] * Q[head][d]        (M = 128 keys, N = H)
 //   O^T[dim][head] += sum_key K[key][dim] * P^T[key][head] (M = 4 x 128 dims, N = H)
-// so one 128 x 512 bf16 key tile staged in shared memory (128-byte swizzled,
-// gathered row by row with cp.async from the selection list or the window)
-// serves as the K-major A operand of the first product and, read along the
-// other axis, as the M/N-major A operand of the second. S^T and O^T live in
+// One 128 x 512 bf16 key tile in shared memory (8 blocks of 64 dims, 128-byte
+// swizzle) is the K-major A operand of the first product and, read along the
+// other axis, the M/N-major A operand of the second. S^T and O^T live in
 // tensor memory (H + 4H columns).
 //
-// Softmax: the thread that owns a key lane holds that key's logits for every
-// head. The per-head offset m_h is updated lazily: only when some logit of a
-// tile exceeds m_h + 8 are the tile's maxima reduced across the block, the O^T
-// accumulators rescaled in tensor memory and the partial sums rescaled; the
-// first tile of a query always takes that path. Probabilities are rounded to
-// bf16 for the second product and summed from the rounded values, so the
-// numerator and the denominator agree. The sink joins only the final
-// normalisation: out = O * e^{m-M} / (l * e^{m-M} + e^{z'-M}), M = max(m, z').
-//
-// One persistent block per SM loops over queries; four warps gather, run the
-// softmax and the epilogue, thread 0 issues the MMAs. Every wait is bounded.
+// Warp roles (one persistent block per SM looping over queries):
+//  * warps 0-3 gather the key rows of each tile (selected entries, or window
+//    rows) with 16-byte cp.async, block by block, keeping up to four 16 KB
+//    blocks in flight per thread; block pair (2j, 2j+1) of the next tile is
+//    refetched as soon as the O^T product of M-tile j has consumed it. One
+//    thread also loads each query's Q with a tiled TMA copy.
+//  * warp 4 allocates tensor memory and issues the MMAs (S^T block by block
+//    as blocks land, then O^T per M-tile), committing to the barriers the
+//    other roles wait on.
+//  * warps 5.. (four per group of 16 heads) own the TMEM lanes (one key, then
+//    one dim, per thread): softmax of each tile into P^T for their heads, and
+//    the normalisation and output of each query.
+// Softmax: the per-head offset m_h is updated lazily -- only when some logit
+// of a tile exceeds m_h + 8 are the tile's maxima of that head group reduced,
+// its O^T columns rescaled in tensor memory and its partial sums rescaled (the
+// first tile always takes this path). Probabilities are rounded to bf16 for
+// the second product and the normaliser sums the rounded values. The sink
+// joins the final normalisation only.
+// Every wait is bounded; on expiry the block records CSA_ERR_TIMEOUT, lets its
+// own copies and products land, frees its tensor memory and returns.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
+#include "tma_host.h"
 
 namespace csa {
 
 namespace {
 
-constexpr int kThreads = 128;
 constexpr int DIM = 512;
 constexpr int KT = 128;
 constexpr float kLazy = 8.f;
+constexpr int kMmaWarp = 4;
+constexpr int kSoftWarp0 = 5;
+constexpr int kGatherBar = 5;        // named barrier of the 4 gather warps (1..4: head groups)
+constexpr int kInFlight = 3;         // 16 KB blocks a gather thread may leave in flight
 
 struct TcAttn {
-    const __nv_bfloat16 *q;
-    const __nv_bfloat16 *ent;
+    const __nv_bfloat16 *ent, *kwin;
     const int32_t *idx;
     int dense, k, m;
     int64_t E;
-    const __nv_bfloat16 *kwin;
     int64_t win_rows;
     const int64_t *win_pos0;
     int n_win;
@@ -56,64 +66,73 @@ struct TcAttn {
 
 template <int H>
 struct Lay {
+    static constexpr int NG = H / 16;                               // head groups
+    static constexpr int THREADS = 32 * (kSoftWarp0 + 4 * NG);
     static constexpr size_t K_OFF = 0;                              // 8 x 16 KB
     static constexpr size_t Q_OFF = 8 * 16384;                      // 8 x H x 128
     static constexpr size_t P_OFF = Q_OFF + 8 * H * 128;            // 2 x H x 128
-    static constexpr size_t PTR_OFF = P_OFF + 2 * H * 128;          // 128 pointers
-    static constexpr size_t F_OFF = PTR_OFF + KT * 8;               // floats: m, red[4], alpha, fin, lsum
-    static constexpr size_t BAR_OFF = F_OFF + ((8 * H * 4 + 63) / 64) * 64;
-    static constexpr size_t TOTAL = BAR_OFF + 64;
+    static constexpr size_t PTR_OFF = P_OFF + 2 * H * 128;          // 128 row pointers
+    static constexpr size_t F_OFF = PTR_OFF + KT * 8;               // m, red[4], fin
+    static constexpr size_t BAR_OFF = F_OFF + ((6 * H * 4 + 63) / 64) * 64;
+    static constexpr size_t TOTAL = BAR_OFF + 256;
     static constexpr uint32_t TMEM_COLS = (5 * H <= 128) ? 128 : (5 * H <= 256 ? 256 : 512);
     static constexpr uint32_t IDESC_S = tc::idesc_bf16(128, H, 0, 0);
     static constexpr uint32_t IDESC_O = tc::idesc_bf16(128, H, 1, 0);
 };
 
-// Loads the H columns starting at `taddr` of this thread's TMEM lane.
-template <int H>
-__device__ __forceinline__ void load_cols(uint32_t taddr, float (&v)[H])
+// Per-query quantities, computed identically by every role.
+struct QInfo {
+    int64_t b, t, V, nsel, nwin, w0, wp0, nk;
+    int ntiles;
+};
+
+__device__ __forceinline__ QInfo query_info(const TcAttn &a, int64_t bt)
 {
-    if constexpr (H >= 32) {
-#pragma unroll
-        for (int c = 0; c < H / 32; c++) {
-            uint32_t r[32];
-            tc::tmem_ld32(taddr + c * 32, r);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; j++)
-                v[c * 32 + j] = __uint_as_float(r[j]);
-        }
-    } else {
-        uint32_t r[16];
-        tc::tmem_ld16(taddr, r);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; j++)
-            v[j] = __uint_as_float(r[j]);
-    }
+    QInfo q;
+    q.b = bt / a.n_q;
+    q.t = a.q_pos[bt];
+    q.V = visible(q.t, a.m, a.E);
+    q.nsel = a.dense ? q.V : a.k;
+    q.w0 = q.t - a.n_win + 1 < 0 ? 0 : q.t - a.n_win + 1;
+    q.nwin = a.n_win > 0 ? q.t - q.w0 + 1 : 0;
+    q.wp0 = a.win_pos0 ? a.win_pos0[q.b] : 0;
+    q.nk = q.nsel + q.nwin;
+    q.ntiles = (int)((q.nk + KT - 1) / KT);
+    return q;
 }
 
-// Multiplies the H columns starting at `taddr` of this thread's lane by
-// f[column], in place (16 columns at a time).
-template <int H>
-__device__ __forceinline__ void scale_cols(uint32_t taddr, const float *f)
+// Source row of key slot j of a query (NULL: empty slot or out of range).
+// `report_bad` records a selection index or window position out of range.
+__device__ __forceinline__ const __nv_bfloat16 *key_row(const TcAttn &a, const QInfo &q,
+                                                        int64_t bt, int64_t j, bool report_bad)
 {
-#pragma unroll 1
-    for (int c = 0; c < H / 16; c++) {
-        uint32_t r[16];
-        tc::tmem_ld16(taddr + c * 16, r);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; j++)
-            r[j] = __float_as_uint(__uint_as_float(r[j]) * f[c * 16 + j]);
-        tc::tmem_st16(taddr + c * 16, r);
+    if (j < q.nsel) {
+        const int64_t s = a.dense ? j : (int64_t)a.idx[bt * a.k + j];
+        if (s < 0)
+            return nullptr;
+        if (s < q.V)
+            return a.ent + (q.b * a.E + s) * DIM;
+        if (report_bad)
+            report(a.err, CSA_ERR_BOUNDS, K_ATTEND_TC, (unsigned)bt, (unsigned)s);
+        return nullptr;
     }
-    tc::tmem_st_wait();
+    if (j < q.nk) {
+        const int64_t p = q.w0 + (j - q.nsel);
+        const int64_t wr = p - q.wp0;
+        if (wr >= 0 && wr < a.win_rows)
+            return a.kwin + (q.b * a.win_rows + wr) * DIM;
+        if (report_bad)
+            report(a.err, CSA_ERR_BOUNDS, K_ATTEND_TC, (unsigned)bt, (unsigned)p);
+    }
+    return nullptr;
 }
 
 template <int H>
-__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const TcAttn a)
+__global__ void __launch_bounds__(Lay<H>::THREADS, 1)
+attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
 {
     using L = Lay<H>;
+    constexpr int NG = L::NG;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *sK = sm + L::K_OFF;
@@ -122,22 +141,33 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const TcAttn a)
     const __nv_bfloat16 **kptr = (const __nv_bfloat16 **)(sm + L::PTR_OFF);
     float *m_run = (float *)(sm + L::F_OFF);     // [H]
     float *red = m_run + H;                      // [4][H]
-    float *alpha = red + 4 * H;                  // [H]
-    float *fin = alpha + H;                      // [H]
+    float *fin = red + 4 * H;                    // [H]
     uint64_t *bars = (uint64_t *)(sm + L::BAR_OFF);
-    uint64_t *sbar = bars, *obar = bars + 1, *done = bars + 2;
-    uint32_t *tmem_slot = (uint32_t *)(bars + 3);
+    uint64_t *kfull = bars;          // [8] key block landed (128 gather arrivals)
+    uint64_t *kfree = bars + 8;      // [4] block pair consumed by O^T M-tile j
+    uint64_t *qfull = bars + 12, *qfree = bars + 13, *sfull = bars + 14, *pfull = bars + 15;
+    uint64_t *ofull = bars + 16, *ofree = bars + 17, *done = bars + 18;
+    uint32_t *tmem_slot = (uint32_t *)(bars + 19);
     int *abort_flag = (int *)(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        tc::mbar_init(sbar, 1);
-        tc::mbar_init(obar, 1);
+        for (int i = 0; i < 8; i++)
+            tc::mbar_init(&kfull[i], 128);
+        for (int i = 0; i < 4; i++)
+            tc::mbar_init(&kfree[i], 1);
+        tc::mbar_init(qfull, 1);
+        tc::mbar_init(qfree, 1);
+        tc::mbar_init(sfull, 1);
+        tc::mbar_init(pfull, 128 * NG);
+        tc::mbar_init(ofull, 1);
+        tc::mbar_init(ofree, 128 * NG);
         tc::mbar_init(done, 1);
         tc::fence_mbar_init();
         *abort_flag = 0;
+        tc::tma_prefetch_desc(&tm_q);
     }
-    if (warp == 0) {
+    if (warp == kMmaWarp) {
         tc::tmem_alloc(tmem_slot, L::TMEM_COLS);
         tc::tmem_relinquish();
     }
@@ -145,261 +175,320 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const TcAttn a)
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_tm = tmem + ((uint32_t)(warp * 32) << 16);
-    const uint32_t sK_a = tc::smem_u32(sK), sQ_a = tc::smem_u32(sQ), sP_a = tc::smem_u32(sP);
+    volatile int *abortv = abort_flag;
 
-    uint32_t g = 0;                     // tiles issued by this block (barrier phases)
-    bool ok = true;
-
-    for (int64_t bt = blockIdx.x; bt < a.nqueries && ok; bt += gridDim.x) {
-        const int64_t b = bt / a.n_q;
-        const int64_t t = a.q_pos[bt];
-        const int64_t V = visible(t, a.m, a.E);
-        const int64_t nsel = a.dense ? V : a.k;
-        const int64_t w0 = t - a.n_win + 1 < 0 ? 0 : t - a.n_win + 1;
-        const int64_t nwin = a.n_win > 0 ? t - w0 + 1 : 0;
-        const int64_t NK = nsel + nwin;
-        const int64_t wp0 = a.win_pos0 ? a.win_pos0[b] : 0;
-        const int ntiles = (int)((NK + KT - 1) / KT);
-
-        // queries of this token -> sQ (K-major, 128-byte swizzle, 8 blocks of 64 dims)
-        for (int ch = tid; ch < H * 64; ch += kThreads) {
-            const int hh = ch >> 6, c16 = ch & 63;
-            uint8_t *dst = sQ + (c16 >> 3) * (H * 128) + hh * 128 + (((c16 & 7) ^ (hh & 7)) << 4);
-            tc::cp_async16(dst, a.q + (bt * H + hh) * DIM + c16 * 8, 16);
-        }
-        for (int hh = tid; hh < H; hh += kThreads)
-            m_run[hh] = -INFINITY;
-        float lpart[H];
-#pragma unroll
-        for (int hh = 0; hh < H; hh++)
-            lpart[hh] = 0.f;
-
-        for (int it = 0; it < ntiles; ++it, ++g) {
-            // the previous tile's products must be done with sK / sP; every
-            // thread takes the same decision, so a timeout never splits the block
-            const bool prev_done = g == 0 || tc::mbar_wait(obar, (g - 1) & 1, abort_flag);
-            if (!__syncthreads_and(prev_done)) {
+    if (warp < 4) {
+        // ------------------------------------------------------------ gather
+        const int gt = tid;                          // 0..127
+        const void *zero_src = a.E > 0 ? (const void *)a.ent : (const void *)a.kwin;
+        uint32_t tctr = 0, qctr = 0, issued = 0, arrived = 0;
+        bool ok = true;
+        // announce every block still in flight: required before any wait on
+        // a barrier that the products of those blocks release
+        auto flush = [&]() {
+            tc::cp_async_wait_group<0>();
+            tc::fence_async_shared();
+            for (; arrived < issued; ++arrived)
+                tc::mbar_arrive(&kfull[arrived & 7]);
+        };
+        for (int64_t bt = blockIdx.x; bt < a.nqueries && ok; bt += gridDim.x, ++qctr) {
+            const QInfo q = query_info(a, bt);
+            flush();
+            const bool qf = qctr == 0 || tc::mbar_wait(qfree, (qctr - 1) & 1, abortv);
+            if (tc::named_bar_or(kGatherBar, 128, !qf)) {
                 ok = false;
                 break;
             }
-            const int64_t j = (int64_t)it * KT + tid;
-            const __nv_bfloat16 *src = nullptr;
-            if (j < NK) {
-                if (j < nsel) {
-                    const int64_t s = a.dense ? j : (int64_t)a.idx[bt * a.k + j];
-                    if (s >= 0) {
-                        if (s < V)
-                            src = a.ent + (b * a.E + s) * DIM;
-                        else
-                            report(a.err, CSA_ERR_BOUNDS, K_ATTEND_TC, (unsigned)bt, (unsigned)s);
-                    }
-                } else {
-                    const int64_t p = w0 + (j - nsel);
-                    const int64_t wr = p - wp0;
-                    if (wr >= 0 && wr < a.win_rows)
-                        src = a.kwin + (b * a.win_rows + wr) * DIM;
-                    else
-                        report(a.err, CSA_ERR_BOUNDS, K_ATTEND_TC, (unsigned)bt, (unsigned)p);
-                }
+            if (gt == 0) {
+                tc::mbar_arrive_expect_tx(qfull, (uint32_t)(H * 1024));
+                for (int kb = 0; kb < 8; kb++)
+                    tc::tma_load_2d(sQ + kb * (H * 128), &tm_q, qfull, kb * 64, (int)(bt * H));
             }
-            const bool valid = src != nullptr;
-            kptr[tid] = src;
-            __syncthreads();
-            // gather the 128 keys: rows of 64 16-byte chunks, coalesced per row
-#pragma unroll 4
-            for (int itc = 0; itc < 64; ++itc) {
-                const int lin = itc * kThreads + tid;
-                const int r = lin >> 6, c16 = lin & 63;
-                const __nv_bfloat16 *sp = kptr[r];
-                uint8_t *dst = sK + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
-                tc::cp_async16(dst, sp ? (const void *)(sp + c16 * 8) : (const void *)a.ent,
-                               sp ? 16u : 0u);
-            }
-            tc::cp_async_wait_all();
-            tc::fence_async_shared();
-            __syncthreads();
-
-            // S^T = K Q^T
-            if (tid == 0) {
-                tc::fence_after();
-#pragma unroll 1
+            for (int i = 0; i < q.ntiles && ok; ++i, ++tctr) {
+                flush();
+                kptr[gt] = key_row(a, q, bt, (int64_t)i * KT + gt, false);
+                tc::named_bar_sync(kGatherBar, 128);
                 for (int kb = 0; kb < 8; kb++) {
+                    if ((kb & 1) == 0 && tctr > 0) {
+                        const bool fr = tc::mbar_wait(&kfree[kb >> 1], (tctr - 1) & 1, abortv);
+                        if (tc::named_bar_or(kGatherBar, 128, !fr)) {
+                            ok = false;
+                            break;
+                        }
+                    }
 #pragma unroll
-                    for (int kk = 0; kk < 4; kk++) {
-                        const uint64_t ad = tc::sdesc_sw128(sK_a + kb * 16384 + kk * 32);
-                        const uint64_t bd = tc::sdesc_sw128(sQ_a + kb * (H * 128) + kk * 32);
-                        tc::mma_f16(tmem, ad, bd, L::IDESC_S, (kb | kk) != 0);
+                    for (int u = 0; u < 8; u++) {
+                        const int lin = u * 128 + gt;
+                        const int r = lin >> 3, c = lin & 7;
+                        const __nv_bfloat16 *sp = kptr[r];
+                        uint8_t *dst = sK + kb * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
+                        tc::cp_async16(dst, sp ? (const void *)(sp + kb * 64 + c * 8) : zero_src,
+                                       sp ? 16u : 0u);
+                    }
+                    tc::cp_async_commit();
+                    ++issued;
+                    if (issued - arrived > kInFlight) {
+                        tc::cp_async_wait_group<kInFlight>();
+                        tc::fence_async_shared();
+                        tc::mbar_arrive(&kfull[arrived & 7]);
+                        ++arrived;
                     }
                 }
-                tc::mma_commit(sbar);
+                tc::named_bar_sync(kGatherBar, 128);     // kptr is rewritten next tile
             }
-            if (!__syncthreads_and(tc::mbar_wait(sbar, g & 1, abort_flag))) {
+        }
+        flush();
+        if (!ok) {
+            *abort_flag = 1;
+            report(a.err, CSA_ERR_TIMEOUT, K_ATTEND_TC, blockIdx.x, 0);
+        }
+        if (gt == 0 && qctr > 0) {
+            volatile int never = 0;
+            static_cast<void>(tc::mbar_wait(qfull, (qctr - 1) & 1, &never, 200000000ull));
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            uint32_t tctr = 0, qctr = 0;
+            bool ok = true;
+            const uint32_t sK_a = tc::smem_u32(sK), sQ_a = tc::smem_u32(sQ), sP_a = tc::smem_u32(sP);
+            for (int64_t bt = blockIdx.x; bt < a.nqueries && ok; bt += gridDim.x, ++qctr) {
+                const QInfo q = query_info(a, bt);
+                bool ofree_done = qctr == 0;
+                if (!tc::mbar_wait(qfull, qctr & 1, abortv)) {
+                    ok = false;
+                    break;
+                }
+                for (int i = 0; i < q.ntiles; ++i, ++tctr) {
+                    for (int kb = 0; kb < 8 && ok; kb++) {
+                        if (!tc::mbar_wait(&kfull[kb], tctr & 1, abortv)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 4; kk++) {
+                            const uint64_t ad = tc::sdesc_sw128(sK_a + kb * 16384 + kk * 32);
+                            const uint64_t bd = tc::sdesc_sw128(sQ_a + kb * (H * 128) + kk * 32);
+                            tc::mma_f16(tmem, ad, bd, L::IDESC_S, (kb | kk) != 0);
+                        }
+                    }
+                    if (!ok)
+                        break;
+                    tc::mma_commit(sfull);
+                    if (i == q.ntiles - 1)
+                        tc::mma_commit(qfree);
+                    if (!ofree_done) {
+                        if (!tc::mbar_wait(ofree, (qctr - 1) & 1, abortv)) {
+                            ok = false;
+                            break;
+                        }
+                        ofree_done = true;
+                    }
+                    if (!tc::mbar_wait(pfull, tctr & 1, abortv)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after();
+                    for (int jt = 0; jt < 4; jt++) {
+#pragma unroll
+                        for (int kk = 0; kk < 8; kk++) {
+                            const uint64_t ad = tc::sdesc_sw128_mn(
+                                sK_a + (2 * jt) * 16384 + kk * 2048, 16384, 1024);
+                            const uint64_t bd =
+                                tc::sdesc_sw128(sP_a + (kk >> 2) * (H * 128) + (kk & 3) * 32);
+                            tc::mma_f16(tmem + H + jt * H, ad, bd, L::IDESC_O, (i > 0) || (kk > 0));
+                        }
+                        tc::mma_commit(&kfree[jt]);
+                    }
+                }
+                if (!ok)
+                    break;
+                if (q.ntiles == 0) {
+                    tc::mma_commit(qfree);
+                    if (!ofree_done && !tc::mbar_wait(ofree, (qctr - 1) & 1, abortv)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                tc::mma_commit(ofull);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report(a.err, CSA_ERR_TIMEOUT, K_ATTEND_TC, blockIdx.x, 1);
+            }
+            tc::mma_commit(done);
+            volatile int never = 0;
+            static_cast<void>(tc::mbar_wait(done, 0, &never, 200000000ull));
+        }
+    } else {
+        // ------------------------------------------------------------ softmax / epilogue
+        const int g = (warp - kSoftWarp0) >> 2;         // head group: heads h0 .. h0+15
+        const int h0 = 16 * g;
+        const int gbar = 1 + g;
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;                   // key (then dim) of this TMEM lane
+        const int et = (warp - kSoftWarp0 - 4 * g) * 32 + lane;   // 0..127 inside the group
+        const uint32_t lane_tm = tmem + ((uint32_t)(q4 * 32) << 16);
+        uint32_t tctr = 0, qctr = 0;
+        bool ok = true;
+        for (int64_t bt = blockIdx.x; bt < a.nqueries && ok; bt += gridDim.x, ++qctr) {
+            const QInfo q = query_info(a, bt);
+            if (et < 16)
+                m_run[h0 + et] = -INFINITY;
+            float lpart[16];
+#pragma unroll
+            for (int u = 0; u < 16; u++)
+                lpart[u] = 0.f;
+            tc::named_bar_sync(gbar, 128);
+            for (int i = 0; i < q.ntiles; ++i, ++tctr) {
+                const bool valid = key_row(a, q, bt, (int64_t)i * KT + r, g == 0) != nullptr;
+                const bool got = tc::mbar_wait(sfull, tctr & 1, abortv);
+                if (tc::named_bar_or(gbar, 128, !got)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after();
+                float z[16];
+                {
+                    uint32_t rr[16];
+                    tc::tmem_ld16(lane_tm + h0, rr);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int u = 0; u < 16; u++)
+                        z[u] = valid ? __uint_as_float(rr[u]) * a.scale : -INFINITY;
+                }
+                bool need = false;
+#pragma unroll
+                for (int u = 0; u < 16; u++)
+                    need |= z[u] > m_run[h0 + u] + kLazy;
+                if (tc::named_bar_or(gbar, 128, need)) {
+#pragma unroll
+                    for (int u = 0; u < 16; u++) {
+                        float v = z[u];
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1)
+                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+                        if (lane == 0)
+                            red[q4 * H + h0 + u] = v;
+                    }
+                    tc::named_bar_sync(gbar, 128);
+                    if (et < 16) {
+                        const int hh = h0 + et;
+                        const float tmax = fmaxf(fmaxf(red[hh], red[H + hh]),
+                                                 fmaxf(red[2 * H + hh], red[3 * H + hh]));
+                        const float mo = m_run[hh];
+                        const float mn = fmaxf(mo, tmax);
+                        fin[hh] = (mn == -INFINITY) ? 1.f : __expf(mo - mn);   // rescale factor
+                        m_run[hh] = mn;
+                    }
+                    tc::named_bar_sync(gbar, 128);
+                    if (i > 0) {
+                        // O^T of the earlier tiles is complete (S of this tile came after it)
+#pragma unroll 1
+                        for (int jt = 0; jt < 4; jt++) {
+                            uint32_t rr[16];
+                            const uint32_t ad = lane_tm + H + jt * H + h0;
+                            tc::tmem_ld16(ad, rr);
+                            tc::tmem_ld_wait();
+#pragma unroll
+                            for (int u = 0; u < 16; u++)
+                                rr[u] = __float_as_uint(__uint_as_float(rr[u]) * fin[h0 + u]);
+                            tc::tmem_st16(ad, rr);
+                        }
+                        tc::tmem_st_wait();
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; u++)
+                        lpart[u] *= fin[h0 + u];
+                }
+                // P^T rows h0..h0+15: 2 blocks of 64 keys, 128-byte swizzle
+                {
+                    uint8_t *prow = sP + (r >> 6) * (H * 128) + (r & 7) * 2;
+                    const int chunk = (r & 63) >> 3;
+#pragma unroll
+                    for (int u = 0; u < 16; u++) {
+                        const int hh = h0 + u;
+                        const float p = valid ? __expf(z[u] - m_run[hh]) : 0.f;
+                        const __nv_bfloat16 pb = __float2bfloat16_rn(p);
+                        lpart[u] += __bfloat162float(pb);
+                        *(__nv_bfloat16 *)(prow + hh * 128 + ((chunk ^ (hh & 7)) << 4)) = pb;
+                    }
+                }
+                tc::fence_async_shared();
+                tc::fence_before();
+                tc::mbar_arrive(pfull);
+            }
+            if (!ok)
+                break;
+            // ---- end of the query: normaliser, sink, output for heads h0..h0+15
+#pragma unroll
+            for (int u = 0; u < 16; u++) {
+                float v = lpart[u];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+                    v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == 0)
+                    red[q4 * H + h0 + u] = v;
+            }
+            tc::named_bar_sync(gbar, 128);
+            if (et < 16) {
+                const int hh = h0 + et;
+                const float l = red[hh] + red[H + hh] + red[2 * H + hh] + red[3 * H + hh];
+                const float mo = m_run[hh];
+                const float zs = a.sink[hh];
+                float f, lse;
+                if (zs == INFINITY) {
+                    f = 0.f;
+                    lse = INFINITY;
+                } else {
+                    const float M = fmaxf(mo, zs);
+                    if (M == -INFINITY) {
+                        f = 0.f;
+                        lse = -INFINITY;
+                    } else {
+                        const float e = __expf(mo - M);
+                        const float den = l * e + __expf(zs - M);
+                        f = e / den;
+                        lse = M + __logf(den);
+                    }
+                }
+                fin[hh] = q.ntiles > 0 ? f : 0.f;
+                if (a.lse)
+                    a.lse[bt * H + hh] = lse;
+            }
+            const bool got = tc::mbar_wait(ofull, qctr & 1, abortv);
+            if (tc::named_bar_or(gbar, 128, !got)) {
                 ok = false;
                 break;
             }
             tc::fence_after();
-            float z[H];
-            load_cols<H>(lane_tm, z);
-            int need = 0;
-#pragma unroll
-            for (int hh = 0; hh < H; hh++) {
-                z[hh] = valid ? z[hh] * a.scale : -INFINITY;
-                need |= z[hh] > m_run[hh] + kLazy;
-            }
-            if (__syncthreads_or(need)) {
-                // exact per-head maxima of this tile, then rescale what came before
-#pragma unroll
-                for (int hh = 0; hh < H; hh++) {
-                    float v = z[hh];
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1)
-                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-                    if (lane == 0)
-                        red[warp * H + hh] = v;
-                }
-                __syncthreads();
-                for (int hh = tid; hh < H; hh += kThreads) {
-                    const float tmax = fmaxf(fmaxf(red[hh], red[H + hh]),
-                                             fmaxf(red[2 * H + hh], red[3 * H + hh]));
-                    const float mo = m_run[hh];
-                    const float mn = fmaxf(mo, tmax);
-                    alpha[hh] = (mn == -INFINITY) ? 1.f : __expf(mo - mn);
-                    m_run[hh] = mn;
-                }
-                __syncthreads();
-                if (it > 0) {
-                    // every earlier product has completed (waited above)
+            __nv_bfloat16 *orow = a.out + bt * H * DIM + r;
 #pragma unroll 1
-                    for (int jt = 0; jt < 4; jt++)
-                        scale_cols<H>(lane_tm + H + jt * H, alpha);
-                }
-#pragma unroll
-                for (int hh = 0; hh < H; hh++)
-                    lpart[hh] *= alpha[hh];
-            }
-            // probabilities -> P^T (K-major rows = heads, 2 blocks of 64 keys)
-            {
-                uint8_t *prow = sP + (tid >> 6) * (H * 128) + (tid & 7) * 2;
-                const int chunk = (tid & 63) >> 3;
-#pragma unroll
-                for (int hh = 0; hh < H; hh++) {
-                    const float p = valid ? __expf(z[hh] - m_run[hh]) : 0.f;
-                    const __nv_bfloat16 pb = __float2bfloat16_rn(p);
-                    lpart[hh] += __bfloat162float(pb);
-                    *(__nv_bfloat16 *)(prow + hh * 128 + ((chunk ^ (hh & 7)) << 4)) = pb;
-                }
-            }
-            tc::fence_async_shared();
-            tc::fence_before();
-            __syncthreads();
-
-            // O^T += K^T P^T
-            if (tid == 0) {
-                tc::fence_after();
-#pragma unroll 1
-                for (int jt = 0; jt < 4; jt++) {
-#pragma unroll
-                    for (int kk = 0; kk < 8; kk++) {
-                        const uint64_t ad =
-                            tc::sdesc_sw128_mn(sK_a + (2 * jt) * 16384 + kk * 2048, 16384, 1024);
-                        const uint64_t bd =
-                            tc::sdesc_sw128(sP_a + (kk >> 2) * (H * 128) + (kk & 3) * 32);
-                        tc::mma_f16(tmem + H + jt * H, ad, bd, L::IDESC_O, (it > 0) || (kk > 0));
-                    }
-                }
-                tc::mma_commit(obar);
-            }
-        }
-        if (!ok)
-            break;
-
-        // ---- end of the query: normaliser, sink, output
-        const bool last_done = ntiles == 0 || tc::mbar_wait(obar, (g - 1) & 1, abort_flag);
-        if (!__syncthreads_and(last_done)) {
-            ok = false;
-            break;
-        }
-        tc::fence_after();
-#pragma unroll
-        for (int hh = 0; hh < H; hh++) {
-            float v = lpart[hh];
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-                v += __shfl_xor_sync(0xffffffffu, v, off);
-            if (lane == 0)
-                red[warp * H + hh] = v;
-        }
-        __syncthreads();
-        for (int hh = tid; hh < H; hh += kThreads) {
-            const float l = red[hh] + red[H + hh] + red[2 * H + hh] + red[3 * H + hh];
-            const float mo = m_run[hh];
-            const float zs = a.sink[hh];
-            float f, lse;
-            if (zs == INFINITY) {
-                f = 0.f;
-                lse = INFINITY;
-            } else {
-                const float M = fmaxf(mo, zs);
-                if (M == -INFINITY) {
-                    f = 0.f;
-                    lse = -INFINITY;
-                } else {
-                    const float e = __expf(mo - M);
-                    const float den = l * e + __expf(zs - M);
-                    f = e / den;
-                    lse = M + __logf(den);
-                }
-            }
-            if (ntiles == 0)
-                f = 0.f;
-            fin[hh] = f;
-            if (a.lse)
-                a.lse[bt * H + hh] = lse;
-        }
-        __syncthreads();
-        // O^T (lane = dim within a 128-dim block) -> sK as [H][512] bf16 -> out
-        __nv_bfloat16 *so = (__nv_bfloat16 *)sK;
-#pragma unroll 1
-        for (int jt = 0; jt < 4; jt++) {
-#pragma unroll 1
-            for (int c = 0; c < H / 16; c++) {
-                uint32_t r[16];
-                if (ntiles > 0) {
-                    tc::tmem_ld16(lane_tm + H + jt * H + c * 16, r);
+            for (int jt = 0; jt < 4; jt++) {
+                uint32_t rr[16];
+                if (q.ntiles > 0) {
+                    tc::tmem_ld16(lane_tm + H + jt * H + h0, rr);
                     tc::tmem_ld_wait();
                 }
 #pragma unroll
-                for (int j = 0; j < 16; j++) {
-                    const int hh = c * 16 + j;
-                    const float o = ntiles > 0 ? __uint_as_float(r[j]) * fin[hh] : 0.f;
-                    so[hh * DIM + jt * 128 + tid] = __float2bfloat16_rn(o);
+                for (int u = 0; u < 16; u++) {
+                    const float o = q.ntiles > 0 ? __uint_as_float(rr[u]) * fin[h0 + u] : 0.f;
+                    orow[(h0 + u) * DIM + jt * 128] = __float2bfloat16_rn(o);
                 }
             }
+            tc::fence_before();
+            tc::mbar_arrive(ofree);
+            tc::named_bar_sync(gbar, 128);     // fin / red / m_run reused next query
         }
-        tc::fence_before();
-        __syncthreads();
-        const uint4 *vs = (const uint4 *)so;
-        uint4 *vd = (uint4 *)(a.out + bt * H * DIM);
-        for (int v = tid; v < H * DIM / 8; v += kThreads)
-            vd[v] = vs[v];
-        __syncthreads();
-    }
-
-    tc::cp_async_wait_all();
-    if (!ok) {
-        *abort_flag = 1;
-        report(a.err, CSA_ERR_TIMEOUT, K_ATTEND_TC, blockIdx.x, g);
-    }
-    if (tid == 0) {
-        // every product issued above has completed once `done` flips
-        tc::mma_commit(done);
-        volatile int never = 0;
-        static_cast<void>(tc::mbar_wait(done, 0, &never, 200000000ull));
+        if (!ok) {
+            *abort_flag = 1;
+            report(a.err, CSA_ERR_TIMEOUT, K_ATTEND_TC, blockIdx.x, 2);
+        }
     }
     tc::fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kMmaWarp) {
         tc::fence_after();
         tc::tmem_dealloc(tmem, L::TMEM_COLS);
     }
@@ -408,15 +497,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const TcAttn a)
 template <int H>
 cudaError_t launch_h(const AttendArgs &a, unsigned *err, cudaStream_t s)
 {
+    CUtensorMap tm_q;
+    if (!make_tmap_2d(&tm_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.B * a.n_q * H,
+                      DIM, H))
+        return cudaErrorInvalidValue;
     TcAttn t;
-    t.q = (const __nv_bfloat16 *)a.q;
     t.ent = (const __nv_bfloat16 *)a.kv.body;
+    t.kwin = (const __nv_bfloat16 *)a.kwin;
     t.idx = a.idx;
     t.dense = a.dense;
     t.k = a.k;
     t.m = a.m;
     t.E = a.E;
-    t.kwin = (const __nv_bfloat16 *)a.kwin;
     t.win_rows = a.win_rows;
     t.win_pos0 = a.win_pos0;
     t.n_win = a.n_win;
@@ -436,8 +528,8 @@ cudaError_t launch_h(const AttendArgs &a, unsigned *err, cudaStream_t s)
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t grid = t.nqueries < sms ? t.nqueries : sms;
-    attend_tc_kernel<H><<<(unsigned)grid, kThreads, smem, s>>>(t);
+    const int64_t grid = t.nqueries < sms ? t.nqueries : sms;
+    attend_tc_kernel<H><<<(unsigned)grid, Lay<H>::THREADS, smem, s>>>(tm_q, t);
     return cudaGetLastError();
 }
 
@@ -450,7 +542,9 @@ cudaError_t launch_attend_tc(const AttendArgs &a, unsigned *err, cudaStream_t s,
         return cudaSuccess;
     if (a.h != 16 && a.h != 32 && a.h != 64)
         return cudaSuccess;
-    if (a.n_win > 0 && !a.kwin)
+    if (a.E <= 0 && (a.n_win == 0 || a.win_rows <= 0))
+        return cudaSuccess;
+    if ((int64_t)a.B * a.n_q * a.h >= INT32_MAX)     // TMA row coordinate of Q
         return cudaSuccess;
     *taken = true;
     switch (a.h) {

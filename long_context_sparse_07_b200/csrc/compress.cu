@@ -194,10 +194,15 @@ cudaError_t launch_compress(const CompressArgs &a, unsigned *err, cudaStream_t s
     const int VEC = a.in_dt == CSA_BF16 ? 8 : 4;
     const int tpe = a.c / VEC;
     const int64_t E = a.n / a.m;
-    // rows per entry and slices: keep roughly 8 rows per slice
+    // Rows of an entry are split over `split` slices when the window is long
+    // (>= 8 rows per slice), or, for narrow rows, when there are too few
+    // entries to keep the GPU busy (>= 2 rows per slice).
     const int rows = a.overlap ? 2 * a.m : a.m;
+    const int64_t target_threads = 148 * 1024;
     int split = 1;
-    while (split * 2 * tpe <= kThreads && rows / (split * 2) >= 8)
+    while (split * 2 * tpe <= kThreads &&
+           (rows / (split * 2) >= 8 ||
+            (tpe <= 32 && rows / (split * 2) >= 2 && E * tpe * split < target_threads)))
         split *= 2;
     const int epb = kThreads / (tpe * split);
     OutDesc o;

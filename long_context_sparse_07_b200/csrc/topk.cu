@@ -148,6 +148,112 @@ topk_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
         out[j] = -1;
 }
 
+// ---------------------------------------------------------------------------
+// Short rows (E <= 32 * kPerLane): one warp per row, keys held in registers,
+// per-warp 256-bin histograms in shared memory, warp ballots for the
+// compaction; no block-wide barrier at all.
+
+constexpr int kPerLane = 64;
+constexpr int kWarpRowsPerBlock = 8;
+
+template <int PER>
+__global__ void __launch_bounds__(32 * kWarpRowsPerBlock)
+topk_warp_kernel(const float *__restrict__ scores, int64_t rows, int64_t E, int64_t ld,
+                 const int64_t *__restrict__ q_pos, int m, int k, int32_t *__restrict__ idx)
+{
+    __shared__ unsigned hist_all[kWarpRowsPerBlock][256];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * kWarpRowsPerBlock + w;
+    if (row >= rows)
+        return;
+    unsigned *hist = hist_all[w];
+    const int64_t V = visible(q_pos[row], m, E);
+    int32_t *out = idx + row * k;
+    if (V <= k) {
+        for (int j = lane; j < k; j += 32)
+            out[j] = j < V ? j : -1;
+        return;
+    }
+    const float *src = scores + row * ld;
+    uint32_t key[PER];
+#pragma unroll
+    for (int i = 0; i < PER; i++) {
+        const int64_t s = (int64_t)i * 32 + lane;
+        key[i] = s < V ? float_key(src[s]) : 0u;
+    }
+    uint32_t prefix = 0, pmask = 0;
+    unsigned need = (unsigned)k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+        for (int b = 0; b < 8; b++)
+            hist[lane * 8 + b] = 0;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < PER; i++) {
+            const int64_t s = (int64_t)i * 32 + lane;
+            if (s < V && (key[i] & pmask) == prefix)
+                atomicAdd(&hist[(key[i] >> shift) & 255u], 1u);
+        }
+        __syncwarp();
+        // lane l owns bins 255-8l .. 248-8l (descending)
+        unsigned local = 0;
+#pragma unroll
+        for (int j = 0; j < 8; j++)
+            local += hist[255 - 8 * lane - j];
+        unsigned incl = local;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off)
+                incl += v;
+        }
+        const unsigned excl = incl - local;
+        unsigned bin = 0, nneed = need;
+        const bool mine = excl < need && need <= incl;
+        if (mine) {
+            unsigned cum = excl;
+            for (int j = 0; j < 8; j++) {
+                const int b = 255 - 8 * lane - j;
+                const unsigned hb = hist[b];
+                if (cum + hb >= need) {
+                    bin = (unsigned)b;
+                    nneed = need - cum;
+                    break;
+                }
+                cum += hb;
+            }
+        }
+        const unsigned owner = __ballot_sync(0xffffffffu, mine);
+        const int src_lane = owner ? __ffs(owner) - 1 : 0;
+        bin = __shfl_sync(0xffffffffu, bin, src_lane);
+        nneed = __shfl_sync(0xffffffffu, nneed, src_lane);
+        prefix |= bin << shift;
+        pmask |= 255u << shift;
+        need = nneed;
+        __syncwarp();
+    }
+    const uint32_t T = prefix;
+    unsigned base = 0, eq_seen = 0;
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < PER; i++) {
+        const int64_t s = (int64_t)i * 32 + lane;
+        const bool in = s < V;
+        const bool gt = in && key[i] > T;
+        const bool eq = in && key[i] == T;
+        const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+        const bool take = gt || (eq && eq_seen + __popc(eqb & lt) < need);
+        const unsigned tb = __ballot_sync(0xffffffffu, take);
+        const unsigned pos = base + __popc(tb & lt);
+        if (take && pos < (unsigned)k)
+            out[pos] = (int32_t)s;
+        base += __popc(tb);
+        eq_seen += __popc(eqb);
+    }
+    for (int j = (int)base + lane; j < k; j += 32)
+        out[j] = -1;
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s)
@@ -155,6 +261,19 @@ cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s)
     (void)err;
     if (a.rows == 0)
         return cudaSuccess;
+    if (a.E <= 32 * kPerLane) {
+        const unsigned blocks = (unsigned)((a.rows + kWarpRowsPerBlock - 1) / kWarpRowsPerBlock);
+        if (a.E <= 32 * 16)
+            topk_warp_kernel<16><<<blocks, 32 * kWarpRowsPerBlock, 0, s>>>(
+                a.scores, a.rows, a.E, a.ld, a.q_pos, a.m, a.k, a.idx);
+        else if (a.E <= 32 * 32)
+            topk_warp_kernel<32><<<blocks, 32 * kWarpRowsPerBlock, 0, s>>>(
+                a.scores, a.rows, a.E, a.ld, a.q_pos, a.m, a.k, a.idx);
+        else
+            topk_warp_kernel<64><<<blocks, 32 * kWarpRowsPerBlock, 0, s>>>(
+                a.scores, a.rows, a.E, a.ld, a.q_pos, a.m, a.k, a.idx);
+        return cudaGetLastError();
+    }
     const int resident = a.E > a.k;
     const int64_t cap = a.E < kResident ? a.E : kResident;
     const size_t smem = resident ? (size_t)cap * sizeof(uint32_t) : 0;
