@@ -234,10 +234,13 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(Dev d)
 
 }  // namespace
 
+size_t attend_tc_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys);
+
+// Scratch of the tensor-core path (split-key partial results); the CUDA-core
+// path needs none.
 size_t attend_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys)
 {
-    (void)B; (void)n_q; (void)h; (void)c; (void)max_keys;
-    return 0;
+    return attend_tc_workspace_size(B, n_q, h, c, max_keys);
 }
 
 cudaError_t launch_attend_tc(const AttendArgs &a, unsigned *err, cudaStream_t s, bool *taken);

@@ -49,6 +49,11 @@ constexpr int kInFlight = 3;         // 16 KB blocks a gather thread may leave i
 
 struct TcAttn {
     const __nv_bfloat16 *ent, *kwin;
+    const uint8_t *ent8;             // fp8 layout: e4m3 body [rows, 448]
+    const float *ent_scale;          //   one scale per 64 body dims [rows, 7]
+    const __nv_bfloat16 *ent_rope;   //   bf16 RoPE dims [rows, 64]
+    int nchunks, tpc;                // split of each query's key tiles over work items
+    float *ws_o, *ws_ml;             // partial O [item][H][512] and (m, l) [item][H][2]
     const int32_t *idx;
     int dense, k, m;
     int64_t E;
@@ -72,7 +77,8 @@ struct Lay {
     static constexpr size_t Q_OFF = 8 * 16384;                      // 8 x H x 128
     static constexpr size_t P_OFF = Q_OFF + 8 * H * 128;            // 2 x H x 128
     static constexpr size_t PTR_OFF = P_OFF + 2 * H * 128;          // 128 row pointers
-    static constexpr size_t F_OFF = PTR_OFF + KT * 8;               // m, red[4], fin
+    static constexpr size_t ROW_OFF = PTR_OFF + KT * 8;             // 128 fp8 entry rows
+    static constexpr size_t F_OFF = ROW_OFF + KT * 8;               // m, red[4], fin
     static constexpr size_t BAR_OFF = F_OFF + ((6 * H * 4 + 63) / 64) * 64;
     static constexpr size_t TOTAL = BAR_OFF + 256;
     static constexpr uint32_t TMEM_COLS = (5 * H <= 128) ? 128 : (5 * H <= 256 ? 256 : 512);
@@ -80,13 +86,15 @@ struct Lay {
     static constexpr uint32_t IDESC_O = tc::idesc_bf16(128, H, 1, 0);
 };
 
-// Per-query quantities, computed identically by every role.
+// Per-work-item quantities (a query, or one chunk of a query's key tiles),
+// computed identically by every role.
 struct QInfo {
     int64_t b, t, V, nsel, nwin, w0, wp0, nk;
-    int ntiles;
+    int ntiles;       // tiles of this item
+    int tile0;        // first key tile of this item
 };
 
-__device__ __forceinline__ QInfo query_info(const TcAttn &a, int64_t bt)
+__device__ __forceinline__ QInfo query_info(const TcAttn &a, int64_t bt, int chunk)
 {
     QInfo q;
     q.b = bt / a.n_q;
@@ -97,21 +105,36 @@ __device__ __forceinline__ QInfo query_info(const TcAttn &a, int64_t bt)
     q.nwin = a.n_win > 0 ? q.t - q.w0 + 1 : 0;
     q.wp0 = a.win_pos0 ? a.win_pos0[q.b] : 0;
     q.nk = q.nsel + q.nwin;
-    q.ntiles = (int)((q.nk + KT - 1) / KT);
+    const int all = (int)((q.nk + KT - 1) / KT);
+    q.tile0 = chunk * a.tpc;
+    int end = q.tile0 + a.tpc;
+    if (end > all)
+        end = all;
+    q.ntiles = end > q.tile0 ? end - q.tile0 : 0;
     return q;
 }
 
 // Source row of key slot j of a query (NULL: empty slot or out of range).
 // `report_bad` records a selection index or window position out of range.
+// With the fp8 entry layout, an entry comes back as *entry_row >= 0 (its row
+// in the cache) and a NULL pointer stands for "not a bf16 row".
+template <bool KV8>
 __device__ __forceinline__ const __nv_bfloat16 *key_row(const TcAttn &a, const QInfo &q,
-                                                        int64_t bt, int64_t j, bool report_bad)
+                                                        int64_t bt, int64_t j, bool report_bad,
+                                                        int64_t *entry_row)
 {
+    *entry_row = -1;
     if (j < q.nsel) {
         const int64_t s = a.dense ? j : (int64_t)a.idx[bt * a.k + j];
         if (s < 0)
             return nullptr;
-        if (s < q.V)
+        if (s < q.V) {
+            if (KV8) {
+                *entry_row = q.b * a.E + s;
+                return nullptr;
+            }
             return a.ent + (q.b * a.E + s) * DIM;
+        }
         if (report_bad)
             report(a.err, CSA_ERR_BOUNDS, K_ATTEND_TC, (unsigned)bt, (unsigned)s);
         return nullptr;
@@ -127,7 +150,7 @@ __device__ __forceinline__ const __nv_bfloat16 *key_row(const TcAttn &a, const Q
     return nullptr;
 }
 
-template <int H>
+template <int H, bool KV8>
 __global__ void __launch_bounds__(Lay<H>::THREADS, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
 {
@@ -139,6 +162,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
     uint8_t *sQ = sm + L::Q_OFF;
     uint8_t *sP = sm + L::P_OFF;
     const __nv_bfloat16 **kptr = (const __nv_bfloat16 **)(sm + L::PTR_OFF);
+    int64_t *krow = (int64_t *)(sm + L::ROW_OFF);
     float *m_run = (float *)(sm + L::F_OFF);     // [H]
     float *red = m_run + H;                      // [4][H]
     float *fin = red + 4 * H;                    // [H]
@@ -149,6 +173,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
     uint64_t *ofull = bars + 16, *ofree = bars + 17, *done = bars + 18;
     uint32_t *tmem_slot = (uint32_t *)(bars + 19);
     int *abort_flag = (int *)(tmem_slot + 1);
+    const int64_t nitems = a.nqueries * a.nchunks;
+    const bool split = a.nchunks > 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -180,7 +206,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
     if (warp < 4) {
         // ------------------------------------------------------------ gather
         const int gt = tid;                          // 0..127
-        const void *zero_src = a.E > 0 ? (const void *)a.ent : (const void *)a.kwin;
+        const void *zero_src = KV8 ? (a.kwin ? (const void *)a.kwin : (const void *)a.ent8)
+                                   : (a.E > 0 ? (const void *)a.ent : (const void *)a.kwin);
         uint32_t tctr = 0, qctr = 0, issued = 0, arrived = 0;
         bool ok = true;
         // announce every block still in flight: required before any wait on
@@ -191,8 +218,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
             for (; arrived < issued; ++arrived)
                 tc::mbar_arrive(&kfull[arrived & 7]);
         };
-        for (int64_t bt = blockIdx.x; bt < a.nqueries && ok; bt += gridDim.x, ++qctr) {
-            const QInfo q = query_info(a, bt);
+        for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++qctr) {
+            const int64_t bt = w / a.nchunks;
+            const QInfo q = query_info(a, bt, (int)(w % a.nchunks));
             flush();
             const bool qf = qctr == 0 || tc::mbar_wait(qfree, (qctr - 1) & 1, abortv);
             if (tc::named_bar_or(kGatherBar, 128, !qf)) {
@@ -206,7 +234,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
             }
             for (int i = 0; i < q.ntiles && ok; ++i, ++tctr) {
                 flush();
-                kptr[gt] = key_row(a, q, bt, (int64_t)i * KT + gt, false);
+                int64_t er;
+                kptr[gt] = key_row<KV8>(a, q, bt, (int64_t)(q.tile0 + i) * KT + gt, false, &er);
+                krow[gt] = er;
                 tc::named_bar_sync(kGatherBar, 128);
                 for (int kb = 0; kb < 8; kb++) {
                     if ((kb & 1) == 0 && tctr > 0) {
@@ -220,10 +250,31 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                     for (int u = 0; u < 8; u++) {
                         const int lin = u * 128 + gt;
                         const int r = lin >> 3, c = lin & 7;
-                        const __nv_bfloat16 *sp = kptr[r];
                         uint8_t *dst = sK + kb * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
-                        tc::cp_async16(dst, sp ? (const void *)(sp + kb * 64 + c * 8) : zero_src,
-                                       sp ? 16u : 0u);
+                        if (KV8 && krow[r] >= 0) {
+                            const int64_t er2 = krow[r];
+                            if (kb < 7) {
+                                // 8 e4m3 codes of one 64-dim scale group -> 8 bf16
+                                const uint2 cw = *(const uint2 *)(a.ent8 + er2 * 448 + kb * 64 + c * 8);
+                                const float sc = a.ent_scale[er2 * 7 + kb];
+                                const uint16_t *c2 = (const uint16_t *)&cw;
+                                __nv_bfloat162 o[4];
+#pragma unroll
+                                for (int e = 0; e < 4; e++) {
+                                    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                                        (__nv_fp8x2_storage_t)c2[e], __NV_E4M3);
+                                    const float2 f = __half22float2(__half2(hr));
+                                    o[e] = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+                                }
+                                *(uint4 *)dst = *(const uint4 *)o;
+                            } else {
+                                tc::cp_async16(dst, a.ent_rope + er2 * 64 + c * 8, 16u);
+                            }
+                        } else {
+                            const __nv_bfloat16 *sp = kptr[r];
+                            tc::cp_async16(dst, sp ? (const void *)(sp + kb * 64 + c * 8) : zero_src,
+                                           sp ? 16u : 0u);
+                        }
                     }
                     tc::cp_async_commit();
                     ++issued;
@@ -234,7 +285,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                         ++arrived;
                     }
                 }
-                tc::named_bar_sync(kGatherBar, 128);     // kptr is rewritten next tile
+                tc::named_bar_sync(kGatherBar, 128);     // kptr / krow rewritten next tile
             }
         }
         flush();
@@ -252,8 +303,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
             uint32_t tctr = 0, qctr = 0;
             bool ok = true;
             const uint32_t sK_a = tc::smem_u32(sK), sQ_a = tc::smem_u32(sQ), sP_a = tc::smem_u32(sP);
-            for (int64_t bt = blockIdx.x; bt < a.nqueries && ok; bt += gridDim.x, ++qctr) {
-                const QInfo q = query_info(a, bt);
+            for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++qctr) {
+                const QInfo q = query_info(a, w / a.nchunks, (int)(w % a.nchunks));
                 bool ofree_done = qctr == 0;
                 if (!tc::mbar_wait(qfull, qctr & 1, abortv)) {
                     ok = false;
@@ -332,8 +383,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
         const uint32_t lane_tm = tmem + ((uint32_t)(q4 * 32) << 16);
         uint32_t tctr = 0, qctr = 0;
         bool ok = true;
-        for (int64_t bt = blockIdx.x; bt < a.nqueries && ok; bt += gridDim.x, ++qctr) {
-            const QInfo q = query_info(a, bt);
+        for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++qctr) {
+            const int64_t bt = w / a.nchunks;
+            const QInfo q = query_info(a, bt, (int)(w % a.nchunks));
             if (et < 16)
                 m_run[h0 + et] = -INFINITY;
             float lpart[16];
@@ -342,7 +394,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                 lpart[u] = 0.f;
             tc::named_bar_sync(gbar, 128);
             for (int i = 0; i < q.ntiles; ++i, ++tctr) {
-                const bool valid = key_row(a, q, bt, (int64_t)i * KT + r, g == 0) != nullptr;
+                int64_t er;
+                const bool valid =
+                    key_row<KV8>(a, q, bt, (int64_t)(q.tile0 + i) * KT + r, g == 0, &er) != nullptr ||
+                    er >= 0;
                 const bool got = tc::mbar_wait(sfull, tctr & 1, abortv);
                 if (tc::named_bar_or(gbar, 128, !got)) {
                     ok = false;
@@ -421,7 +476,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
             }
             if (!ok)
                 break;
-            // ---- end of the query: normaliser, sink, output for heads h0..h0+15
+            // ---- end of the item: normaliser, sink, output for heads h0..h0+15
 #pragma unroll
             for (int u = 0; u < 16; u++) {
                 float v = lpart[u];
@@ -436,26 +491,33 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                 const int hh = h0 + et;
                 const float l = red[hh] + red[H + hh] + red[2 * H + hh] + red[3 * H + hh];
                 const float mo = m_run[hh];
-                const float zs = a.sink[hh];
-                float f, lse;
-                if (zs == INFINITY) {
-                    f = 0.f;
-                    lse = INFINITY;
+                if (split) {
+                    // partial result of this key chunk: raw accumulator, its offset and sum
+                    fin[hh] = 1.f;
+                    a.ws_ml[(w * H + hh) * 2] = mo;
+                    a.ws_ml[(w * H + hh) * 2 + 1] = l;
                 } else {
-                    const float M = fmaxf(mo, zs);
-                    if (M == -INFINITY) {
+                    const float zs = a.sink[hh];
+                    float f, lse;
+                    if (zs == INFINITY) {
                         f = 0.f;
-                        lse = -INFINITY;
+                        lse = INFINITY;
                     } else {
-                        const float e = __expf(mo - M);
-                        const float den = l * e + __expf(zs - M);
-                        f = e / den;
-                        lse = M + __logf(den);
+                        const float M = fmaxf(mo, zs);
+                        if (M == -INFINITY) {
+                            f = 0.f;
+                            lse = -INFINITY;
+                        } else {
+                            const float e = __expf(mo - M);
+                            const float den = l * e + __expf(zs - M);
+                            f = e / den;
+                            lse = M + __logf(den);
+                        }
                     }
+                    fin[hh] = q.ntiles > 0 ? f : 0.f;
+                    if (a.lse)
+                        a.lse[bt * H + hh] = lse;
                 }
-                fin[hh] = q.ntiles > 0 ? f : 0.f;
-                if (a.lse)
-                    a.lse[bt * H + hh] = lse;
             }
             const bool got = tc::mbar_wait(ofull, qctr & 1, abortv);
             if (tc::named_bar_or(gbar, 128, !got)) {
@@ -463,23 +525,38 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                 break;
             }
             tc::fence_after();
-            __nv_bfloat16 *orow = a.out + bt * H * DIM + r;
+            if (split) {
+                float *orow = a.ws_o + (w * H) * DIM + r;
 #pragma unroll 1
-            for (int jt = 0; jt < 4; jt++) {
-                uint32_t rr[16];
-                if (q.ntiles > 0) {
-                    tc::tmem_ld16(lane_tm + H + jt * H + h0, rr);
-                    tc::tmem_ld_wait();
-                }
+                for (int jt = 0; jt < 4; jt++) {
+                    uint32_t rr[16];
+                    if (q.ntiles > 0) {
+                        tc::tmem_ld16(lane_tm + H + jt * H + h0, rr);
+                        tc::tmem_ld_wait();
+                    }
 #pragma unroll
-                for (int u = 0; u < 16; u++) {
-                    const float o = q.ntiles > 0 ? __uint_as_float(rr[u]) * fin[h0 + u] : 0.f;
-                    orow[(h0 + u) * DIM + jt * 128] = __float2bfloat16_rn(o);
+                    for (int u = 0; u < 16; u++)
+                        orow[(h0 + u) * DIM + jt * 128] = q.ntiles > 0 ? __uint_as_float(rr[u]) : 0.f;
+                }
+            } else {
+                __nv_bfloat16 *orow = a.out + bt * H * DIM + r;
+#pragma unroll 1
+                for (int jt = 0; jt < 4; jt++) {
+                    uint32_t rr[16];
+                    if (q.ntiles > 0) {
+                        tc::tmem_ld16(lane_tm + H + jt * H + h0, rr);
+                        tc::tmem_ld_wait();
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; u++) {
+                        const float o = q.ntiles > 0 ? __uint_as_float(rr[u]) * fin[h0 + u] : 0.f;
+                        orow[(h0 + u) * DIM + jt * 128] = __float2bfloat16_rn(o);
+                    }
                 }
             }
             tc::fence_before();
             tc::mbar_arrive(ofree);
-            tc::named_bar_sync(gbar, 128);     // fin / red / m_run reused next query
+            tc::named_bar_sync(gbar, 128);     // fin / red / m_run reused next item
         }
         if (!ok) {
             *abort_flag = 1;
@@ -494,7 +571,67 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
     }
 }
 
-template <int H>
+// Joins the key chunks of each (query, head): out = sum_c O_c e^{m_c - M} /
+// (sum_c l_c e^{m_c - M} + e^{z' - M}), M = max(max_c m_c, z'), the sink z'
+// entering once here.
+__global__ void __launch_bounds__(128)
+combine_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_ml, int nchunks, int H,
+               const float *__restrict__ sink, __nv_bfloat16 *__restrict__ out,
+               float *__restrict__ lse)
+{
+    const int64_t bt = blockIdx.x;
+    const int hh = blockIdx.y;
+    const float zs = sink[hh];
+    float M = zs;
+    for (int c = 0; c < nchunks; c++)
+        M = fmaxf(M, ws_ml[((bt * nchunks + c) * H + hh) * 2]);
+    float den = 0.f, l_out;
+    const bool zero = zs == INFINITY || M == -INFINITY;
+    if (!zero) {
+        den = __expf(zs - M);
+        for (int c = 0; c < nchunks; c++) {
+            const float *ml = ws_ml + ((bt * nchunks + c) * H + hh) * 2;
+            if (ml[0] != -INFINITY)
+                den += ml[1] * __expf(ml[0] - M);
+        }
+        l_out = M + __logf(den);
+    } else {
+        l_out = zs == INFINITY ? INFINITY : -INFINITY;
+    }
+    for (int d = threadIdx.x; d < DIM; d += blockDim.x) {
+        float o = 0.f;
+        if (!zero) {
+            for (int c = 0; c < nchunks; c++) {
+                const float mc = ws_ml[((bt * nchunks + c) * H + hh) * 2];
+                if (mc != -INFINITY)
+                    o += ws_o[((bt * nchunks + c) * H + hh) * DIM + d] * __expf(mc - M);
+            }
+            o /= den;
+        }
+        out[(bt * H + hh) * DIM + d] = __float2bfloat16_rn(o);
+    }
+    if (threadIdx.x == 0 && lse)
+        lse[bt * H + hh] = l_out;
+}
+
+// Split of each query's key tiles over work items when there are too few
+// queries to fill the GPU: about two items per SM.
+void split_plan(int64_t nq, int64_t max_keys, int *nchunks, int *tpc)
+{
+    const int64_t tiles = (max_keys + KT - 1) / KT;
+    *nchunks = 1;
+    *tpc = 1 << 28;
+    if (nq <= 0 || nq >= 74 || tiles <= 1)
+        return;
+    int64_t want = (296 + nq - 1) / nq;
+    if (want > tiles)
+        want = tiles;
+    const int64_t t = (tiles + want - 1) / want;
+    *tpc = (int)t;
+    *nchunks = (int)((tiles + t - 1) / t);
+}
+
+template <int H, bool KV8>
 cudaError_t launch_h(const AttendArgs &a, unsigned *err, cudaStream_t s)
 {
     CUtensorMap tm_q;
@@ -502,7 +639,10 @@ cudaError_t launch_h(const AttendArgs &a, unsigned *err, cudaStream_t s)
                       DIM, H))
         return cudaErrorInvalidValue;
     TcAttn t;
-    t.ent = (const __nv_bfloat16 *)a.kv.body;
+    t.ent = KV8 ? nullptr : (const __nv_bfloat16 *)a.kv.body;
+    t.ent8 = KV8 ? (const uint8_t *)a.kv.body : nullptr;
+    t.ent_scale = KV8 ? a.kv.scale : nullptr;
+    t.ent_rope = KV8 ? (const __nv_bfloat16 *)a.kv.rope : nullptr;
     t.kwin = (const __nv_bfloat16 *)a.kwin;
     t.idx = a.idx;
     t.dense = a.dense;
@@ -520,25 +660,56 @@ cudaError_t launch_h(const AttendArgs &a, unsigned *err, cudaStream_t s)
     t.out = (__nv_bfloat16 *)a.out;
     t.lse = a.lse;
     t.err = err;
+    split_plan(t.nqueries, (a.dense ? a.E : a.k) + a.n_win, &t.nchunks, &t.tpc);
+    t.ws_o = (float *)a.ws;
+    t.ws_ml = t.nchunks > 1 ? t.ws_o + (size_t)t.nqueries * t.nchunks * H * DIM : nullptr;
+    if (t.nchunks > 1 && !a.ws)
+        return cudaErrorInvalidValue;
     const size_t smem = Lay<H>::TOTAL + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<H>,
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<H, KV8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t grid = t.nqueries < sms ? t.nqueries : sms;
-    attend_tc_kernel<H><<<(unsigned)grid, Lay<H>::THREADS, smem, s>>>(tm_q, t);
+    const int64_t items = t.nqueries * t.nchunks;
+    const int64_t grid = items < sms ? items : sms;
+    attend_tc_kernel<H, KV8><<<(unsigned)grid, Lay<H>::THREADS, smem, s>>>(tm_q, t);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || t.nchunks == 1)
+        return e;
+    combine_kernel<<<dim3((unsigned)t.nqueries, H), 128, 0, s>>>(t.ws_o, t.ws_ml, t.nchunks, H,
+                                                                   a.sink, t.out, a.lse);
     return cudaGetLastError();
+}
+
+bool takes_fp8(const AttendArgs &a)
+{
+    return a.kv.dt == CSA_E4M3 && a.kv.rope_dims == 64 && a.kv.scale_group == 64 &&
+           a.kv.rope != nullptr;
 }
 
 }  // namespace
 
+size_t attend_tc_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys)
+{
+    if (c != DIM || (h != 16 && h != 32 && h != 64))
+        return 0;
+    int nchunks, tpc;
+    split_plan((int64_t)B * n_q, max_keys, &nchunks, &tpc);
+    if (nchunks <= 1)
+        return 0;
+    return (size_t)B * n_q * nchunks * h * (DIM + 2) * sizeof(float);
+}
+
 cudaError_t launch_attend_tc(const AttendArgs &a, unsigned *err, cudaStream_t s, bool *taken)
 {
     *taken = false;
-    if (a.q_dt != CSA_BF16 || a.kv.dt != CSA_BF16 || a.kv.c != DIM)
+    if (a.q_dt != CSA_BF16 || a.kv.c != DIM)
+        return cudaSuccess;
+    const bool fp8 = takes_fp8(a);
+    if (a.kv.dt != CSA_BF16 && !fp8)
         return cudaSuccess;
     if (a.h != 16 && a.h != 32 && a.h != 64)
         return cudaSuccess;
@@ -547,10 +718,17 @@ cudaError_t launch_attend_tc(const AttendArgs &a, unsigned *err, cudaStream_t s,
     if ((int64_t)a.B * a.n_q * a.h >= INT32_MAX)     // TMA row coordinate of Q
         return cudaSuccess;
     *taken = true;
+    if (fp8) {
+        switch (a.h) {
+        case 16: return launch_h<16, true>(a, err, s);
+        case 32: return launch_h<32, true>(a, err, s);
+        default: return launch_h<64, true>(a, err, s);
+        }
+    }
     switch (a.h) {
-    case 16: return launch_h<16>(a, err, s);
-    case 32: return launch_h<32>(a, err, s);
-    default: return launch_h<64>(a, err, s);
+    case 16: return launch_h<16, false>(a, err, s);
+    case 32: return launch_h<32, false>(a, err, s);
+    default: return launch_h<64, false>(a, err, s);
     }
 }
 

@@ -237,12 +237,14 @@ def _attend_case(B, n, E, m, h, c, k, n_win, dtype, seed, rows=None, kv_layout="
     scale = 1.0 / math.sqrt(c)
     qp = torch.as_tensor(pos, dtype=torch.int64).to(DEV)
     wp = torch.as_tensor(win_pos0).to(DEV)
+    nws = abi.csa_mqa_workspace_size(B, n_q, h, c, (E if dense else k) + n_win)
+    ws = torch.empty(nws, device=DEV, dtype=torch.uint8) if nws else None
     if dense:
         abi.hca_dense_mqa(q.to(DEV), ent, E, m, kwin.to(DEV), wp, n_win, qp, sink.to(DEV),
-                          scale, out, lse)
+                          scale, out, lse, workspace=ws)
     else:
         abi.csa_sparse_mqa(q.to(DEV), ent, E, m, idx.to(DEV), k, kwin.to(DEV), wp, n_win, qp,
-                           sink.to(DEV), scale, out, lse)
+                           sink.to(DEV), scale, out, lse, workspace=ws)
     if bad_index:
         with pytest.raises(abi.CsaError) as ei:
             abi.csa_get_error()
@@ -286,6 +288,24 @@ def test_attend_sparse_decode_fp8_layout():
 def test_attend_dense_hca_sampled():
     rows = sample_rows(128 * 40, 128, 96, 3)
     _attend_case(1, 128 * 40, 40, 128, 64, 512, 0, 128, "bf16", 35, rows=rows, dense=True)
+
+
+def test_attend_split_keys_dense_bf16_few_queries():
+    # few queries, many keys: each query's key tiles are split over blocks and
+    # joined by the combine step (scratch from csa_mqa_workspace_size)
+    rows = np.array([0, 15, 16 * 700 - 1, 16 * 1500, 16 * 3000 - 1, 16 * 2999 + 5])
+    _attend_case(1, 16 * 3000, 3000, 16, 32, 512, 0, 128, "bf16", 40, rows=rows, dense=True)
+
+
+def test_attend_split_keys_sparse_bf16_h16():
+    rows = np.array([3, 4000, 4 * 2000 - 1])
+    _attend_case(1, 4 * 2000, 2000, 4, 16, 512, 1024, 128, "bf16", 41, rows=rows)
+
+
+def test_attend_split_keys_decode_fp8_h64_hca():
+    L = 128 * 300
+    _attend_case(2, L, 300, 128, 64, 512, 0, 128, "bf16", 42, rows=np.array([L - 1]),
+                 kv_layout="fp8", dense=True)
 
 
 def test_attend_dense_f32_small():
