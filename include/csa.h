@@ -210,6 +210,34 @@ csa_status hca_dense_mqa(const void *q, csa_dtype q_dt, csa_entries kv, int64_t 
 size_t csa_mqa_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys);
 
 /*
+ * csa_sparse_mqa_noalloc -- csa_sparse_mqa without a workspace argument, for
+ * callers that cannot allocate device memory on their hot path (code hosted
+ * by a framework that owns all device memory through pre-reserved pools, or
+ * a decode loop that cannot afford the device-wide synchronisation an
+ * allocation may cause). The method on the reference pages has no
+ * counterpart of this call: it only changes where the scratch lives.
+ *   Scratch (the split-key partial results) comes from one file-scope device
+ *   array of csa_noalloc_scratch_bytes() bytes (16 MiB) that every GPU loading
+ *   the library holds until the process exits. The call allocates nothing.
+ *   Every other argument, the results and the error behaviour are those of
+ *   csa_sparse_mqa. A shape whose scratch (csa_mqa_workspace_size) exceeds the
+ *   array returns CSA_ERR_UNSUPPORTED, launches nothing and says so in
+ *   csa_last_message().
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make it before capturing the stream into a graph.
+ *   All calls share the one array and each call overwrites the part it uses
+ *   before reading it, so nothing needs clearing; but calls that may overlap
+ *   on the GPU (different streams, or different host threads on one device)
+ *   race on it and must be serialised by the caller.
+ */
+csa_status csa_sparse_mqa_noalloc(const void *q, csa_dtype q_dt, csa_entries kv, int64_t E, int m,
+                                  const int32_t *idx, int k, const void *kwin, int64_t win_rows,
+                                  const int64_t *win_pos0, int n_win, const int64_t *q_pos,
+                                  const float *sink, int B, int64_t n_q, int h, float scale,
+                                  void *out, float *lse, void *stream);
+size_t csa_noalloc_scratch_bytes(void);
+
+/*
  * csa_get_error -- synchronises the current device, reads and clears its
  * device error word, and returns the status it held (CSA_OK if none). When
  * buf is not NULL, a description (at most len bytes, NUL-terminated) is

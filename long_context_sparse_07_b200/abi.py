@@ -27,7 +27,8 @@ STATUS = {0: "CSA_OK", -1: "CSA_ERR_INVALID_ARG", -2: "CSA_ERR_UNSUPPORTED",
 # every symbol that include/csa.h declares
 EXPORTS = ("csa_abi_version", "csa_status_string", "csa_last_message", "csa_compress_kv",
            "csa_indexer_scores", "csa_topk", "csa_topk_workspace_size", "csa_sparse_mqa",
-           "hca_dense_mqa", "csa_mqa_workspace_size", "csa_get_error")
+           "hca_dense_mqa", "csa_mqa_workspace_size", "csa_sparse_mqa_noalloc",
+           "csa_noalloc_scratch_bytes", "csa_get_error")
 
 
 class CsaError(RuntimeError):
@@ -79,6 +80,11 @@ def load(path: str = LIB_PATH):
                                 _I, _F, _P, _P, _P, _S, _P]
     L.csa_mqa_workspace_size.restype = _S
     L.csa_mqa_workspace_size.argtypes = [_I, _I64, _I, _I, _I64]
+    L.csa_sparse_mqa_noalloc.restype = _I
+    L.csa_sparse_mqa_noalloc.argtypes = [_P, _I, _Entries, _I64, _I, _P, _I, _P, _I64, _P, _I, _P,
+                                         _P, _I, _I64, _I, _F, _P, _P, _P]
+    L.csa_noalloc_scratch_bytes.restype = _S
+    L.csa_noalloc_scratch_bytes.argtypes = []
     L.csa_get_error.restype = _I
     L.csa_get_error.argtypes = [ctypes.c_char_p, _S]
     _lib = L
@@ -178,6 +184,22 @@ def csa_sparse_mqa(q, kv: Entries, E: int, m: int, idx, k: int, kwin, win_pos0, 
                                  _ptr(kwin), win_rows, _ptr(win_pos0), n_win, _ptr(q_pos),
                                  _ptr(sink), B, n_q, h, scale, _ptr(out), _ptr(lse),
                                  _ptr(workspace), ws, _stream(stream)))
+
+
+def csa_sparse_mqa_noalloc(q, kv: Entries, E: int, m: int, idx, k: int, kwin, win_pos0,
+                           n_win: int, q_pos, sink, scale: float, out, lse=None, stream=None):
+    """csa_sparse_mqa with the library's fixed device scratch instead of a
+    workspace: for callers that cannot allocate device memory."""
+    B, n_q, h, c = q.shape
+    win_rows = kwin.shape[-2] if kwin is not None else 0
+    _check(load().csa_sparse_mqa_noalloc(_ptr(q), dtype_code(q), kv.struct(), E, m, _ptr(idx), k,
+                                         _ptr(kwin), win_rows, _ptr(win_pos0), n_win,
+                                         _ptr(q_pos), _ptr(sink), B, n_q, h, scale, _ptr(out),
+                                         _ptr(lse), _stream(stream)))
+
+
+def csa_noalloc_scratch_bytes() -> int:
+    return int(load().csa_noalloc_scratch_bytes())
 
 
 def hca_dense_mqa(q, kv: Entries, E: int, m: int, kwin, win_pos0, n_win: int, q_pos, sink,

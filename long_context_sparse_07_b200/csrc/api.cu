@@ -88,6 +88,10 @@ csa_status check_entries(const csa_entries &t, int c, bool allow_fp8, const char
 
 }  // namespace
 
+namespace csa {
+void set_last_message(const char *msg) { snprintf(g_msg, sizeof g_msg, "%s", msg); }
+}  // namespace csa
+
 extern "C" {
 
 int csa_abi_version(void) { return 1; }

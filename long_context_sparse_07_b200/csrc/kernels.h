@@ -65,6 +65,9 @@ struct AttendArgs {
     size_t ws_bytes;
 };
 cudaError_t launch_attend(const AttendArgs &a, unsigned *err, cudaStream_t s);
+
+// Sets the text that csa_last_message() returns on this thread.
+void set_last_message(const char *msg);
 size_t attend_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys);
 
 }  // namespace csa
