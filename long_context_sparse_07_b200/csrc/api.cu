@@ -184,8 +184,7 @@ csa_status csa_indexer_scores(const void *qI, const float *qI_scale, const float
 
 size_t csa_topk_workspace_size(int64_t rows, int64_t E, int k)
 {
-    (void)rows; (void)E; (void)k;
-    return 0;
+    return csa::topk_workspace_size(rows, E, k);
 }
 
 csa_status csa_topk(const float *scores, int64_t rows, int64_t E, int64_t ld,
@@ -193,7 +192,6 @@ csa_status csa_topk(const float *scores, int64_t rows, int64_t E, int64_t ld,
                     size_t ws_bytes, void *stream)
 {
     const char *w = "csa_topk";
-    (void)workspace; (void)ws_bytes;
     REQUIRE(scores && q_pos && idx, CSA_ERR_INVALID_ARG, "%s: scores, q_pos and idx required", w);
     REQUIRE(rows >= 0 && rows <= INT32_MAX && E >= 0 && E <= INT32_MAX && ld >= E,
             CSA_ERR_INVALID_ARG, "%s: bad rows / E / ld", w);
@@ -201,7 +199,12 @@ csa_status csa_topk(const float *scores, int64_t rows, int64_t E, int64_t ld,
     REQUIRE(m >= 1, CSA_ERR_INVALID_ARG, "%s: m must be >= 1", w);
     unsigned *err = err_word();
     REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
-    csa::TopkArgs a{scores, rows, E, ld, q_pos, m, k, idx};
+    const size_t need = csa::topk_workspace_size(rows, E, k);
+    REQUIRE(ws_bytes >= need && (need == 0 || workspace), CSA_ERR_INVALID_ARG,
+            "%s: workspace of %zu bytes required", w, need);
+    REQUIRE(((uintptr_t)workspace & 255u) == 0, CSA_ERR_INVALID_ARG,
+            "%s: workspace must be 256-byte aligned", w);
+    csa::TopkArgs a{scores, rows, E, ld, q_pos, m, k, idx, workspace};
     return launched(csa::launch_topk(a, err, (cudaStream_t)stream), w);
 }
 

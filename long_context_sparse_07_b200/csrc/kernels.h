@@ -38,8 +38,10 @@ struct TopkArgs {
     const int64_t *q_pos;
     int m, k;
     int32_t *idx;
+    void *ws;
 };
 cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s);
+size_t topk_workspace_size(int64_t rows, int64_t E, int k);
 
 struct AttendArgs {
     const void *q;

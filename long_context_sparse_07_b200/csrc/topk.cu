@@ -48,27 +48,30 @@ __device__ __forceinline__ unsigned block_rank(bool flag, Shared &sh, unsigned *
     return before + in_warp;
 }
 
-__global__ void __launch_bounds__(kThreads)
-topk_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
-            const int64_t *__restrict__ q_pos, int m, int k, int32_t *__restrict__ idx,
-            int resident)
-{
-    extern __shared__ uint32_t keys[];
-    __shared__ Shared sh;
-    const int64_t row = blockIdx.x;
-    const int64_t V = visible(q_pos[row], m, E);
-    int32_t *out = idx + row * k;
-    const float *src = scores + row * ld;
+// Source of one row: order-preserving key and the index it reports.
+struct RowScores {
+    const float *src;
+    __device__ __forceinline__ uint32_t key(int64_t p) const { return float_key(src[p]); }
+    __device__ __forceinline__ int32_t index(int64_t p) const { return (int32_t)p; }
+};
 
-    if (V <= k) {
-        for (int j = threadIdx.x; j < k; j += kThreads)
-            out[j] = j < V ? j : -1;
-        return;
-    }
-    const bool res = resident && V <= kResident;
+struct RowCandidates {
+    const uint32_t *keys;
+    const int32_t *idx;
+    __device__ __forceinline__ uint32_t key(int64_t p) const { return keys[p]; }
+    __device__ __forceinline__ int32_t index(int64_t p) const { return idx[p]; }
+};
+
+// Top-k of positions [0, V) of `src` (V > k) by (key descending, position
+// ascending), written to out[0..k) in position order. Positions must be in
+// ascending order of the index they report, so ties go to lower indices.
+template <typename Src>
+__device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restrict__ out,
+                             uint32_t *keys, bool res, Shared &sh)
+{
     if (res) {
         for (int64_t s = threadIdx.x; s < V; s += kThreads)
-            keys[s] = float_key(src[s]);
+            keys[s] = src.key(s);
         __syncthreads();
     }
 
@@ -83,7 +86,7 @@ topk_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
         }
         __syncthreads();
         for (int64_t s = threadIdx.x; s < V; s += kThreads) {
-            const uint32_t u = res ? keys[s] : float_key(src[s]);
+            const uint32_t u = res ? keys[s] : src.key(s);
             if ((u & pmask) == prefix)
                 atomicAdd(&sh.hist[(u >> shift) & 255u], 1u);
         }
@@ -125,14 +128,14 @@ topk_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
         __syncthreads();
     }
 
-    // compaction in index order
+    // compaction in position order
     const uint32_t T = prefix;
     unsigned base = 0, eq_seen = 0;
     for (int64_t c0 = 0; c0 < V; c0 += kThreads) {
         const int64_t s = c0 + threadIdx.x;
         uint32_t u = 0;
         if (s < V)
-            u = res ? keys[s] : float_key(src[s]);
+            u = res ? keys[s] : src.key(s);
         const bool gt = s < V && u > T;
         const bool eq = s < V && u == T;
         unsigned eq_tot, take_tot;
@@ -140,12 +143,235 @@ topk_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
         const bool take = gt || (eq && eq_seen + eq_rank < need);
         const unsigned pos = block_rank(take, sh, &take_tot);
         if (take && base + pos < (unsigned)k)
-            out[base + pos] = (int32_t)s;
+            out[base + pos] = src.index(s);
         base += take_tot;
         eq_seen += eq_tot;
     }
     for (int j = (int)base + threadIdx.x; j < k; j += kThreads)
         out[j] = -1;
+}
+
+__global__ void __launch_bounds__(kThreads)
+topk_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
+            const int64_t *__restrict__ q_pos, int m, int k, int32_t *__restrict__ idx,
+            int resident)
+{
+    extern __shared__ uint32_t keys[];
+    __shared__ Shared sh;
+    const int64_t row = blockIdx.x;
+    const int64_t V = visible(q_pos[row], m, E);
+    int32_t *out = idx + row * k;
+    if (V <= k) {
+        for (int j = threadIdx.x; j < k; j += kThreads)
+            out[j] = j < V ? j : -1;
+        return;
+    }
+    RowScores src{scores + row * ld};
+    block_select(src, V, k, out, keys, resident && V <= kResident, sh);
+}
+
+// ---------------------------------------------------------------------------
+// Long rows (many entries, few rows: decode): the row is cut into chunks of
+// kChunk entries handled by separate blocks, in four launches:
+//   1. per-chunk histograms of the top 12 key bits;
+//   2. per row: the bin b that holds the k-th largest key, and for each chunk
+//      the offset of its candidates (keys in bins >= b) in index order;
+//   3. per chunk: the candidates (key, index) compacted to those offsets;
+//   4. per row: the exact block radix select over the candidates.
+// Scratch (caller workspace): histograms, offsets and candidate lists.
+
+constexpr int64_t kChunk = 8192;
+constexpr int kBins = 4096;
+constexpr int64_t kMultiMinE = 65536;
+
+struct MultiWs {
+    uint32_t *hist;      // [rows][nchunks][kBins]
+    uint32_t *off;       // [rows][nchunks + 2]: candidate offsets, total, threshold bin
+    uint32_t *ckey;      // [rows][E]
+    int32_t *cidx;       // [rows][E]
+};
+
+__host__ __device__ inline MultiWs multi_ws(void *base, int64_t rows, int64_t E)
+{
+    const int64_t nchunks = (E + kChunk - 1) / kChunk;
+    MultiWs w;
+    char *p = (char *)base;
+    w.hist = (uint32_t *)p;
+    p += rows * nchunks * kBins * sizeof(uint32_t);
+    w.off = (uint32_t *)p;
+    p += ((rows * (nchunks + 2) * sizeof(uint32_t) + 255) / 256) * 256;
+    w.ckey = (uint32_t *)p;
+    p += rows * E * sizeof(uint32_t);
+    w.cidx = (int32_t *)p;
+    return w;
+}
+
+__global__ void __launch_bounds__(256)
+topk_hist_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
+                 const int64_t *__restrict__ q_pos, int m, int k, MultiWs w)
+{
+    __shared__ uint32_t hist[kBins];
+    const int64_t row = blockIdx.y, c = blockIdx.x;
+    const int64_t nchunks = gridDim.x;
+    const int64_t V = visible(q_pos[row], m, E);
+    for (int b = threadIdx.x; b < kBins; b += blockDim.x)
+        hist[b] = 0;
+    __syncthreads();
+    if (V > k) {
+        const float *src = scores + row * ld;
+        const int64_t s1 = (c + 1) * kChunk < V ? (c + 1) * kChunk : V;
+        for (int64_t s = c * kChunk + threadIdx.x; s < s1; s += blockDim.x)
+            atomicAdd(&hist[float_key(src[s]) >> 20], 1u);
+    }
+    __syncthreads();
+    uint32_t *dst = w.hist + (row * nchunks + c) * kBins;
+    for (int b = threadIdx.x; b < kBins; b += blockDim.x)
+        dst[b] = hist[b];
+}
+
+__global__ void __launch_bounds__(1024)
+topk_thresh_kernel(const int64_t *__restrict__ q_pos, int64_t E, int m, int k, int nchunks,
+                   MultiWs w)
+{
+    __shared__ uint32_t tot[kBins];
+    __shared__ uint32_t wsum[32];
+    __shared__ int tbin;
+    const int64_t row = blockIdx.x;
+    const int64_t V = visible(q_pos[row], m, E);
+    uint32_t *off = w.off + row * (nchunks + 2);
+    if (V <= k)
+        return;
+    const uint32_t *h = w.hist + row * (int64_t)nchunks * kBins;
+    for (int b = threadIdx.x; b < kBins; b += blockDim.x) {
+        uint32_t t = 0;
+        for (int c = 0; c < nchunks; c++)
+            t += h[(int64_t)c * kBins + b];
+        tot[b] = t;
+    }
+    __syncthreads();
+    // descending bins: thread i owns bins 4095-4i .. 4092-4i
+    const int i = threadIdx.x;
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < 4; j++)
+        local += tot[kBins - 1 - 4 * i - j];
+    // block inclusive scan of `local` in thread order
+    uint32_t v = local;
+    const int lane = i & 31, wid = i >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o)
+            v += x;
+    }
+    if (lane == 31)
+        wsum[wid] = v;
+    __syncthreads();
+    if (wid == 0) {
+        uint32_t x = wsum[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o)
+                x += y;
+        }
+        wsum[lane] = x;
+    }
+    __syncthreads();
+    const uint32_t incl = v + (wid > 0 ? wsum[wid - 1] : 0u);
+    const uint32_t excl = incl - local;
+    if (excl < (uint32_t)k && (uint32_t)k <= incl) {
+        uint32_t cum = excl;
+        for (int j = 0; j < 4; j++) {
+            const int b = kBins - 1 - 4 * i - j;
+            cum += tot[b];
+            if (cum >= (uint32_t)k) {
+                tbin = b;
+                break;
+            }
+        }
+    }
+    __syncthreads();
+    const int b0 = tbin;
+    // candidates of each chunk: keys in bins >= b0; exclusive offsets in chunk order
+    if (threadIdx.x < 32) {
+        uint32_t run = 0;
+        for (int c0 = 0; c0 < nchunks; c0 += 32) {
+            const int c = c0 + lane;
+            uint32_t cnt = 0;
+            if (c < nchunks)
+                for (int b = b0; b < kBins; b++)
+                    cnt += h[(int64_t)c * kBins + b];
+            uint32_t x = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o)
+                    x += y;
+            }
+            if (c < nchunks)
+                off[c] = run + x - cnt;
+            run += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) {
+            off[nchunks] = run;
+            off[nchunks + 1] = (uint32_t)b0;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+topk_collect_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
+                    const int64_t *__restrict__ q_pos, int m, int k, MultiWs w)
+{
+    __shared__ Shared sh;
+    const int64_t row = blockIdx.y, c = blockIdx.x;
+    const int nchunks = gridDim.x;
+    const int64_t V = visible(q_pos[row], m, E);
+    if (V <= k)
+        return;
+    const uint32_t *off = w.off + row * (nchunks + 2);
+    const uint32_t b0 = off[nchunks + 1];
+    uint32_t base = off[c];
+    const float *src = scores + row * ld;
+    uint32_t *ck = w.ckey + row * E;
+    int32_t *ci = w.cidx + row * E;
+    const int64_t s1 = (c + 1) * kChunk < V ? (c + 1) * kChunk : V;
+    for (int64_t c0 = c * kChunk; c0 < s1; c0 += kThreads) {
+        const int64_t s = c0 + threadIdx.x;
+        uint32_t u = 0;
+        bool cand = false;
+        if (s < s1) {
+            u = float_key(src[s]);
+            cand = (u >> 20) >= b0;
+        }
+        unsigned tot;
+        const unsigned pos = block_rank(cand, sh, &tot);
+        if (cand) {
+            ck[base + pos] = u;
+            ci[base + pos] = (int32_t)s;
+        }
+        base += tot;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+topk_final_kernel(const int64_t *__restrict__ q_pos, int64_t E, int m, int k, int nchunks,
+                  MultiWs w, int32_t *__restrict__ idx)
+{
+    extern __shared__ uint32_t keys[];
+    __shared__ Shared sh;
+    const int64_t row = blockIdx.x;
+    const int64_t V = visible(q_pos[row], m, E);
+    int32_t *out = idx + row * k;
+    if (V <= k) {
+        for (int j = threadIdx.x; j < k; j += kThreads)
+            out[j] = j < V ? j : -1;
+        return;
+    }
+    const int64_t C = w.off[row * (nchunks + 2) + nchunks];
+    RowCandidates src{w.ckey + row * E, w.cidx + row * E};
+    block_select(src, C, k, out, keys, C <= kResident, sh);
 }
 
 // ---------------------------------------------------------------------------
@@ -256,6 +482,16 @@ topk_warp_kernel(const float *__restrict__ scores, int64_t rows, int64_t E, int6
 
 }  // namespace
 
+size_t topk_workspace_size(int64_t rows, int64_t E, int k)
+{
+    (void)k;
+    if (E < kMultiMinE || rows > 65535 || rows <= 0)
+        return 0;
+    const int64_t nchunks = (E + kChunk - 1) / kChunk;
+    return (size_t)rows * nchunks * kBins * 4 +
+           ((size_t)rows * (nchunks + 2) * 4 + 255) / 256 * 256 + (size_t)rows * E * 8;
+}
+
 cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s)
 {
     (void)err;
@@ -274,11 +510,25 @@ cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s)
                 a.scores, a.rows, a.E, a.ld, a.q_pos, a.m, a.k, a.idx);
         return cudaGetLastError();
     }
+    cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kResident * (int)sizeof(uint32_t));
+    if (topk_workspace_size(a.rows, a.E, a.k) > 0) {
+        const int nchunks = (int)((a.E + kChunk - 1) / kChunk);
+        const MultiWs w = multi_ws(a.ws, a.rows, a.E);
+        topk_hist_kernel<<<dim3(nchunks, (unsigned)a.rows), 256, 0, s>>>(a.scores, a.E, a.ld,
+                                                                         a.q_pos, a.m, a.k, w);
+        topk_thresh_kernel<<<(unsigned)a.rows, 1024, 0, s>>>(a.q_pos, a.E, a.m, a.k, nchunks, w);
+        topk_collect_kernel<<<dim3(nchunks, (unsigned)a.rows), kThreads, 0, s>>>(
+            a.scores, a.E, a.ld, a.q_pos, a.m, a.k, w);
+        cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kResident * (int)sizeof(uint32_t));
+        topk_final_kernel<<<(unsigned)a.rows, kThreads, kResident * sizeof(uint32_t), s>>>(
+            a.q_pos, a.E, a.m, a.k, nchunks, w, a.idx);
+        return cudaGetLastError();
+    }
     const int resident = a.E > a.k;
     const int64_t cap = a.E < kResident ? a.E : kResident;
     const size_t smem = resident ? (size_t)cap * sizeof(uint32_t) : 0;
-    cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kResident * (int)sizeof(uint32_t));
     topk_kernel<<<(unsigned)a.rows, kThreads, smem, s>>>(a.scores, a.E, a.ld, a.q_pos, a.m,
                                                          a.k, a.idx, resident);
     return cudaGetLastError();

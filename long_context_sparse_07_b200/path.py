@@ -33,8 +33,12 @@ def _dev(ops: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tensor]:
 class CsaPrefill:
     """One causal CSA prefill of a single sequence (batch 1)."""
 
-    launches_per_step = 5
     kind = "csa"
+
+    @property
+    def launches_per_step(self):
+        """Kernels launched by one step (top-k of long rows takes four)."""
+        return 4 + (4 if self.topk_ws is not None else 1)
 
     def __init__(self, w, ops: Dict[str, torch.Tensor], device="cuda"):
         self.w = w
@@ -51,6 +55,8 @@ class CsaPrefill:
             self.kI = Entries(torch.empty(E, w.cI, device=device, dtype=DT[w.idx_dtype]), w.cI)
         self.scores = torch.empty(1, n, E, device=device, dtype=torch.float32)
         self.idx = torch.empty(n, w.k, device=device, dtype=torch.int32)
+        nt = abi.csa_topk_workspace_size(n, E, w.k)
+        self.topk_ws = torch.empty(nt, device=device, dtype=torch.uint8) if nt else None
         self.out = torch.empty(1, n, w.h, c, device=device, dtype=DT[w.dtype])
         self.lse = torch.empty(1, n, w.h, device=device, dtype=torch.float32)
         self.scale = 1.0 / math.sqrt(c)
@@ -74,7 +80,8 @@ class CsaPrefill:
 
     def select(self, stream=None):
         w = self.w
-        abi.csa_topk(self.scores[0], self.q_pos, w.m, w.k, self.idx, w.E, stream=stream)
+        abi.csa_topk(self.scores[0], self.q_pos, w.m, w.k, self.idx, w.E, workspace=self.topk_ws,
+                     stream=stream)
 
     def attend(self, stream=None):
         d, w = self.d, self.w
@@ -144,8 +151,14 @@ class HcaPrefill:
 class Decode:
     """One batched decode step over long CSA and HCA caches."""
 
-    launches_per_step = 4
     kind = "decode"
+
+    @property
+    def launches_per_step(self):
+        """indexer + top-k (4 for long rows) + two attention calls, each with
+        a combine launch when it splits the keys of each query."""
+        return (1 + (4 if self.topk_ws is not None else 1) + (2 if self.ws is not None else 1)
+                + (2 if self.hws is not None else 1))
 
     def __init__(self, w, ops: Dict[str, torch.Tensor], device="cuda"):
         self.w = w
@@ -171,6 +184,8 @@ class Decode:
         self.hlse = torch.empty_like(self.lse)
         self.scale = 1.0 / math.sqrt(w.c)
         maxk = w.k + w.n_win
+        nt = abi.csa_topk_workspace_size(B, self.E, w.k)
+        self.topk_ws = torch.empty(nt, device=device, dtype=torch.uint8) if nt else None
         self.ws = self._workspace(B, w, maxk, device)
         self.hws = self._workspace(B, w, self.E_hca + w.n_win, device)
 
@@ -187,7 +202,7 @@ class Decode:
     def select(self, stream=None):
         w = self.w
         abi.csa_topk(self.scores.view(w.batch, self.E), self.d["q_pos"].view(-1), w.m, w.k,
-                     self.idx, self.E, stream=stream)
+                     self.idx, self.E, workspace=self.topk_ws, stream=stream)
 
     def attend(self, stream=None):
         d, w = self.d, self.w

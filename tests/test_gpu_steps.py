@@ -161,7 +161,9 @@ def _topk_case(rows, E, k, m, pos, seed):
     sc = W.score_rows(seed, rows, E)
     q_pos = torch.as_tensor(pos, dtype=torch.int64)
     idx = torch.full((rows, k), -7, device=DEV, dtype=torch.int32)
-    abi.csa_topk(sc.to(DEV), q_pos.to(DEV), m, k, idx, E)
+    nws = abi.csa_topk_workspace_size(rows, E, k)
+    ws = torch.empty(nws, device=DEV, dtype=torch.uint8) if nws else None
+    abi.csa_topk(sc.to(DEV), q_pos.to(DEV), m, k, idx, E, workspace=ws)
     abi.csa_get_error()
     ref = oracle.topk(sc.double().numpy(), q_pos.numpy(), m, k)
     got = idx.cpu().numpy()
@@ -184,6 +186,24 @@ def test_topk_long_rows_resident_and_streamed():
     # rows of 32768 (staged in shared memory) and 262144 (re-read from L2)
     _topk_case(6, 32768, 1024, 4, [4 * 32768 - 1, 40000, 4 * 30000, 4000, 4 * 32768 - 1, 5], 22)
     _topk_case(3, 262144, 1024, 4, [4 * 262144 - 1] * 3, 23)
+
+
+def test_topk_long_rows_split_over_blocks():
+    # rows past 65536 entries go through the four-launch chunked path with a
+    # caller workspace: candidates of the threshold bin across chunk borders,
+    # short rows (V <= k) mixed in, and a row with massive ties
+    rows, E, k = 5, 100000, 700
+    pos = [E - 1, 70000, 500, E - 1, 80000]
+    _topk_case(rows, E, k, 1, pos, 24)
+    sc = torch.zeros(2, E)
+    sc[1, ::3] = 1.0
+    q_pos = torch.tensor([E - 1, E - 1], dtype=torch.int64)
+    idx = torch.empty(2, k, device=DEV, dtype=torch.int32)
+    ws = torch.empty(abi.csa_topk_workspace_size(2, E, k), device=DEV, dtype=torch.uint8)
+    abi.csa_topk(sc.to(DEV), q_pos.to(DEV), 1, k, idx, E, workspace=ws)
+    abi.csa_get_error()
+    ref = oracle.topk(sc.double().numpy(), q_pos.numpy(), 1, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
 
 
 def test_topk_all_equal_scores_prefers_low_indices():
