@@ -41,7 +41,7 @@ namespace {
 
 constexpr int DIM = 512;
 constexpr int KT = 128;
-constexpr float kLazy = 8.f;
+constexpr float kLazy2 = 11.5f;     // lazy-rescale margin, base-2 units (about e^8)
 constexpr int kMmaWarp = 4;
 constexpr int kSoftWarp0 = 5;
 constexpr int kGatherBar = 5;        // named barrier of the 4 gather warps (1..4: head groups)
@@ -68,6 +68,21 @@ struct TcAttn {
     float *lse;
     unsigned *err;
 };
+
+// 2^x and log2(x) from the special-function unit (approximate, about 2 ulp).
+__device__ __forceinline__ float fast_ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float fast_lg2(float x)
+{
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 template <int H>
 struct Lay {
@@ -374,6 +389,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
         }
     } else {
         // ------------------------------------------------------------ softmax / epilogue
+        // Logits are kept in base-2 units, z2 = (q . k) * scale * log2(e), so
+        // every probability is one ex2 of a difference; offsets m2 live in
+        // registers, replicated in every thread of the head group.
+        const float scale2 = a.scale * 1.4426950408889634f;
         const int g = (warp - kSoftWarp0) >> 2;         // head group: heads h0 .. h0+15
         const int h0 = 16 * g;
         const int gbar = 1 + g;
@@ -386,13 +405,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
         for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++qctr) {
             const int64_t bt = w / a.nchunks;
             const QInfo q = query_info(a, bt, (int)(w % a.nchunks));
-            if (et < 16)
-                m_run[h0 + et] = -INFINITY;
-            float lpart[16];
+            float m2[16], lpart[16];
 #pragma unroll
-            for (int u = 0; u < 16; u++)
+            for (int u = 0; u < 16; u++) {
+                m2[u] = -INFINITY;
                 lpart[u] = 0.f;
-            tc::named_bar_sync(gbar, 128);
+            }
             for (int i = 0; i < q.ntiles; ++i, ++tctr) {
                 int64_t er;
                 const bool valid =
@@ -411,12 +429,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int u = 0; u < 16; u++)
-                        z[u] = valid ? __uint_as_float(rr[u]) * a.scale : -INFINITY;
+                        z[u] = valid ? __uint_as_float(rr[u]) * scale2 : -INFINITY;
                 }
                 bool need = false;
 #pragma unroll
                 for (int u = 0; u < 16; u++)
-                    need |= z[u] > m_run[h0 + u] + kLazy;
+                    need |= z[u] > m2[u] + kLazy2;
                 if (tc::named_bar_or(gbar, 128, need)) {
 #pragma unroll
                     for (int u = 0; u < 16; u++) {
@@ -428,16 +446,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                             red[q4 * H + h0 + u] = v;
                     }
                     tc::named_bar_sync(gbar, 128);
-                    if (et < 16) {
-                        const int hh = h0 + et;
+                    float alpha[16];
+#pragma unroll
+                    for (int u = 0; u < 16; u++) {
+                        const int hh = h0 + u;
                         const float tmax = fmaxf(fmaxf(red[hh], red[H + hh]),
                                                  fmaxf(red[2 * H + hh], red[3 * H + hh]));
-                        const float mo = m_run[hh];
-                        const float mn = fmaxf(mo, tmax);
-                        fin[hh] = (mn == -INFINITY) ? 1.f : __expf(mo - mn);   // rescale factor
-                        m_run[hh] = mn;
+                        const float mn = fmaxf(m2[u], tmax);
+                        alpha[u] = (mn == -INFINITY) ? 1.f : fast_ex2(m2[u] - mn);
+                        m2[u] = mn;
                     }
-                    tc::named_bar_sync(gbar, 128);
+                    tc::named_bar_sync(gbar, 128);          // red is rewritten later
                     if (i > 0) {
                         // O^T of the earlier tiles is complete (S of this tile came after it)
 #pragma unroll 1
@@ -448,26 +467,30 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                             tc::tmem_ld_wait();
 #pragma unroll
                             for (int u = 0; u < 16; u++)
-                                rr[u] = __float_as_uint(__uint_as_float(rr[u]) * fin[h0 + u]);
+                                rr[u] = __float_as_uint(__uint_as_float(rr[u]) * alpha[u]);
                             tc::tmem_st16(ad, rr);
                         }
                         tc::tmem_st_wait();
                     }
 #pragma unroll
                     for (int u = 0; u < 16; u++)
-                        lpart[u] *= fin[h0 + u];
+                        lpart[u] *= alpha[u];
                 }
                 // P^T rows h0..h0+15: 2 blocks of 64 keys, 128-byte swizzle
                 {
                     uint8_t *prow = sP + (r >> 6) * (H * 128) + (r & 7) * 2;
                     const int chunk = (r & 63) >> 3;
 #pragma unroll
-                    for (int u = 0; u < 16; u++) {
+                    for (int u = 0; u < 16; u += 2) {
+                        const float p0 = valid ? fast_ex2(z[u] - m2[u]) : 0.f;
+                        const float p1 = valid ? fast_ex2(z[u + 1] - m2[u + 1]) : 0.f;
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                        const float2 pr = __bfloat1622float2(pb);
+                        lpart[u] += pr.x;
+                        lpart[u + 1] += pr.y;
                         const int hh = h0 + u;
-                        const float p = valid ? __expf(z[u] - m_run[hh]) : 0.f;
-                        const __nv_bfloat16 pb = __float2bfloat16_rn(p);
-                        lpart[u] += __bfloat162float(pb);
-                        *(__nv_bfloat16 *)(prow + hh * 128 + ((chunk ^ (hh & 7)) << 4)) = pb;
+                        *(__nv_bfloat16 *)(prow + hh * 128 + ((chunk ^ (hh & 7)) << 4)) = pb.x;
+                        *(__nv_bfloat16 *)(prow + (hh + 1) * 128 + ((chunk ^ ((hh + 1) & 7)) << 4)) = pb.y;
                     }
                 }
                 tc::fence_async_shared();
@@ -487,37 +510,41 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                     red[q4 * H + h0 + u] = v;
             }
             tc::named_bar_sync(gbar, 128);
-            if (et < 16) {
-                const int hh = h0 + et;
+            float f[16];
+#pragma unroll
+            for (int u = 0; u < 16; u++) {
+                const int hh = h0 + u;
                 const float l = red[hh] + red[H + hh] + red[2 * H + hh] + red[3 * H + hh];
-                const float mo = m_run[hh];
                 if (split) {
-                    // partial result of this key chunk: raw accumulator, its offset and sum
-                    fin[hh] = 1.f;
-                    a.ws_ml[(w * H + hh) * 2] = mo;
-                    a.ws_ml[(w * H + hh) * 2 + 1] = l;
-                } else {
-                    const float zs = a.sink[hh];
-                    float f, lse;
-                    if (zs == INFINITY) {
-                        f = 0.f;
-                        lse = INFINITY;
-                    } else {
-                        const float M = fmaxf(mo, zs);
-                        if (M == -INFINITY) {
-                            f = 0.f;
-                            lse = -INFINITY;
-                        } else {
-                            const float e = __expf(mo - M);
-                            const float den = l * e + __expf(zs - M);
-                            f = e / den;
-                            lse = M + __logf(den);
-                        }
+                    // partial of this key chunk: raw accumulator, offset (natural units), sum
+                    f[u] = 1.f;
+                    if (et == u) {
+                        a.ws_ml[(w * H + hh) * 2] = m2[u] * 0.6931471805599453f;
+                        a.ws_ml[(w * H + hh) * 2 + 1] = l;
                     }
-                    fin[hh] = q.ntiles > 0 ? f : 0.f;
-                    if (a.lse)
-                        a.lse[bt * H + hh] = lse;
+                    continue;
                 }
+                const float zs = a.sink[hh];
+                float fu, lse;
+                if (zs == INFINITY) {
+                    fu = 0.f;
+                    lse = INFINITY;
+                } else {
+                    const float zs2 = zs * 1.4426950408889634f;
+                    const float M2 = fmaxf(m2[u], zs2);
+                    if (M2 == -INFINITY) {
+                        fu = 0.f;
+                        lse = -INFINITY;
+                    } else {
+                        const float e = fast_ex2(m2[u] - M2);
+                        const float den = l * e + fast_ex2(zs2 - M2);
+                        fu = e / den;
+                        lse = (M2 + fast_lg2(den)) * 0.6931471805599453f;
+                    }
+                }
+                f[u] = q.ntiles > 0 ? fu : 0.f;
+                if (et == u && a.lse)
+                    a.lse[bt * H + hh] = lse;
             }
             const bool got = tc::mbar_wait(ofull, qctr & 1, abortv);
             if (tc::named_bar_or(gbar, 128, !got)) {
@@ -525,38 +552,44 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                 break;
             }
             tc::fence_after();
-            if (split) {
-                float *orow = a.ws_o + (w * H) * DIM + r;
 #pragma unroll 1
-                for (int jt = 0; jt < 4; jt++) {
+            for (int jt = 0; jt < 4; jt++) {
+                float o[16];
+                if (q.ntiles > 0) {
                     uint32_t rr[16];
-                    if (q.ntiles > 0) {
-                        tc::tmem_ld16(lane_tm + H + jt * H + h0, rr);
-                        tc::tmem_ld_wait();
-                    }
+                    tc::tmem_ld16(lane_tm + H + jt * H + h0, rr);
+                    tc::tmem_ld_wait();
 #pragma unroll
                     for (int u = 0; u < 16; u++)
-                        orow[(h0 + u) * DIM + jt * 128] = q.ntiles > 0 ? __uint_as_float(rr[u]) : 0.f;
-                }
-            } else {
-                __nv_bfloat16 *orow = a.out + bt * H * DIM + r;
-#pragma unroll 1
-                for (int jt = 0; jt < 4; jt++) {
-                    uint32_t rr[16];
-                    if (q.ntiles > 0) {
-                        tc::tmem_ld16(lane_tm + H + jt * H + h0, rr);
-                        tc::tmem_ld_wait();
-                    }
+                        o[u] = __uint_as_float(rr[u]) * f[u];
+                } else {
 #pragma unroll
-                    for (int u = 0; u < 16; u++) {
-                        const float o = q.ntiles > 0 ? __uint_as_float(rr[u]) * fin[h0 + u] : 0.f;
-                        orow[(h0 + u) * DIM + jt * 128] = __float2bfloat16_rn(o);
+                    for (int u = 0; u < 16; u++)
+                        o[u] = 0.f;
+                }
+                if (split) {
+                    float *orow = a.ws_o + (w * H) * DIM + jt * 128 + r;
+#pragma unroll
+                    for (int u = 0; u < 16; u++)
+                        orow[(h0 + u) * DIM] = o[u];
+                } else {
+                    // lanes r and r^1 swap halves so that each stores bf16 pairs of
+                    // adjacent dims: even lanes heads h0..h0+7, odd lanes h0+8..h0+15
+                    const bool odd = lane & 1;
+                    __nv_bfloat162 *orow = (__nv_bfloat162 *)(a.out + bt * H * DIM + jt * 128 + (r & ~1));
+#pragma unroll
+                    for (int u = 0; u < 8; u++) {
+                        const float mine = odd ? o[u + 8] : o[u];
+                        const float other = __shfl_xor_sync(0xffffffffu, odd ? o[u] : o[u + 8], 1);
+                        const int hh = h0 + (odd ? u + 8 : u);
+                        orow[hh * (DIM / 2)] = odd ? __floats2bfloat162_rn(other, mine)
+                                                   : __floats2bfloat162_rn(mine, other);
                     }
                 }
             }
             tc::fence_before();
             tc::mbar_arrive(ofree);
-            tc::named_bar_sync(gbar, 128);     // fin / red / m_run reused next item
+            tc::named_bar_sync(gbar, 128);     // red reused next item
         }
         if (!ok) {
             *abort_flag = 1;

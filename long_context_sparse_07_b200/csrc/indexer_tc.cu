@@ -288,11 +288,18 @@ cudaError_t launch_one(const IndexerArgs &a, unsigned *err, cudaStream_t s)
     t.m = a.m;
     t.kb = a.cI * esize / 128;
     const int64_t ttiles = (a.n_q + NT - 1) / NT;
-    // few token tiles: split the keys of each tile over several blocks
+    // few token tiles: split the keys of each tile over several blocks, sized
+    // so that all blocks run in one wave (two resident blocks per SM)
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t target = 2 * (int64_t)sms;
     t.key_chunk = a.E;
     t.nchunks = 1;
-    if (ttiles * a.B < 296) {
-        t.key_chunk = 2048;
+    if (ttiles * a.B < target) {
+        const int64_t want = (target + ttiles * a.B - 1) / (ttiles * a.B);
+        const int64_t per = (a.E + want - 1) / want;
+        t.key_chunk = (per + 127) / 128 * 128;
         t.nchunks = (int)((a.E + t.key_chunk - 1) / t.key_chunk);
     }
     t.scores = a.scores;

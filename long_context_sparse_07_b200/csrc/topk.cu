@@ -293,15 +293,25 @@ topk_thresh_kernel(const int64_t *__restrict__ q_pos, int64_t E, int m, int k, i
     }
     __syncthreads();
     const int b0 = tbin;
-    // candidates of each chunk: keys in bins >= b0; exclusive offsets in chunk order
+    // candidates of each chunk (keys in bins >= b0): one warp per chunk sums
+    // its bins, then one warp turns the counts into offsets in chunk order
+    __shared__ uint32_t ccount[1024];
+    for (int c = wid; c < nchunks; c += 32) {
+        uint32_t cnt = 0;
+        for (int b = b0 + lane; b < kBins; b += 32)
+            cnt += h[(int64_t)c * kBins + b];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        if (lane == 0)
+            ccount[c] = cnt;
+    }
+    __syncthreads();
     if (threadIdx.x < 32) {
         uint32_t run = 0;
         for (int c0 = 0; c0 < nchunks; c0 += 32) {
             const int c = c0 + lane;
-            uint32_t cnt = 0;
-            if (c < nchunks)
-                for (int b = b0; b < kBins; b++)
-                    cnt += h[(int64_t)c * kBins + b];
+            const uint32_t cnt = c < nchunks ? ccount[c] : 0u;
             uint32_t x = cnt;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -485,7 +495,7 @@ topk_warp_kernel(const float *__restrict__ scores, int64_t rows, int64_t E, int6
 size_t topk_workspace_size(int64_t rows, int64_t E, int k)
 {
     (void)k;
-    if (E < kMultiMinE || rows > 65535 || rows <= 0)
+    if (E < kMultiMinE || rows > 65535 || rows <= 0 || (E + kChunk - 1) / kChunk > 1024)
         return 0;
     const int64_t nchunks = (E + kChunk - 1) / kChunk;
     return (size_t)rows * nchunks * kBins * 4 +
