@@ -56,6 +56,7 @@ struct TcAttn {
     float *ws_o, *ws_ml;             // partial O [item][H][512] and (m, l) [item][H][2]
     const int32_t *idx;
     int dense, k, m;
+    int tma_ent, tma_win;            // whole-tile TMA boxes available per source
     int64_t E;
     int64_t win_rows;
     const int64_t *win_pos0;
@@ -105,6 +106,7 @@ struct Lay {
 // computed identically by every role.
 struct QInfo {
     int64_t b, t, V, nsel, nwin, w0, wp0, nk;
+    int64_t wbeg;     // first window slot: nsel rounded up to 8 (8-slot groups never mix)
     int ntiles;       // tiles of this item
     int tile0;        // first key tile of this item
 };
@@ -119,7 +121,8 @@ __device__ __forceinline__ QInfo query_info(const TcAttn &a, int64_t bt, int chu
     q.w0 = q.t - a.n_win + 1 < 0 ? 0 : q.t - a.n_win + 1;
     q.nwin = a.n_win > 0 ? q.t - q.w0 + 1 : 0;
     q.wp0 = a.win_pos0 ? a.win_pos0[q.b] : 0;
-    q.nk = q.nsel + q.nwin;
+    q.wbeg = (q.nsel + 7) & ~(int64_t)7;
+    q.nk = q.wbeg + q.nwin;
     const int all = (int)((q.nk + KT - 1) / KT);
     q.tile0 = chunk * a.tpc;
     int end = q.tile0 + a.tpc;
@@ -154,8 +157,8 @@ __device__ __forceinline__ const __nv_bfloat16 *key_row(const TcAttn &a, const Q
             report(a.err, CSA_ERR_BOUNDS, K_ATTEND_TC, (unsigned)bt, (unsigned)s);
         return nullptr;
     }
-    if (j < q.nk) {
-        const int64_t p = q.w0 + (j - q.nsel);
+    if (j >= q.wbeg && j < q.nk) {
+        const int64_t p = q.w0 + (j - q.wbeg);
         const int64_t wr = p - q.wp0;
         if (wr >= 0 && wr < a.win_rows)
             return a.kwin + (q.b * a.win_rows + wr) * DIM;
@@ -167,7 +170,8 @@ __device__ __forceinline__ const __nv_bfloat16 *key_row(const TcAttn &a, const Q
 
 template <int H, bool KV8>
 __global__ void __launch_bounds__(Lay<H>::THREADS, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
+attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ent,
+                 const __grid_constant__ CUtensorMap tm_win, const TcAttn a)
 {
     using L = Lay<H>;
     constexpr int NG = L::NG;
@@ -207,6 +211,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
         tc::fence_mbar_init();
         *abort_flag = 0;
         tc::tma_prefetch_desc(&tm_q);
+        tc::tma_prefetch_desc(&tm_ent);
+        tc::tma_prefetch_desc(&tm_win);
     }
     if (warp == kMmaWarp) {
         tc::tmem_alloc(tmem_slot, L::TMEM_COLS);
@@ -250,9 +256,30 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
             for (int i = 0; i < q.ntiles && ok; ++i, ++tctr) {
                 flush();
                 int64_t er;
-                kptr[gt] = key_row<KV8>(a, q, bt, (int64_t)(q.tile0 + i) * KT + gt, false, &er);
+                const int64_t jt0 = (int64_t)(q.tile0 + i) * KT;
+                const __nv_bfloat16 *kp = key_row<KV8>(a, q, bt, jt0 + gt, false, &er);
+                kptr[gt] = kp;
                 krow[gt] = er;
-                tc::named_bar_sync(kGatherBar, 128);
+                // A tile whose 128 rows are consecutive rows of one bf16 source
+                // (dense entries, a selection that is a run, window positions)
+                // goes by one tiled TMA box per 64-dim slice; any other tile by
+                // per-thread 16-byte copies.
+                int tma_src = 0, tma_row = 0;
+                {
+                    int64_t er0;
+                    const __nv_bfloat16 *p0 = key_row<KV8>(a, q, bt, jt0, false, &er0);
+                    const bool src_ent = jt0 < q.nsel, src_win = jt0 >= q.wbeg;
+                    const bool same = (jt0 + gt < q.nsel) == src_ent && (jt0 + gt >= q.wbeg) == src_win;
+                    bool run = p0 != nullptr && same && kp == p0 + (int64_t)gt * DIM;
+                    const __nv_bfloat16 *base = src_ent ? a.ent : a.kwin;
+                    const int64_t row0 = p0 ? (p0 - base) / DIM : 0;
+                    run = run && row0 <= 0x7fffffff - KT && (src_ent ? a.tma_ent : a.tma_win);
+                    const bool all_run = !tc::named_bar_or(kGatherBar, 128, !run);
+                    if (all_run) {
+                        tma_src = src_ent ? 1 : 2;
+                        tma_row = (int)row0;
+                    }
+                }
                 for (int kb = 0; kb < 8; kb++) {
                     if ((kb & 1) == 0 && tctr > 0) {
                         const bool fr = tc::mbar_wait(&kfree[kb >> 1], (tctr - 1) & 1, abortv);
@@ -260,6 +287,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const TcAttn a)
                             ok = false;
                             break;
                         }
+                    }
+                    if (tma_src != 0) {
+                        if (gt == 0) {
+                            tc::mbar_expect_tx(&kfull[kb], 16384u);
+                            tc::tma_load_2d(sK + kb * 16384, tma_src == 1 ? &tm_ent : &tm_win,
+                                            &kfull[kb], kb * 64, tma_row);
+                        }
+                        tc::cp_async_commit();
+                        ++issued;
+                        if (issued - arrived > kInFlight) {
+                            tc::cp_async_wait_group<kInFlight>();
+                            tc::fence_async_shared();
+                            tc::mbar_arrive(&kfull[arrived & 7]);
+                            ++arrived;
+                        }
+                        continue;
                     }
 #pragma unroll
                     for (int u = 0; u < 8; u++) {
@@ -671,6 +714,22 @@ cudaError_t launch_h(const AttendArgs &a, unsigned *err, cudaStream_t s)
     if (!make_tmap_2d(&tm_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.B * a.n_q * H,
                       DIM, H))
         return cudaErrorInvalidValue;
+    // whole-tile boxes (KT rows) of the bf16 entries and of the window rows,
+    // for tiles that are one run of consecutive rows
+    CUtensorMap tm_ent, tm_win;
+    const uint64_t ent_rows = (uint64_t)a.B * a.E, win_rows = (uint64_t)a.B * a.win_rows;
+    const bool have_ent = !KV8 && ent_rows >= (uint64_t)KT;
+    const bool have_win = a.n_win > 0 && win_rows >= (uint64_t)KT;
+    if (have_ent && !make_tmap_2d(&tm_ent, a.kv.body, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ent_rows,
+                                  DIM, KT))
+        return cudaErrorInvalidValue;
+    if (have_win && !make_tmap_2d(&tm_win, a.kwin, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, win_rows,
+                                  DIM, KT))
+        return cudaErrorInvalidValue;
+    if (!have_ent)
+        tm_ent = have_win ? tm_win : tm_q;
+    if (!have_win)
+        tm_win = tm_ent;
     TcAttn t;
     t.ent = KV8 ? nullptr : (const __nv_bfloat16 *)a.kv.body;
     t.ent8 = KV8 ? (const uint8_t *)a.kv.body : nullptr;
@@ -679,6 +738,8 @@ cudaError_t launch_h(const AttendArgs &a, unsigned *err, cudaStream_t s)
     t.kwin = (const __nv_bfloat16 *)a.kwin;
     t.idx = a.idx;
     t.dense = a.dense;
+    t.tma_ent = have_ent;
+    t.tma_win = have_win;
     t.k = a.k;
     t.m = a.m;
     t.E = a.E;
@@ -708,7 +769,7 @@ cudaError_t launch_h(const AttendArgs &a, unsigned *err, cudaStream_t s)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t items = t.nqueries * t.nchunks;
     const int64_t grid = items < sms ? items : sms;
-    attend_tc_kernel<H, KV8><<<(unsigned)grid, Lay<H>::THREADS, smem, s>>>(tm_q, t);
+    attend_tc_kernel<H, KV8><<<(unsigned)grid, Lay<H>::THREADS, smem, s>>>(tm_q, tm_ent, tm_win, t);
     e = cudaGetLastError();
     if (e != cudaSuccess || t.nchunks == 1)
         return e;

@@ -346,3 +346,17 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
 
 }  // namespace tc
 }  // namespace csa
+
+namespace csa {
+namespace tc {
+
+// Adds `bytes` to the transaction count the current phase of `bar` waits
+// for, without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+}  // namespace tc
+}  // namespace csa
