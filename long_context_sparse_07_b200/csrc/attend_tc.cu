@@ -95,7 +95,7 @@ struct Lay {
     static constexpr size_t PTR_OFF = P_OFF + 2 * H * 128;          // 128 row pointers
     static constexpr size_t ROW_OFF = PTR_OFF + KT * 8;             // 128 fp8 entry rows
     static constexpr size_t F_OFF = ROW_OFF + KT * 8;               // m, red[4], fin
-    static constexpr size_t BAR_OFF = F_OFF + ((6 * H * 4 + 63) / 64) * 64;
+    static constexpr size_t BAR_OFF = F_OFF + ((8 * H * 4 + 63) / 64) * 64;
     static constexpr size_t TOTAL = BAR_OFF + 256;
     static constexpr uint32_t TMEM_COLS = (5 * H <= 128) ? 128 : (5 * H <= 256 ? 256 : 512);
     static constexpr uint32_t IDESC_S = tc::idesc_bf16(128, H, 0, 0);
@@ -184,7 +184,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     int64_t *krow = (int64_t *)(sm + L::ROW_OFF);
     float *m_run = (float *)(sm + L::F_OFF);     // [H]
     float *red = m_run + H;                      // [4][H]
-    float *fin = red + 4 * H;                    // [H]
+    float *sink2 = red + 4 * H;                  // [H] sink logits, base-2 units
+    float *m_new = sink2 + H;                    // [H] offsets after a rescale
+    float *alpha_s = m_new + H;                  // [H] rescale factors
     uint64_t *bars = (uint64_t *)(sm + L::BAR_OFF);
     uint64_t *kfull = bars;          // [8] key block landed (128 gather arrivals)
     uint64_t *kfree = bars + 8;      // [4] block pair consumed by O^T M-tile j
@@ -213,6 +215,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc::tma_prefetch_desc(&tm_q);
         tc::tma_prefetch_desc(&tm_ent);
         tc::tma_prefetch_desc(&tm_win);
+    }
+    for (int hh = tid; hh < H; hh += blockDim.x) {
+        sink2[hh] = a.sink[hh] * 1.4426950408889634f;
+        m_run[hh] = -INFINITY;
     }
     if (warp == kMmaWarp) {
         tc::tmem_alloc(tmem_slot, L::TMEM_COLS);
@@ -304,29 +310,40 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         }
                         continue;
                     }
+                    // fp8 entries: all eight code loads of this block go out
+                    // before any is converted, so their latencies overlap
+                    int64_t er8[8];
+                    uint2 cw[8];
+                    float sc8[8];
+#pragma unroll
+                    for (int u = 0; u < 8; u++) {
+                        const int r = (u * 128 + gt) >> 3, c = gt & 7;
+                        er8[u] = KV8 ? krow[r] : -1;
+                        if (KV8 && kb < 7 && er8[u] >= 0) {
+                            cw[u] = __ldg((const uint2 *)(a.ent8 + er8[u] * 448 + kb * 64 + c * 8));
+                            sc8[u] = __ldg(a.ent_scale + er8[u] * 7 + kb);
+                        }
+                    }
 #pragma unroll
                     for (int u = 0; u < 8; u++) {
                         const int lin = u * 128 + gt;
                         const int r = lin >> 3, c = lin & 7;
                         uint8_t *dst = sK + kb * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
-                        if (KV8 && krow[r] >= 0) {
-                            const int64_t er2 = krow[r];
+                        if (KV8 && er8[u] >= 0) {
                             if (kb < 7) {
                                 // 8 e4m3 codes of one 64-dim scale group -> 8 bf16
-                                const uint2 cw = *(const uint2 *)(a.ent8 + er2 * 448 + kb * 64 + c * 8);
-                                const float sc = a.ent_scale[er2 * 7 + kb];
-                                const uint16_t *c2 = (const uint16_t *)&cw;
+                                const uint16_t *c2 = (const uint16_t *)&cw[u];
                                 __nv_bfloat162 o[4];
 #pragma unroll
                                 for (int e = 0; e < 4; e++) {
                                     const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
                                         (__nv_fp8x2_storage_t)c2[e], __NV_E4M3);
                                     const float2 f = __half22float2(__half2(hr));
-                                    o[e] = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+                                    o[e] = __floats2bfloat162_rn(f.x * sc8[u], f.y * sc8[u]);
                                 }
                                 *(uint4 *)dst = *(const uint4 *)o;
                             } else {
-                                tc::cp_async16(dst, a.ent_rope + er2 * 64 + c * 8, 16u);
+                                tc::cp_async16(dst, a.ent_rope + er8[u] * 64 + c * 8, 16u);
                             }
                         } else {
                             const __nv_bfloat16 *sp = kptr[r];
@@ -361,6 +378,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             uint32_t tctr = 0, qctr = 0;
             bool ok = true;
             const uint32_t sK_a = tc::smem_u32(sK), sQ_a = tc::smem_u32(sQ), sP_a = tc::smem_u32(sP);
+            const uint64_t adS = tc::sdesc_sw128(sK_a), bdS = tc::sdesc_sw128(sQ_a);
+            const uint64_t adO = tc::sdesc_sw128_mn(sK_a, 16384, 1024), bdO = tc::sdesc_sw128(sP_a);
             for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++qctr) {
                 const QInfo q = query_info(a, w / a.nchunks, (int)(w % a.nchunks));
                 bool ofree_done = qctr == 0;
@@ -369,18 +388,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     break;
                 }
                 for (int i = 0; i < q.ntiles; ++i, ++tctr) {
-                    for (int kb = 0; kb < 8 && ok; kb++) {
+                    // descriptors advance by constants: 16 KB per key block and
+                    // H x 128 B per Q block (>> 4), 32 B per 16-dim step (>> 4)
+#pragma unroll 1
+                    for (int kb = 0; kb < 8; kb++) {
                         if (!tc::mbar_wait(&kfull[kb], tctr & 1, abortv)) {
                             ok = false;
                             break;
                         }
                         tc::fence_after();
+                        const uint64_t ad = adS + (uint64_t)(kb * 1024), bd = bdS + (uint64_t)(kb * (H * 8));
+                        tc::mma_f16(tmem, ad, bd, L::IDESC_S, kb != 0);
 #pragma unroll
-                        for (int kk = 0; kk < 4; kk++) {
-                            const uint64_t ad = tc::sdesc_sw128(sK_a + kb * 16384 + kk * 32);
-                            const uint64_t bd = tc::sdesc_sw128(sQ_a + kb * (H * 128) + kk * 32);
-                            tc::mma_f16(tmem, ad, bd, L::IDESC_S, (kb | kk) != 0);
-                        }
+                        for (int kk = 1; kk < 4; kk++)
+                            tc::mma_f16(tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), L::IDESC_S, 1u);
                     }
                     if (!ok)
                         break;
@@ -399,15 +420,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         break;
                     }
                     tc::fence_after();
+                    const uint32_t acc0 = i > 0;
+#pragma unroll 1
                     for (int jt = 0; jt < 4; jt++) {
+                        const uint64_t ad = adO + (uint64_t)(jt * 2048);
+                        const uint32_t d = tmem + H + jt * H;
+                        tc::mma_f16(d, ad, bdO, L::IDESC_O, acc0);
 #pragma unroll
-                        for (int kk = 0; kk < 8; kk++) {
-                            const uint64_t ad = tc::sdesc_sw128_mn(
-                                sK_a + (2 * jt) * 16384 + kk * 2048, 16384, 1024);
-                            const uint64_t bd =
-                                tc::sdesc_sw128(sP_a + (kk >> 2) * (H * 128) + (kk & 3) * 32);
-                            tc::mma_f16(tmem + H + jt * H, ad, bd, L::IDESC_O, (i > 0) || (kk > 0));
-                        }
+                        for (int kk = 1; kk < 8; kk++)
+                            tc::mma_f16(d, ad + (uint64_t)(kk * 128),
+                                        bdO + (uint64_t)((kk >> 2) * (H * 8) + (kk & 3) * 2),
+                                        L::IDESC_O, 1u);
                         tc::mma_commit(&kfree[jt]);
                     }
                 }
@@ -448,12 +471,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++qctr) {
             const int64_t bt = w / a.nchunks;
             const QInfo q = query_info(a, bt, (int)(w % a.nchunks));
-            float m2[16], lpart[16];
+            // running offsets m_run[h0..h0+15] (base 2) start at -inf for every item
+            float lpart[16];
 #pragma unroll
-            for (int u = 0; u < 16; u++) {
-                m2[u] = -INFINITY;
+            for (int u = 0; u < 16; u++)
                 lpart[u] = 0.f;
-            }
             for (int i = 0; i < q.ntiles; ++i, ++tctr) {
                 int64_t er;
                 const bool valid =
@@ -474,6 +496,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     for (int u = 0; u < 16; u++)
                         z[u] = valid ? __uint_as_float(rr[u]) * scale2 : -INFINITY;
                 }
+                float m2[16];
+#pragma unroll
+                for (int u = 0; u < 16; u += 4) {
+                    const float4 mv = *(const float4 *)(m_run + h0 + u);
+                    m2[u] = mv.x;
+                    m2[u + 1] = mv.y;
+                    m2[u + 2] = mv.z;
+                    m2[u + 3] = mv.w;
+                }
                 bool need = false;
 #pragma unroll
                 for (int u = 0; u < 16; u++)
@@ -489,17 +520,28 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             red[q4 * H + h0 + u] = v;
                     }
                     tc::named_bar_sync(gbar, 128);
-                    float alpha[16];
-#pragma unroll
-                    for (int u = 0; u < 16; u++) {
-                        const int hh = h0 + u;
+                    // one thread per head: new offset and the factor for what is summed
+                    float mn = 0.f;
+                    if (et < 16) {
+                        const int hh = h0 + et;
                         const float tmax = fmaxf(fmaxf(red[hh], red[H + hh]),
                                                  fmaxf(red[2 * H + hh], red[3 * H + hh]));
-                        const float mn = fmaxf(m2[u], tmax);
-                        alpha[u] = (mn == -INFINITY) ? 1.f : fast_ex2(m2[u] - mn);
-                        m2[u] = mn;
+                        const float mo = m_run[hh];
+                        mn = fmaxf(mo, tmax);
+                        m_new[hh] = mn;
+                        alpha_s[hh] = (mn == -INFINITY) ? 1.f : fast_ex2(mo - mn);
                     }
-                    tc::named_bar_sync(gbar, 128);          // red is rewritten later
+                    tc::named_bar_sync(gbar, 128);
+                    if (et < 16)
+                        m_run[h0 + et] = mn;
+#pragma unroll
+                    for (int u = 0; u < 16; u += 4) {
+                        const float4 mv = *(const float4 *)(m_new + h0 + u);
+                        m2[u] = mv.x;
+                        m2[u + 1] = mv.y;
+                        m2[u + 2] = mv.z;
+                        m2[u + 3] = mv.w;
+                    }
                     if (i > 0) {
                         // O^T of the earlier tiles is complete (S of this tile came after it)
 #pragma unroll 1
@@ -510,14 +552,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             tc::tmem_ld_wait();
 #pragma unroll
                             for (int u = 0; u < 16; u++)
-                                rr[u] = __float_as_uint(__uint_as_float(rr[u]) * alpha[u]);
+                                rr[u] = __float_as_uint(__uint_as_float(rr[u]) * alpha_s[h0 + u]);
                             tc::tmem_st16(ad, rr);
                         }
                         tc::tmem_st_wait();
                     }
 #pragma unroll
                     for (int u = 0; u < 16; u++)
-                        lpart[u] *= alpha[u];
+                        lpart[u] *= alpha_s[h0 + u];
                 }
                 // P^T rows h0..h0+15: 2 blocks of 64 keys, 128-byte swizzle
                 {
@@ -562,24 +604,24 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     // partial of this key chunk: raw accumulator, offset (natural units), sum
                     f[u] = 1.f;
                     if (et == u) {
-                        a.ws_ml[(w * H + hh) * 2] = m2[u] * 0.6931471805599453f;
+                        a.ws_ml[(w * H + hh) * 2] = m_run[hh] * 0.6931471805599453f;
                         a.ws_ml[(w * H + hh) * 2 + 1] = l;
                     }
                     continue;
                 }
-                const float zs = a.sink[hh];
+                const float zs2 = sink2[hh];
                 float fu, lse;
-                if (zs == INFINITY) {
+                if (zs2 == INFINITY) {
                     fu = 0.f;
                     lse = INFINITY;
                 } else {
-                    const float zs2 = zs * 1.4426950408889634f;
-                    const float M2 = fmaxf(m2[u], zs2);
+                    const float mh = m_run[hh];
+                    const float M2 = fmaxf(mh, zs2);
                     if (M2 == -INFINITY) {
                         fu = 0.f;
                         lse = -INFINITY;
                     } else {
-                        const float e = fast_ex2(m2[u] - M2);
+                        const float e = fast_ex2(mh - M2);
                         const float den = l * e + fast_ex2(zs2 - M2);
                         fu = e / den;
                         lse = (M2 + fast_lg2(den)) * 0.6931471805599453f;
@@ -632,7 +674,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             tc::fence_before();
             tc::mbar_arrive(ofree);
-            tc::named_bar_sync(gbar, 128);     // red reused next item
+            tc::named_bar_sync(gbar, 128);     // red and m_run reused next item
+            if (et < 16)
+                m_run[h0 + et] = -INFINITY;
         }
         if (!ok) {
             *abort_flag = 1;
