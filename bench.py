@@ -154,6 +154,33 @@ def time_steps(p, steps, flush, stream):
     return out, per_kernel
 
 
+def time_steps_graph(p, steps, flush, stream):
+    """time_steps with the step captured once in a CUDA graph and replayed:
+    the graph launches every kernel of the step, so kernels of a few
+    microseconds are timed without host launch gaps between them."""
+    names = [n for n, _ in p.phases()]
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
+    g = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        evs[0].record()
+        for i, (_, f) in enumerate(p.phases()):
+            f(None)
+            evs[i + 1].record()
+    torch.cuda.synchronize()
+    per_kernel = {n: [] for n in names}
+    out = []
+    for _ in range(steps):
+        flush.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        out.append(evs[0].elapsed_time(evs[-1]))
+        for i, n in enumerate(names):
+            per_kernel[n].append(evs[i].elapsed_time(evs[i + 1]))
+    del g
+    return out, per_kernel
+
+
 def time_e2e(p, steps, stream):
     """Same step with inputs copied from pinned host memory and the result
     read back, inside the timed region."""
@@ -243,8 +270,12 @@ def run_ours(args, w):
         torch.cuda.synchronize()
 
     barrier()
+    graph = args.graph == "on" or (args.graph == "auto" and w.kind == "decode")
     with ClockSampler(local) as clk:
-        step_ms, kern_ms = time_steps(p, args.steps, flush, stream)
+        if graph:
+            step_ms, kern_ms = time_steps_graph(p, args.steps, flush, stream)
+        else:
+            step_ms, kern_ms = time_steps(p, args.steps, flush, stream)
     barrier()
     abi.csa_get_error()
     mean_ms = sum(step_ms) / len(step_ms)
@@ -294,6 +325,7 @@ def run_ours(args, w):
                        "h": w.h, "hI": w.hI, "cI": w.cI, "n_win": w.n_win,
                        "indexer_dtype": w.idx_dtype, "batch_per_gpu": w.batch,
                        "l2": "flushed between timed steps (512 MiB write)",
+                       "launch": "CUDA graph replay" if graph else "eager",
                        "parallelism": "dp%d (independent sequences)" % world},
             "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
@@ -376,6 +408,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", default="auto", choices=["auto", "on", "off"],
+                    help="replay the timed step from a CUDA graph (auto: decode only)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

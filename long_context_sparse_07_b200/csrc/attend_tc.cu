@@ -2,26 +2,32 @@
 // 5th-generation tensor cores (CSA Eq. 18-19, HCA Eq. 24-26, Module D).
 //
 // All H heads of a query share one key set, and every key is also its own
-// value. Keys therefore go on the M axis of both contractions:
-//   S^T[key][head]  = sum_d K[key][d] * Q[head][d]        (M = 128 keys, N = H)
-//   O^T[dim][head] += sum_key K[key][dim] * P^T[key][head] (M = 4 x 128 dims, N = H)
-// One 128 x 512 bf16 key tile in shared memory (8 blocks of 64 dims, 128-byte
-// swizzle) is the K-major A operand of the first product and, read along the
-// other axis, the M/N-major A operand of the second. S^T and O^T live in
-// tensor memory (H + 4H columns).
+// value. Keys are taken in tiles of 64, double-buffered in shared memory, and
+// go on the M axis of both contractions:
+//   S^T  M = 128 rows: the tile's 64 keys twice, rows 0-63 with dims 0-255 and
+//        rows 64-127 with dims 256-511; N = 2H columns: Q dims 0-255 for heads
+//        0..H-1, Q dims 256-511 for heads H..2H-1. Row r < 64 of the first H
+//        columns plus row r + 64 of the last H columns is the logit of key r;
+//        the other two quarters are not used. (M stays 128, and the tile is
+//        half the size of a 128-key one, so two fit beside Q.)
+//   O^T[dim][head] += sum_key K[key][dim] P^T[key][head]: M = 128 dims (the
+//        64-dim blocks j and j + 4), N = H, four M-tiles.
+// A tile is 8 slots of 8 KB (64 rows x 128 bytes, 128-byte swizzle); slot 2p
+// holds dims 64p.., slot 2p+1 dims 256 + 64p.., so the 16 KB slot pair p is
+// the K-major A operand of the S^T product for dims {64p.., 256 + 64p..} and,
+// read along the other axis, the M/N-major A operand of O^T M-tile p.
 //
 // Warp roles (one persistent block per SM looping over queries):
-//  * warps 0-3 gather the key rows of each tile (selected entries, or window
-//    rows) with 16-byte cp.async, block by block, keeping up to four 16 KB
-//    blocks in flight per thread; block pair (2j, 2j+1) of the next tile is
-//    refetched as soon as the O^T product of M-tile j has consumed it. One
-//    thread also loads each query's Q with a tiled TMA copy.
-//  * warp 4 allocates tensor memory and issues the MMAs (S^T block by block
-//    as blocks land, then O^T per M-tile), committing to the barriers the
-//    other roles wait on.
-//  * warps 5.. (four per group of 16 heads) own the TMEM lanes (one key, then
-//    one dim, per thread): softmax of each tile into P^T for their heads, and
-//    the normalisation and output of each query.
+//  * warps 0-3 gather each tile into the free buffer: one tiled TMA box per
+//    slot when the 64 keys are consecutive rows of one source, else 16-byte
+//    cp.async per thread (fp8 entries are decoded to bf16 on the way). One
+//    thread also loads each query's Q with tiled TMA copies.
+//  * warp 4 allocates tensor memory and issues the MMAs: the S^T product of a
+//    tile as soon as it has landed and the O^T product of the tile before it
+//    as soon as its probabilities are written, whichever is ready first.
+//  * warps 5.. (four per group of 16 heads) own the TMEM lanes: they add the
+//    two halves of each logit (through shared memory), take the softmax into
+//    P^T for their heads, and normalise and write each query's output.
 // Softmax: the per-head offset m_h is updated lazily -- only when some logit
 // of a tile exceeds m_h + 8 are the tile's maxima of that head group reduced,
 // its O^T columns rescaled in tensor memory and its partial sums rescaled (the
@@ -40,12 +46,11 @@ namespace csa {
 namespace {
 
 constexpr int DIM = 512;
-constexpr int KT = 128;
-constexpr float kLazy2 = 11.5f;     // lazy-rescale margin, base-2 units (about e^8)
+constexpr int KT = 64;               // keys per tile
+constexpr float kLazy2 = 11.5f;      // lazy-rescale margin, base-2 units (about e^8)
 constexpr int kMmaWarp = 4;
 constexpr int kSoftWarp0 = 5;
 constexpr int kGatherBar = 5;        // named barrier of the 4 gather warps (1..4: head groups)
-constexpr int kInFlight = 3;         // 16 KB blocks a gather thread may leave in flight
 
 struct TcAttn {
     const __nv_bfloat16 *ent, *kwin;
@@ -85,20 +90,26 @@ __device__ __forceinline__ float fast_lg2(float x)
     return y;
 }
 
+// slot of 64-dim block kb inside a tile (pairs {p, p + 4} side by side)
+__host__ __device__ constexpr int slot_of(int kb) { return (kb & 3) * 2 + (kb >> 2); }
+
 template <int H>
 struct Lay {
     static constexpr int NG = H / 16;                               // head groups
     static constexpr int THREADS = 32 * (kSoftWarp0 + 4 * NG);
-    static constexpr size_t K_OFF = 0;                              // 8 x 16 KB
-    static constexpr size_t Q_OFF = 8 * 16384;                      // 8 x H x 128
-    static constexpr size_t P_OFF = Q_OFF + 8 * H * 128;            // 2 x H x 128
-    static constexpr size_t PTR_OFF = P_OFF + 2 * H * 128;          // 128 row pointers
-    static constexpr size_t ROW_OFF = PTR_OFF + KT * 8;             // 128 fp8 entry rows
-    static constexpr size_t F_OFF = ROW_OFF + KT * 8;               // m, red[4], fin
+    static constexpr size_t K_OFF = 0;                              // 2 x 64 KB tiles
+    static constexpr size_t Q_OFF = 2 * 65536;                      // 4 pairs x 2H x 128
+    static constexpr size_t P_OFF = Q_OFF + 8 * H * 128;            // H x 128 (64 keys)
+    static constexpr size_t X_OFF = P_OFF + H * 128;                // NG x 8 x 128 floats
+    static constexpr size_t PTR_OFF = X_OFF + NG * 8 * 128 * 4;     // 64 row pointers
+    static constexpr size_t ROW_OFF = PTR_OFF + KT * 8;             // 64 fp8 entry rows
+    static constexpr size_t F_OFF = ROW_OFF + KT * 8;               // 8 x H floats
     static constexpr size_t BAR_OFF = F_OFF + ((8 * H * 4 + 63) / 64) * 64;
     static constexpr size_t TOTAL = BAR_OFF + 256;
-    static constexpr uint32_t TMEM_COLS = (5 * H <= 128) ? 128 : (5 * H <= 256 ? 256 : 512);
-    static constexpr uint32_t IDESC_S = tc::idesc_bf16(128, H, 0, 0);
+    static constexpr uint32_t S_COLS = 2 * H;                       // per S^T buffer
+    static constexpr uint32_t O_COL = 4 * H;                        // after 2 S^T buffers
+    static constexpr uint32_t TMEM_COLS = (8 * H <= 128) ? 128 : (8 * H <= 256 ? 256 : 512);
+    static constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 2 * H, 0, 0);
     static constexpr uint32_t IDESC_O = tc::idesc_bf16(128, H, 1, 0);
 };
 
@@ -106,7 +117,7 @@ struct Lay {
 // computed identically by every role.
 struct QInfo {
     int64_t b, t, V, nsel, nwin, w0, wp0, nk;
-    int64_t wbeg;     // first window slot: nsel rounded up to 8 (8-slot groups never mix)
+    int64_t wbeg;     // first window slot: nsel rounded up to 8
     int ntiles;       // tiles of this item
     int tile0;        // first key tile of this item
 };
@@ -168,6 +179,21 @@ __device__ __forceinline__ const __nv_bfloat16 *key_row(const TcAttn &a, const Q
     return nullptr;
 }
 
+// 16 e4m3 codes times one scale -> 16 bf16 in two 16-byte chunks.
+__device__ __forceinline__ void decode16(const uint4 &cw, float sc, uint4 *lo, uint4 *hi)
+{
+    const uint16_t *c2 = (const uint16_t *)&cw;
+    __nv_bfloat162 o[8];
+#pragma unroll
+    for (int e = 0; e < 8; e++) {
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)c2[e], __NV_E4M3);
+        const float2 f = __half22float2(__half2(hr));
+        o[e] = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+    }
+    *lo = *(const uint4 *)&o[0];
+    *hi = *(const uint4 *)&o[4];
+}
+
 template <int H, bool KV8>
 __global__ void __launch_bounds__(Lay<H>::THREADS, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ent,
@@ -180,33 +206,38 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint8_t *sK = sm + L::K_OFF;
     uint8_t *sQ = sm + L::Q_OFF;
     uint8_t *sP = sm + L::P_OFF;
+    float *sX = (float *)(sm + L::X_OFF);
     const __nv_bfloat16 **kptr = (const __nv_bfloat16 **)(sm + L::PTR_OFF);
     int64_t *krow = (int64_t *)(sm + L::ROW_OFF);
-    float *m_run = (float *)(sm + L::F_OFF);     // [H]
-    float *red = m_run + H;                      // [4][H]
+    float *m_run = (float *)(sm + L::F_OFF);     // [H] running offsets, base 2
+    float *red = m_run + H;                      // [4][H] per-warp maxima / sums
     float *sink2 = red + 4 * H;                  // [H] sink logits, base-2 units
     float *m_new = sink2 + H;                    // [H] offsets after a rescale
     float *alpha_s = m_new + H;                  // [H] rescale factors
     uint64_t *bars = (uint64_t *)(sm + L::BAR_OFF);
-    uint64_t *kfull = bars;          // [8] key block landed (128 gather arrivals)
-    uint64_t *kfree = bars + 8;      // [4] block pair consumed by O^T M-tile j
-    uint64_t *qfull = bars + 12, *qfree = bars + 13, *sfull = bars + 14, *pfull = bars + 15;
-    uint64_t *ofull = bars + 16, *ofree = bars + 17, *done = bars + 18;
-    uint32_t *tmem_slot = (uint32_t *)(bars + 19);
+    uint64_t *kfull = bars;          // [2] tile landed (128 gather arrivals + TMA bytes)
+    uint64_t *kfree = bars + 2;      // [2] tile consumed by its O^T product
+    uint64_t *sfull = bars + 4;      // [2] S^T product done
+    uint64_t *pfull = bars + 6;      // P^T written (all head groups)
+    uint64_t *odone = bars + 7;      // O^T product of a tile done (one phase per tile)
+    uint64_t *qfull = bars + 8, *qfree = bars + 9;
+    uint64_t *ofull = bars + 10, *ofree = bars + 11, *done = bars + 12;
+    uint32_t *tmem_slot = (uint32_t *)(bars + 13);
     int *abort_flag = (int *)(tmem_slot + 1);
     const int64_t nitems = a.nqueries * a.nchunks;
     const bool split = a.nchunks > 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int i = 0; i < 8; i++)
+        for (int i = 0; i < 2; i++) {
             tc::mbar_init(&kfull[i], 128);
-        for (int i = 0; i < 4; i++)
             tc::mbar_init(&kfree[i], 1);
+            tc::mbar_init(&sfull[i], 1);
+        }
+        tc::mbar_init(pfull, 128 * NG);
+        tc::mbar_init(odone, 1);
         tc::mbar_init(qfull, 1);
         tc::mbar_init(qfree, 1);
-        tc::mbar_init(sfull, 1);
-        tc::mbar_init(pfull, 128 * NG);
         tc::mbar_init(ofull, 1);
         tc::mbar_init(ofree, 128 * NG);
         tc::mbar_init(done, 1);
@@ -235,20 +266,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int gt = tid;                          // 0..127
         const void *zero_src = KV8 ? (a.kwin ? (const void *)a.kwin : (const void *)a.ent8)
                                    : (a.E > 0 ? (const void *)a.ent : (const void *)a.kwin);
-        uint32_t tctr = 0, qctr = 0, issued = 0, arrived = 0;
+        uint32_t t = 0, qctr = 0;
         bool ok = true;
-        // announce every block still in flight: required before any wait on
-        // a barrier that the products of those blocks release
-        auto flush = [&]() {
-            tc::cp_async_wait_group<0>();
-            tc::fence_async_shared();
-            for (; arrived < issued; ++arrived)
-                tc::mbar_arrive(&kfull[arrived & 7]);
-        };
         for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++qctr) {
             const int64_t bt = w / a.nchunks;
             const QInfo q = query_info(a, bt, (int)(w % a.nchunks));
-            flush();
+            // Q buffer free once the previous item's last S^T product is done
             const bool qf = qctr == 0 || tc::mbar_wait(qfree, (qctr - 1) & 1, abortv);
             if (tc::named_bar_or(kGatherBar, 128, !qf)) {
                 ok = false;
@@ -257,194 +280,229 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (gt == 0) {
                 tc::mbar_arrive_expect_tx(qfull, (uint32_t)(H * 1024));
                 for (int kb = 0; kb < 8; kb++)
-                    tc::tma_load_2d(sQ + kb * (H * 128), &tm_q, qfull, kb * 64, (int)(bt * H));
+                    tc::tma_load_2d(sQ + (kb & 3) * (2 * H * 128) + (kb >> 2) * (H * 128), &tm_q,
+                                    qfull, kb * 64, (int)(bt * H));
             }
-            for (int i = 0; i < q.ntiles && ok; ++i, ++tctr) {
-                flush();
-                int64_t er;
-                const int64_t jt0 = (int64_t)(q.tile0 + i) * KT;
-                const __nv_bfloat16 *kp = key_row<KV8>(a, q, bt, jt0 + gt, false, &er);
-                kptr[gt] = kp;
-                krow[gt] = er;
-                // A tile whose 128 rows are consecutive rows of one bf16 source
-                // (dense entries, a selection that is a run, window positions)
-                // goes by one tiled TMA box per 64-dim slice; any other tile by
-                // per-thread 16-byte copies.
-                int tma_src = 0, tma_row = 0;
-                {
-                    int64_t er0;
-                    const __nv_bfloat16 *p0 = key_row<KV8>(a, q, bt, jt0, false, &er0);
-                    const bool src_ent = jt0 < q.nsel, src_win = jt0 >= q.wbeg;
-                    const bool same = (jt0 + gt < q.nsel) == src_ent && (jt0 + gt >= q.wbeg) == src_win;
-                    bool run = p0 != nullptr && same && kp == p0 + (int64_t)gt * DIM;
-                    const __nv_bfloat16 *base = src_ent ? a.ent : a.kwin;
-                    const int64_t row0 = p0 ? (p0 - base) / DIM : 0;
-                    run = run && row0 <= 0x7fffffff - KT && (src_ent ? a.tma_ent : a.tma_win);
-                    const bool all_run = !tc::named_bar_or(kGatherBar, 128, !run);
-                    if (all_run) {
-                        tma_src = src_ent ? 1 : 2;
-                        tma_row = (int)row0;
+            for (int i = 0; i < q.ntiles; ++i, ++t) {
+                const int b = t & 1;
+                uint8_t *kbuf = sK + b * 65536;
+                // buffer b is free once the O^T product of tile t - 2 is done
+                if (t >= 2) {
+                    const bool fr = tc::mbar_wait(&kfree[b], ((t - 2) >> 1) & 1, abortv);
+                    if (tc::named_bar_or(kGatherBar, 128, !fr)) {
+                        ok = false;
+                        break;
                     }
                 }
-                for (int kb = 0; kb < 8; kb++) {
-                    if ((kb & 1) == 0 && tctr > 0) {
-                        const bool fr = tc::mbar_wait(&kfree[kb >> 1], (tctr - 1) & 1, abortv);
-                        if (tc::named_bar_or(kGatherBar, 128, !fr)) {
-                            ok = false;
-                            break;
-                        }
+                const int64_t jt0 = (int64_t)(q.tile0 + i) * KT;
+                // A tile whose 64 rows are consecutive rows of one bf16 source
+                // (dense entries, a selection that is a run, window positions)
+                // goes by one tiled TMA box per slot; any other tile by
+                // per-thread copies.
+                bool run = true;
+                int64_t row0 = 0;
+                const bool src_ent = jt0 < q.nsel;
+                if (gt < KT) {
+                    int64_t er, er0;
+                    const __nv_bfloat16 *kp = key_row<KV8>(a, q, bt, jt0 + gt, true, &er);
+                    kptr[gt] = kp;
+                    krow[gt] = er;
+                    const __nv_bfloat16 *p0 = key_row<KV8>(a, q, bt, jt0, false, &er0);
+                    const bool src_win = jt0 >= q.wbeg;
+                    const bool same = (jt0 + gt < q.nsel) == src_ent && (jt0 + gt >= q.wbeg) == src_win;
+                    run = p0 != nullptr && same && kp == p0 + (int64_t)gt * DIM;
+                    const __nv_bfloat16 *base = src_ent ? a.ent : a.kwin;
+                    row0 = p0 ? (p0 - base) / DIM : 0;
+                    run = run && row0 <= 0x7fffffff - KT && (src_ent ? a.tma_ent : a.tma_win);
+                }
+                const bool all_run = !tc::named_bar_or(kGatherBar, 128, !run);
+                if (all_run) {
+                    if (gt == 0) {
+                        tc::mbar_expect_tx(&kfull[b], 65536u);
+#pragma unroll 1
+                        for (int kb = 0; kb < 8; kb++)
+                            tc::tma_load_2d(kbuf + slot_of(kb) * 8192, src_ent ? &tm_ent : &tm_win,
+                                            &kfull[b], kb * 64, (int)row0);
                     }
-                    if (tma_src != 0) {
-                        if (gt == 0) {
-                            tc::mbar_expect_tx(&kfull[kb], 16384u);
-                            tc::tma_load_2d(sK + kb * 16384, tma_src == 1 ? &tm_ent : &tm_win,
-                                            &kfull[kb], kb * 64, tma_row);
-                        }
-                        tc::cp_async_commit();
-                        ++issued;
-                        if (issued - arrived > kInFlight) {
-                            tc::cp_async_wait_group<kInFlight>();
-                            tc::fence_async_shared();
-                            tc::mbar_arrive(&kfull[arrived & 7]);
-                            ++arrived;
-                        }
-                        continue;
-                    }
-                    // fp8 entries: all eight code loads of this block go out
-                    // before any is converted, so their latencies overlap
-                    int64_t er8[8];
-                    uint2 cw[8];
-                    float sc8[8];
+                } else if (KV8) {
+                    // two threads per row: body bytes [224 * half, +224) as 14
+                    // pieces of 16 codes (each inside one 64-dim scale group),
+                    // decoded to bf16; RoPE dims and bf16 window rows by cp.async
+                    const int row = gt >> 1, half = gt & 1;
+                    const int64_t er = krow[row];
+                    uint8_t *rbase = kbuf + row * 128;
+                    if (er >= 0) {
+#pragma unroll 1
+                        for (int bat = 0; bat < 2; bat++) {
+                            uint4 cw[7];
+                            float sc[7];
 #pragma unroll
-                    for (int u = 0; u < 8; u++) {
-                        const int r = (u * 128 + gt) >> 3, c = gt & 7;
-                        er8[u] = KV8 ? krow[r] : -1;
-                        if (KV8 && kb < 7 && er8[u] >= 0) {
-                            cw[u] = __ldg((const uint2 *)(a.ent8 + er8[u] * 448 + kb * 64 + c * 8));
-                            sc8[u] = __ldg(a.ent_scale + er8[u] * 7 + kb);
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; u++) {
-                        const int lin = u * 128 + gt;
-                        const int r = lin >> 3, c = lin & 7;
-                        uint8_t *dst = sK + kb * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
-                        if (KV8 && er8[u] >= 0) {
-                            if (kb < 7) {
-                                // 8 e4m3 codes of one 64-dim scale group -> 8 bf16
-                                const uint16_t *c2 = (const uint16_t *)&cw[u];
-                                __nv_bfloat162 o[4];
-#pragma unroll
-                                for (int e = 0; e < 4; e++) {
-                                    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
-                                        (__nv_fp8x2_storage_t)c2[e], __NV_E4M3);
-                                    const float2 f = __half22float2(__half2(hr));
-                                    o[e] = __floats2bfloat162_rn(f.x * sc8[u], f.y * sc8[u]);
-                                }
-                                *(uint4 *)dst = *(const uint4 *)o;
-                            } else {
-                                tc::cp_async16(dst, a.ent_rope + er8[u] * 64 + c * 8, 16u);
+                            for (int j = 0; j < 7; j++) {
+                                const int byte = (half * 14 + bat * 7 + j) * 16;
+                                cw[j] = __ldg((const uint4 *)(a.ent8 + er * 448 + byte));
+                                sc[j] = __ldg(a.ent_scale + er * 7 + (byte >> 6));
                             }
-                        } else {
-                            const __nv_bfloat16 *sp = kptr[r];
-                            tc::cp_async16(dst, sp ? (const void *)(sp + kb * 64 + c * 8) : zero_src,
+#pragma unroll
+                            for (int j = 0; j < 7; j++) {
+                                const int byte = (half * 14 + bat * 7 + j) * 16;
+                                const int kb = byte >> 6, c0 = (byte & 63) >> 3;
+                                uint8_t *sb = rbase + slot_of(kb) * 8192;
+                                uint4 lo, hi;
+                                decode16(cw[j], sc[j], &lo, &hi);
+                                *(uint4 *)(sb + ((c0 ^ (row & 7)) << 4)) = lo;
+                                *(uint4 *)(sb + (((c0 + 1) ^ (row & 7)) << 4)) = hi;
+                            }
+                        }
+#pragma unroll
+                        for (int c = half * 4; c < half * 4 + 4; c++)
+                            tc::cp_async16(rbase + slot_of(7) * 8192 + ((c ^ (row & 7)) << 4),
+                                           a.ent_rope + er * 64 + c * 8, 16u);
+                    } else {
+                        const __nv_bfloat16 *sp = kptr[row];
+#pragma unroll 1
+                        for (int kb = half * 4; kb < half * 4 + 4; kb++)
+#pragma unroll
+                            for (int c = 0; c < 8; c++)
+                                tc::cp_async16(rbase + slot_of(kb) * 8192 + ((c ^ (row & 7)) << 4),
+                                               sp ? (const void *)(sp + kb * 64 + c * 8) : zero_src,
+                                               sp ? 16u : 0u);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int kb = 0; kb < 8; kb++) {
+                        uint8_t *sb = kbuf + slot_of(kb) * 8192;
+#pragma unroll
+                        for (int u = 0; u < 4; u++) {
+                            const int row = (u * 128 + gt) >> 3, c = gt & 7;
+                            const __nv_bfloat16 *sp = kptr[row];
+                            tc::cp_async16(sb + row * 128 + ((c ^ (row & 7)) << 4),
+                                           sp ? (const void *)(sp + kb * 64 + c * 8) : zero_src,
                                            sp ? 16u : 0u);
                         }
                     }
-                    tc::cp_async_commit();
-                    ++issued;
-                    if (issued - arrived > kInFlight) {
-                        tc::cp_async_wait_group<kInFlight>();
-                        tc::fence_async_shared();
-                        tc::mbar_arrive(&kfull[arrived & 7]);
-                        ++arrived;
-                    }
                 }
+                tc::cp_async_commit();
+                tc::cp_async_wait_all();
+                tc::fence_async_shared();
+                tc::mbar_arrive(&kfull[b]);
                 tc::named_bar_sync(kGatherBar, 128);     // kptr / krow rewritten next tile
             }
         }
-        flush();
+        tc::cp_async_wait_all();
         if (!ok) {
             *abort_flag = 1;
             report(a.err, CSA_ERR_TIMEOUT, K_ATTEND_TC, blockIdx.x, 0);
         }
-        if (gt == 0 && qctr > 0) {
-            volatile int never = 0;
-            static_cast<void>(tc::mbar_wait(qfull, (qctr - 1) & 1, &never, 200000000ull));
-        }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
         if (lane == 0) {
-            uint32_t tctr = 0, qctr = 0;
-            bool ok = true;
             const uint32_t sK_a = tc::smem_u32(sK), sQ_a = tc::smem_u32(sQ), sP_a = tc::smem_u32(sP);
+            // descriptors advance by constants (byte offsets >> 4)
             const uint64_t adS = tc::sdesc_sw128(sK_a), bdS = tc::sdesc_sw128(sQ_a);
-            const uint64_t adO = tc::sdesc_sw128_mn(sK_a, 16384, 1024), bdO = tc::sdesc_sw128(sP_a);
+            const uint64_t adO = tc::sdesc_sw128_mn(sK_a, 8192, 1024), bdO = tc::sdesc_sw128(sP_a);
+            uint32_t t = 0, qctr = 0;
+            bool ok = true;
+            // the tile whose O^T product is still to be issued
+            bool pend = false, pend_first = false, pend_last = false;
+            uint32_t pend_t = 0, pend_q = 0;
+            auto issue_s = [&](uint32_t ts) {
+                const int b = ts & 1;
+#pragma unroll 1
+                for (int p = 0; p < 4; p++) {
+                    const uint64_t ad = adS + (uint64_t)(b * 4096 + p * 1024);
+                    const uint64_t bd = bdS + (uint64_t)(p * (H * 16));
+                    tc::mma_f16(tmem + b * L::S_COLS, ad, bd, L::IDESC_S, p != 0);
+#pragma unroll
+                    for (int kk = 1; kk < 4; kk++)
+                        tc::mma_f16(tmem + b * L::S_COLS, ad + (uint64_t)(kk * 2),
+                                    bd + (uint64_t)(kk * 2), L::IDESC_S, 1u);
+                }
+                tc::mma_commit(&sfull[b]);
+            };
+            auto issue_o = [&]() {
+                const int b = pend_t & 1;
+                const uint32_t acc0 = pend_first ? 0u : 1u;
+#pragma unroll 1
+                for (int jt = 0; jt < 4; jt++) {
+                    const uint64_t ad = adO + (uint64_t)(b * 4096 + jt * 1024);
+                    const uint32_t d = tmem + L::O_COL + jt * H;
+                    tc::mma_f16(d, ad, bdO, L::IDESC_O, acc0);
+#pragma unroll
+                    for (int kk = 1; kk < 4; kk++)
+                        tc::mma_f16(d, ad + (uint64_t)(kk * 128), bdO + (uint64_t)(kk * 2),
+                                    L::IDESC_O, 1u);
+                }
+                tc::mma_commit(&kfree[b]);
+                tc::mma_commit(odone);
+                if (pend_last)
+                    tc::mma_commit(ofull);
+                pend = false;
+            };
+            // O^T of the first tile of item pend_q overwrites the accumulator:
+            // the epilogue of item pend_q - 1 must have read it
+            auto o_ready = [&]() {
+                if (!tc::mbar_test_wait(pfull, pend_t & 1))
+                    return false;
+                return !pend_first || pend_q == 0 || tc::mbar_test_wait(ofree, (pend_q - 1) & 1);
+            };
+            // Issues S^T of tile ts (when wanted) and the pending O^T product,
+            // each as soon as its inputs are ready. Bounded in time.
+            auto advance = [&](bool want_s, uint32_t ts) -> bool {
+                const uint64_t t0 = tc::global_ns();
+                for (uint32_t it = 1;; ++it) {
+                    if (want_s && tc::mbar_test_wait(&kfull[ts & 1], (ts >> 1) & 1)) {
+                        tc::fence_after();
+                        issue_s(ts);
+                        want_s = false;
+                    }
+                    if (pend && o_ready()) {
+                        tc::fence_after();
+                        issue_o();
+                    }
+                    if (!want_s && !pend)
+                        return true;
+                    if ((it & 255u) == 0u && (*abortv || tc::global_ns() - t0 > 2000000000ull))
+                        return false;
+                }
+            };
             for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++qctr) {
                 const QInfo q = query_info(a, w / a.nchunks, (int)(w % a.nchunks));
-                bool ofree_done = qctr == 0;
                 if (!tc::mbar_wait(qfull, qctr & 1, abortv)) {
                     ok = false;
                     break;
                 }
-                for (int i = 0; i < q.ntiles; ++i, ++tctr) {
-                    // descriptors advance by constants: 16 KB per key block and
-                    // H x 128 B per Q block (>> 4), 32 B per 16-dim step (>> 4)
-#pragma unroll 1
-                    for (int kb = 0; kb < 8; kb++) {
-                        if (!tc::mbar_wait(&kfull[kb], tctr & 1, abortv)) {
-                            ok = false;
-                            break;
-                        }
-                        tc::fence_after();
-                        const uint64_t ad = adS + (uint64_t)(kb * 1024), bd = bdS + (uint64_t)(kb * (H * 8));
-                        tc::mma_f16(tmem, ad, bd, L::IDESC_S, kb != 0);
-#pragma unroll
-                        for (int kk = 1; kk < 4; kk++)
-                            tc::mma_f16(tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), L::IDESC_S, 1u);
-                    }
-                    if (!ok)
+                if (q.ntiles == 0) {
+                    // no keys: finish the pending product, then hand an (unused)
+                    // O^T to this item's epilogue once the previous one has read it
+                    if (pend && !advance(false, 0)) {
+                        ok = false;
                         break;
-                    tc::mma_commit(sfull);
+                    }
+                    if (qctr > 0 && !tc::mbar_wait(ofree, (qctr - 1) & 1, abortv)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::mma_commit(qfree);
+                    tc::mma_commit(ofull);
+                    continue;
+                }
+                for (int i = 0; i < q.ntiles; ++i, ++t) {
+                    // S^T of tile t (its Q is resident) and O^T of tile t - 1
+                    if (!advance(true, t)) {
+                        ok = false;
+                        break;
+                    }
                     if (i == q.ntiles - 1)
                         tc::mma_commit(qfree);
-                    if (!ofree_done) {
-                        if (!tc::mbar_wait(ofree, (qctr - 1) & 1, abortv)) {
-                            ok = false;
-                            break;
-                        }
-                        ofree_done = true;
-                    }
-                    if (!tc::mbar_wait(pfull, tctr & 1, abortv)) {
-                        ok = false;
-                        break;
-                    }
-                    tc::fence_after();
-                    const uint32_t acc0 = i > 0;
-#pragma unroll 1
-                    for (int jt = 0; jt < 4; jt++) {
-                        const uint64_t ad = adO + (uint64_t)(jt * 2048);
-                        const uint32_t d = tmem + H + jt * H;
-                        tc::mma_f16(d, ad, bdO, L::IDESC_O, acc0);
-#pragma unroll
-                        for (int kk = 1; kk < 8; kk++)
-                            tc::mma_f16(d, ad + (uint64_t)(kk * 128),
-                                        bdO + (uint64_t)((kk >> 2) * (H * 8) + (kk & 3) * 2),
-                                        L::IDESC_O, 1u);
-                        tc::mma_commit(&kfree[jt]);
-                    }
+                    pend = true;
+                    pend_t = t;
+                    pend_first = i == 0;
+                    pend_last = i == q.ntiles - 1;
+                    pend_q = qctr;
                 }
-                if (!ok)
-                    break;
-                if (q.ntiles == 0) {
-                    tc::mma_commit(qfree);
-                    if (!ofree_done && !tc::mbar_wait(ofree, (qctr - 1) & 1, abortv)) {
-                        ok = false;
-                        break;
-                    }
-                }
-                tc::mma_commit(ofull);
             }
+            if (ok && pend && !advance(false, 0))
+                ok = false;
             if (!ok) {
                 *abort_flag = 1;
                 report(a.err, CSA_ERR_TIMEOUT, K_ATTEND_TC, blockIdx.x, 1);
@@ -456,76 +514,86 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     } else {
         // ------------------------------------------------------------ softmax / epilogue
         // Logits are kept in base-2 units, z2 = (q . k) * scale * log2(e), so
-        // every probability is one ex2 of a difference; offsets m2 live in
-        // registers, replicated in every thread of the head group.
+        // every probability is one ex2 of a difference.
         const float scale2 = a.scale * 1.4426950408889634f;
         const int g = (warp - kSoftWarp0) >> 2;         // head group: heads h0 .. h0+15
         const int h0 = 16 * g;
         const int gbar = 1 + g;
         const int q4 = warp & 3;
-        const int r = q4 * 32 + lane;                   // key (then dim) of this TMEM lane
+        const int r = q4 * 32 + lane;                   // TMEM lane of this thread
+        const int half = r >> 6;                        // S^T half: dims 0-255 / 256-511
+        const int kidx = r & 63;                        // key of the tile
+        const int hk = h0 + 8 * half;                   // first of the 8 heads kept here
         const int et = (warp - kSoftWarp0 - 4 * g) * 32 + lane;   // 0..127 inside the group
         const uint32_t lane_tm = tmem + ((uint32_t)(q4 * 32) << 16);
-        uint32_t tctr = 0, qctr = 0;
+        float *xg = sX + g * (8 * 128);                 // [8][128] partial logits handed over
+        uint32_t t = 0, qctr = 0;
         bool ok = true;
         for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++qctr) {
             const int64_t bt = w / a.nchunks;
             const QInfo q = query_info(a, bt, (int)(w % a.nchunks));
-            // running offsets m_run[h0..h0+15] (base 2) start at -inf for every item
-            float lpart[16];
+            float lpart[8];
 #pragma unroll
-            for (int u = 0; u < 16; u++)
+            for (int u = 0; u < 8; u++)
                 lpart[u] = 0.f;
-            for (int i = 0; i < q.ntiles; ++i, ++tctr) {
+            for (int i = 0; i < q.ntiles; ++i, ++t) {
                 int64_t er;
                 const bool valid =
-                    key_row<KV8>(a, q, bt, (int64_t)(q.tile0 + i) * KT + r, g == 0, &er) != nullptr ||
+                    key_row<KV8>(a, q, bt, (int64_t)(q.tile0 + i) * KT + kidx, false, &er) != nullptr ||
                     er >= 0;
-                const bool got = tc::mbar_wait(sfull, tctr & 1, abortv);
+                const bool got = tc::mbar_wait(&sfull[t & 1], (t >> 1) & 1, abortv);
                 if (tc::named_bar_or(gbar, 128, !got)) {
                     ok = false;
                     break;
                 }
                 tc::fence_after();
-                float z[16];
+                float z[8];
                 {
                     uint32_t rr[16];
-                    tc::tmem_ld16(lane_tm + h0, rr);
+                    tc::tmem_ld16(lane_tm + (t & 1) * L::S_COLS + half * H + h0, rr);
                     tc::tmem_ld_wait();
+                    // hand the other half's 8 heads to the partner lane r ^ 64
 #pragma unroll
-                    for (int u = 0; u < 16; u++)
-                        z[u] = valid ? __uint_as_float(rr[u]) * scale2 : -INFINITY;
+                    for (int j = 0; j < 8; j++)
+                        xg[j * 128 + r] = __uint_as_float(half ? rr[j] : rr[8 + j]);
+                    tc::named_bar_sync(gbar, 128);
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        const float mine = __uint_as_float(half ? rr[8 + j] : rr[j]);
+                        z[j] = valid ? (mine + xg[j * 128 + (r ^ 64)]) * scale2 : -INFINITY;
+                    }
                 }
-                float m2[16];
-#pragma unroll
-                for (int u = 0; u < 16; u += 4) {
-                    const float4 mv = *(const float4 *)(m_run + h0 + u);
-                    m2[u] = mv.x;
-                    m2[u + 1] = mv.y;
-                    m2[u + 2] = mv.z;
-                    m2[u + 3] = mv.w;
+                float m8[8];
+                {
+                    const float4 m0 = *(const float4 *)(m_run + hk);
+                    const float4 m1 = *(const float4 *)(m_run + hk + 4);
+                    m8[0] = m0.x; m8[1] = m0.y; m8[2] = m0.z; m8[3] = m0.w;
+                    m8[4] = m1.x; m8[5] = m1.y; m8[6] = m1.z; m8[7] = m1.w;
                 }
                 bool need = false;
 #pragma unroll
-                for (int u = 0; u < 16; u++)
-                    need |= z[u] > m2[u] + kLazy2;
+                for (int j = 0; j < 8; j++)
+                    need |= z[j] > m8[j] + kLazy2;
+                bool o_waited = false;
                 if (tc::named_bar_or(gbar, 128, need)) {
+                    // maxima of this tile: warps 0,1 of the group hold heads
+                    // h0..h0+7, warps 2,3 heads h0+8..h0+15
 #pragma unroll
-                    for (int u = 0; u < 16; u++) {
-                        float v = z[u];
+                    for (int j = 0; j < 8; j++) {
+                        float v = z[j];
 #pragma unroll
                         for (int off = 16; off > 0; off >>= 1)
                             v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
                         if (lane == 0)
-                            red[q4 * H + h0 + u] = v;
+                            red[q4 * H + hk + j] = v;
                     }
                     tc::named_bar_sync(gbar, 128);
                     // one thread per head: new offset and the factor for what is summed
                     float mn = 0.f;
                     if (et < 16) {
                         const int hh = h0 + et;
-                        const float tmax = fmaxf(fmaxf(red[hh], red[H + hh]),
-                                                 fmaxf(red[2 * H + hh], red[3 * H + hh]));
+                        const int qa = et < 8 ? 0 : 2;
+                        const float tmax = fmaxf(red[qa * H + hh], red[(qa + 1) * H + hh]);
                         const float mo = m_run[hh];
                         mn = fmaxf(mo, tmax);
                         m_new[hh] = mn;
@@ -534,20 +602,25 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     tc::named_bar_sync(gbar, 128);
                     if (et < 16)
                         m_run[h0 + et] = mn;
-#pragma unroll
-                    for (int u = 0; u < 16; u += 4) {
-                        const float4 mv = *(const float4 *)(m_new + h0 + u);
-                        m2[u] = mv.x;
-                        m2[u + 1] = mv.y;
-                        m2[u + 2] = mv.z;
-                        m2[u + 3] = mv.w;
+                    {
+                        const float4 m0 = *(const float4 *)(m_new + hk);
+                        const float4 m1 = *(const float4 *)(m_new + hk + 4);
+                        m8[0] = m0.x; m8[1] = m0.y; m8[2] = m0.z; m8[3] = m0.w;
+                        m8[4] = m1.x; m8[5] = m1.y; m8[6] = m1.z; m8[7] = m1.w;
                     }
                     if (i > 0) {
-                        // O^T of the earlier tiles is complete (S of this tile came after it)
+                        // O^T of the tiles before must be complete before rescaling
+                        const bool od = tc::mbar_wait(odone, (t - 1) & 1, abortv);
+                        if (tc::named_bar_or(gbar, 128, !od)) {
+                            ok = false;
+                            break;
+                        }
+                        o_waited = true;
+                        tc::fence_after();
 #pragma unroll 1
                         for (int jt = 0; jt < 4; jt++) {
                             uint32_t rr[16];
-                            const uint32_t ad = lane_tm + H + jt * H + h0;
+                            const uint32_t ad = lane_tm + L::O_COL + jt * H + h0;
                             tc::tmem_ld16(ad, rr);
                             tc::tmem_ld_wait();
 #pragma unroll
@@ -558,24 +631,36 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         tc::tmem_st_wait();
                     }
 #pragma unroll
-                    for (int u = 0; u < 16; u++)
-                        lpart[u] *= alpha_s[h0 + u];
+                    for (int j = 0; j < 8; j++)
+                        lpart[j] *= alpha_s[hk + j];
                 }
-                // P^T rows h0..h0+15: 2 blocks of 64 keys, 128-byte swizzle
-                {
-                    uint8_t *prow = sP + (r >> 6) * (H * 128) + (r & 7) * 2;
-                    const int chunk = (r & 63) >> 3;
+                __nv_bfloat162 pb[4];
 #pragma unroll
-                    for (int u = 0; u < 16; u += 2) {
-                        const float p0 = valid ? fast_ex2(z[u] - m2[u]) : 0.f;
-                        const float p1 = valid ? fast_ex2(z[u + 1] - m2[u + 1]) : 0.f;
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                        const float2 pr = __bfloat1622float2(pb);
-                        lpart[u] += pr.x;
-                        lpart[u + 1] += pr.y;
-                        const int hh = h0 + u;
-                        *(__nv_bfloat16 *)(prow + hh * 128 + ((chunk ^ (hh & 7)) << 4)) = pb.x;
-                        *(__nv_bfloat16 *)(prow + (hh + 1) * 128 + ((chunk ^ ((hh + 1) & 7)) << 4)) = pb.y;
+                for (int j = 0; j < 8; j += 2) {
+                    const float p0 = valid ? fast_ex2(z[j] - m8[j]) : 0.f;
+                    const float p1 = valid ? fast_ex2(z[j + 1] - m8[j + 1]) : 0.f;
+                    pb[j / 2] = __floats2bfloat162_rn(p0, p1);
+                    const float2 pr = __bfloat1622float2(pb[j / 2]);
+                    lpart[j] += pr.x;
+                    lpart[j + 1] += pr.y;
+                }
+                // P^T is free once the O^T product of the previous tile is done
+                if (t > 0 && !o_waited) {
+                    const bool od = tc::mbar_wait(odone, (t - 1) & 1, abortv);
+                    if (tc::named_bar_or(gbar, 128, !od)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                {
+                    // P^T rows hk..hk+7 (one per head, 64 keys, 128-byte swizzle)
+                    uint8_t *pbase = sP + (kidx & 7) * 2;
+                    const int chunk = kidx >> 3;
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        const int hh = hk + j;
+                        const __nv_bfloat16 v = (j & 1) ? pb[j / 2].y : pb[j / 2].x;
+                        *(__nv_bfloat16 *)(pbase + hh * 128 + ((chunk ^ (hh & 7)) << 4)) = v;
                     }
                 }
                 tc::fence_async_shared();
@@ -586,50 +671,61 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 break;
             // ---- end of the item: normaliser, sink, output for heads h0..h0+15
 #pragma unroll
-            for (int u = 0; u < 16; u++) {
-                float v = lpart[u];
+            for (int j = 0; j < 8; j++) {
+                float v = lpart[j];
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1)
                     v += __shfl_xor_sync(0xffffffffu, v, off);
                 if (lane == 0)
-                    red[q4 * H + h0 + u] = v;
+                    red[q4 * H + hk + j] = v;
+            }
+            tc::named_bar_sync(gbar, 128);
+            // one thread per head: the output factor (alpha_s is free here)
+            if (et < 16) {
+                const int hh = h0 + et;
+                const int qa = et < 8 ? 0 : 2;
+                const float l = red[qa * H + hh] + red[(qa + 1) * H + hh];
+                float fh;
+                if (split) {
+                    // partial of this key chunk: raw accumulator, offset (natural units), sum
+                    fh = 1.f;
+                    a.ws_ml[(w * H + hh) * 2] = m_run[hh] * 0.6931471805599453f;
+                    a.ws_ml[(w * H + hh) * 2 + 1] = l;
+                } else {
+                    const float zs2 = sink2[hh];
+                    float lse;
+                    if (zs2 == INFINITY) {
+                        fh = 0.f;
+                        lse = INFINITY;
+                    } else {
+                        const float mh = m_run[hh];
+                        const float M2 = fmaxf(mh, zs2);
+                        if (M2 == -INFINITY) {
+                            fh = 0.f;
+                            lse = -INFINITY;
+                        } else {
+                            const float e = fast_ex2(mh - M2);
+                            const float den = l * e + fast_ex2(zs2 - M2);
+                            fh = e / den;
+                            lse = (M2 + fast_lg2(den)) * 0.6931471805599453f;
+                        }
+                    }
+                    if (q.ntiles == 0)
+                        fh = 0.f;
+                    if (a.lse)
+                        a.lse[bt * H + hh] = lse;
+                }
+                alpha_s[hh] = fh;
             }
             tc::named_bar_sync(gbar, 128);
             float f[16];
 #pragma unroll
-            for (int u = 0; u < 16; u++) {
-                const int hh = h0 + u;
-                const float l = red[hh] + red[H + hh] + red[2 * H + hh] + red[3 * H + hh];
-                if (split) {
-                    // partial of this key chunk: raw accumulator, offset (natural units), sum
-                    f[u] = 1.f;
-                    if (et == u) {
-                        a.ws_ml[(w * H + hh) * 2] = m_run[hh] * 0.6931471805599453f;
-                        a.ws_ml[(w * H + hh) * 2 + 1] = l;
-                    }
-                    continue;
-                }
-                const float zs2 = sink2[hh];
-                float fu, lse;
-                if (zs2 == INFINITY) {
-                    fu = 0.f;
-                    lse = INFINITY;
-                } else {
-                    const float mh = m_run[hh];
-                    const float M2 = fmaxf(mh, zs2);
-                    if (M2 == -INFINITY) {
-                        fu = 0.f;
-                        lse = -INFINITY;
-                    } else {
-                        const float e = fast_ex2(mh - M2);
-                        const float den = l * e + fast_ex2(zs2 - M2);
-                        fu = e / den;
-                        lse = (M2 + fast_lg2(den)) * 0.6931471805599453f;
-                    }
-                }
-                f[u] = q.ntiles > 0 ? fu : 0.f;
-                if (et == u && a.lse)
-                    a.lse[bt * H + hh] = lse;
+            for (int u = 0; u < 16; u += 4) {
+                const float4 fv = *(const float4 *)(alpha_s + h0 + u);
+                f[u] = fv.x;
+                f[u + 1] = fv.y;
+                f[u + 2] = fv.z;
+                f[u + 3] = fv.w;
             }
             const bool got = tc::mbar_wait(ofull, qctr & 1, abortv);
             if (tc::named_bar_or(gbar, 128, !got)) {
@@ -637,12 +733,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 break;
             }
             tc::fence_after();
+            // O^T M-tile jt: lanes 0-63 dims 64 jt.., lanes 64-127 dims 256 + 64 jt..
 #pragma unroll 1
             for (int jt = 0; jt < 4; jt++) {
+                const int d = (half ? 256 : 0) + 64 * jt + kidx;
                 float o[16];
                 if (q.ntiles > 0) {
                     uint32_t rr[16];
-                    tc::tmem_ld16(lane_tm + H + jt * H + h0, rr);
+                    tc::tmem_ld16(lane_tm + L::O_COL + jt * H + h0, rr);
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int u = 0; u < 16; u++)
@@ -653,7 +751,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         o[u] = 0.f;
                 }
                 if (split) {
-                    float *orow = a.ws_o + (w * H) * DIM + jt * 128 + r;
+                    float *orow = a.ws_o + (w * H) * DIM + d;
 #pragma unroll
                     for (int u = 0; u < 16; u++)
                         orow[(h0 + u) * DIM] = o[u];
@@ -661,7 +759,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     // lanes r and r^1 swap halves so that each stores bf16 pairs of
                     // adjacent dims: even lanes heads h0..h0+7, odd lanes h0+8..h0+15
                     const bool odd = lane & 1;
-                    __nv_bfloat162 *orow = (__nv_bfloat162 *)(a.out + bt * H * DIM + jt * 128 + (r & ~1));
+                    __nv_bfloat162 *orow = (__nv_bfloat162 *)(a.out + bt * H * DIM + (d & ~1));
 #pragma unroll
                     for (int u = 0; u < 8; u++) {
                         const float mine = odd ? o[u + 8] : o[u];
