@@ -286,14 +286,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int i = 0; i < q.ntiles; ++i, ++t) {
                 const int b = t & 1;
                 uint8_t *kbuf = sK + b * 65536;
-                // buffer b is free once the O^T product of tile t - 2 is done
-                if (t >= 2) {
-                    const bool fr = tc::mbar_wait(&kfree[b], ((t - 2) >> 1) & 1, abortv);
-                    if (tc::named_bar_or(kGatherBar, 128, !fr)) {
-                        ok = false;
-                        break;
-                    }
-                }
                 const int64_t jt0 = (int64_t)(q.tile0 + i) * KT;
                 // A tile whose 64 rows are consecutive rows of one bf16 source
                 // (dense entries, a selection that is a run, window positions)
@@ -316,6 +308,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     run = run && row0 <= 0x7fffffff - KT && (src_ent ? a.tma_ent : a.tma_win);
                 }
                 const bool all_run = !tc::named_bar_or(kGatherBar, 128, !run);
+                // buffer b is free once the O^T product of tile t - 2 is done
+                // (the row pointers above are worked out before waiting)
+                if (t >= 2) {
+                    const bool fr = tc::mbar_wait(&kfree[b], ((t - 2) >> 1) & 1, abortv);
+                    if (tc::named_bar_or(kGatherBar, 128, !fr)) {
+                        ok = false;
+                        break;
+                    }
+                }
                 if (all_run) {
                     if (gt == 0) {
                         tc::mbar_expect_tx(&kfull[b], 65536u);
@@ -332,6 +333,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const int64_t er = krow[row];
                     uint8_t *rbase = kbuf + row * 128;
                     if (er >= 0) {
+                        // both batches' lines requested from HBM at once
+                        const uint8_t *rp = a.ent8 + er * 448 + half * 224;
+#pragma unroll
+                        for (int off = 0; off < 224; off += 64)
+                            tc::prefetch_l2(rp + off);
 #pragma unroll 1
                         for (int bat = 0; bat < 2; bat++) {
                             uint4 cw[7];
@@ -368,18 +374,24 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                                sp ? 16u : 0u);
                     }
                 } else {
-#pragma unroll 1
-                    for (int kb = 0; kb < 8; kb++) {
-                        uint8_t *sb = kbuf + slot_of(kb) * 8192;
+                    // this thread's 4 rows, read once (a pointer re-read from
+                    // shared memory before every copy would serialise the issue)
+                    const __nv_bfloat16 *sp[4];
+                    uint8_t *dp[4];
 #pragma unroll
-                        for (int u = 0; u < 4; u++) {
-                            const int row = (u * 128 + gt) >> 3, c = gt & 7;
-                            const __nv_bfloat16 *sp = kptr[row];
-                            tc::cp_async16(sb + row * 128 + ((c ^ (row & 7)) << 4),
-                                           sp ? (const void *)(sp + kb * 64 + c * 8) : zero_src,
-                                           sp ? 16u : 0u);
-                        }
+                    for (int u = 0; u < 4; u++) {
+                        const int row = u * 16 + (gt >> 3), c = gt & 7;
+                        const __nv_bfloat16 *p = kptr[row];
+                        sp[u] = p ? p + c * 8 : nullptr;
+                        dp[u] = kbuf + row * 128 + ((c ^ (row & 7)) << 4);
                     }
+#pragma unroll
+                    for (int kb = 0; kb < 8; kb++)
+#pragma unroll
+                        for (int u = 0; u < 4; u++)
+                            tc::cp_async16(dp[u] + slot_of(kb) * 8192,
+                                           sp[u] ? (const void *)(sp[u] + kb * 64) : zero_src,
+                                           sp[u] ? 16u : 0u);
                 }
                 tc::cp_async_commit();
                 tc::cp_async_wait_all();
@@ -756,18 +768,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     for (int u = 0; u < 16; u++)
                         orow[(h0 + u) * DIM] = o[u];
                 } else {
-                    // lanes r and r^1 swap halves so that each stores bf16 pairs of
-                    // adjacent dims: even lanes heads h0..h0+7, odd lanes h0+8..h0+15
-                    const bool odd = lane & 1;
-                    __nv_bfloat162 *orow = (__nv_bfloat162 *)(a.out + bt * H * DIM + (d & ~1));
+                    // this warp's 32 dims x 16 heads go through its 1 KB of the
+                    // group's exchange area as [head][dim], then out as 16-byte
+                    // runs of 8 dims of one head
+                    __nv_bfloat16 *xs = (__nv_bfloat16 *)xg + (et >> 5) * 512;
 #pragma unroll
-                    for (int u = 0; u < 8; u++) {
-                        const float mine = odd ? o[u + 8] : o[u];
-                        const float other = __shfl_xor_sync(0xffffffffu, odd ? o[u] : o[u + 8], 1);
-                        const int hh = h0 + (odd ? u + 8 : u);
-                        orow[hh * (DIM / 2)] = odd ? __floats2bfloat162_rn(other, mine)
-                                                   : __floats2bfloat162_rn(mine, other);
+                    for (int u = 0; u < 16; u++)
+                        xs[u * 32 + lane] = __float2bfloat16_rn(o[u]);
+                    __syncwarp();
+                    const int dbase = d - lane;
+#pragma unroll
+                    for (int c2 = 0; c2 < 2; c2++) {
+                        const int c = lane + 32 * c2, head = c >> 2, part = c & 3;
+                        const uint4 v = *(const uint4 *)(xs + head * 32 + part * 8);
+                        *(uint4 *)(a.out + (bt * H + h0 + head) * DIM + dbase + part * 8) = v;
                     }
+                    __syncwarp();
                 }
             }
             tc::fence_before();

@@ -28,6 +28,29 @@ struct OutDesc {
     csa_dtype dt;
 };
 
+// 16 bytes of T (8 bf16 or 4 f32) as floats.
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4 &u, float *v);
+template <>
+__device__ __forceinline__ void unpack16<float>(const uint4 &u, float *v)
+{
+    v[0] = __uint_as_float(u.x);
+    v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z);
+    v[3] = __uint_as_float(u.w);
+}
+template <>
+__device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4 &u, float *v)
+{
+    const __nv_bfloat162 *h = (const __nv_bfloat162 *)&u;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+        const float2 f = __bfloat1622float2(h[e]);
+        v[2 * e] = f.x;
+        v[2 * e + 1] = f.y;
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 compress_kernel(const T *__restrict__ Ca, const T *__restrict__ Cb, const T *__restrict__ Za,
@@ -57,38 +80,56 @@ compress_kernel(const T *__restrict__ Ca, const T *__restrict__ Cb, const T *__r
     }
     if (live) {
         const int rows = (overlap && i > 0) ? 2 * m : m;
-        for (int r = slice; r < rows; r += split) {
-            const T *cp, *zp;
-            const float *bp;
-            if (r < m) {
-                const int64_t row = (int64_t)m * i + r;
-                cp = Ca + row * c + ch;
-                zp = Za + row * c + ch;
-                bp = Ba + (int64_t)r * c + ch;
-            } else {
-                const int64_t row = (int64_t)m * (i - 1) + (r - m);
-                cp = Cb + row * c + ch;
-                zp = Zb + row * c + ch;
-                bp = Bb + (int64_t)(r - m) * c + ch;
+        // UNR rows of this slice are loaded before any is folded in, so their
+        // memory latencies overlap (16 bytes of C, of Z and VEC bias values each)
+        constexpr int UNR = 4;
+        for (int r0 = slice; r0 < rows; r0 += split * UNR) {
+            uint4 craw[UNR], zraw[UNR];
+            float bv[UNR][VEC];
+#pragma unroll
+            for (int q = 0; q < UNR; q++) {
+                const int r = r0 + q * split;
+                if (r < rows) {
+                    const T *cp, *zp;
+                    const float *bp;
+                    if (r < m) {
+                        const int64_t row = (int64_t)m * i + r;
+                        cp = Ca + row * c + ch;
+                        zp = Za + row * c + ch;
+                        bp = Ba + (int64_t)r * c + ch;
+                    } else {
+                        const int64_t row = (int64_t)m * (i - 1) + (r - m);
+                        cp = Cb + row * c + ch;
+                        zp = Zb + row * c + ch;
+                        bp = Bb + (int64_t)(r - m) * c + ch;
+                    }
+                    craw[q] = __ldg((const uint4 *)cp);
+                    zraw[q] = __ldg((const uint4 *)zp);
+#pragma unroll
+                    for (int v = 0; v < VEC; v += 4)
+                        load4(bp + v, bv[q] + v);
+                }
             }
-            float cv[VEC], zv[VEC], bv[VEC];
-            Vec<T>::load(cp, cv);
-            Vec<T>::load(zp, zv);
 #pragma unroll
-            for (int v = 0; v < VEC; v += 4)
-                load4(bp + v, bv + v);
+            for (int q = 0; q < UNR; q++) {
+                if (r0 + q * split >= rows)
+                    break;
+                float cv[VEC], zv[VEC];
+                unpack16<T>(craw[q], cv);
+                unpack16<T>(zraw[q], zv);
 #pragma unroll
-            for (int v = 0; v < VEC; v++) {
-                const float l = zv[v] + bv[v];
-                if (l > mx[v]) {
-                    const float f = expf(mx[v] - l);
-                    sum[v] = sum[v] * f + 1.f;
-                    acc[v] = acc[v] * f + cv[v];
-                    mx[v] = l;
-                } else {
-                    const float p = expf(l - mx[v]);
-                    sum[v] += p;
-                    acc[v] += p * cv[v];
+                for (int v = 0; v < VEC; v++) {
+                    const float l = zv[v] + bv[q][v];
+                    if (l > mx[v]) {
+                        const float f = expf(mx[v] - l);
+                        sum[v] = sum[v] * f + 1.f;
+                        acc[v] = acc[v] * f + cv[v];
+                        mx[v] = l;
+                    } else {
+                        const float pr = expf(l - mx[v]);
+                        sum[v] += pr;
+                        acc[v] += pr * cv[v];
+                    }
                 }
             }
         }
