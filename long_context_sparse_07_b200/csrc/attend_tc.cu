@@ -333,7 +333,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const int64_t er = krow[row];
                     uint8_t *rbase = kbuf + row * 128;
                     if (er >= 0) {
-                        // both batches' lines requested from HBM at once
+                        // RoPE dims first (asynchronous), and both batches'
+                        // lines requested from HBM at once
+#pragma unroll
+                        for (int c = half * 4; c < half * 4 + 4; c++)
+                            tc::cp_async16(rbase + slot_of(7) * 8192 + ((c ^ (row & 7)) << 4),
+                                           a.ent_rope + er * 64 + c * 8, 16u);
                         const uint8_t *rp = a.ent8 + er * 448 + half * 224;
 #pragma unroll
                         for (int off = 0; off < 224; off += 64)
@@ -359,10 +364,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                 *(uint4 *)(sb + (((c0 + 1) ^ (row & 7)) << 4)) = hi;
                             }
                         }
-#pragma unroll
-                        for (int c = half * 4; c < half * 4 + 4; c++)
-                            tc::cp_async16(rbase + slot_of(7) * 8192 + ((c ^ (row & 7)) << 4),
-                                           a.ent_rope + er * 64 + c * 8, 16u);
                     } else {
                         const __nv_bfloat16 *sp = kptr[row];
 #pragma unroll 1
@@ -807,45 +808,84 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
 // Joins the key chunks of each (query, head): out = sum_c O_c e^{m_c - M} /
 // (sum_c l_c e^{m_c - M} + e^{z' - M}), M = max(max_c m_c, z'), the sink z'
-// entering once here.
+// entering once here. The per-chunk weights are worked out once per block;
+// each thread then owns 4 dims and keeps several chunk loads in flight.
+constexpr int kMaxChunks = 512;
+
 __global__ void __launch_bounds__(128)
 combine_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_ml, int nchunks, int H,
                const float *__restrict__ sink, __nv_bfloat16 *__restrict__ out,
                float *__restrict__ lse)
 {
+    __shared__ float wt[kMaxChunks];
+    __shared__ float red[4];
+    __shared__ float s_M, s_den;
     const int64_t bt = blockIdx.x;
     const int hh = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float *ml = ws_ml + (bt * nchunks * H + hh) * 2;     // chunk c at + c * H * 2
     const float zs = sink[hh];
-    float M = zs;
-    for (int c = 0; c < nchunks; c++)
-        M = fmaxf(M, ws_ml[((bt * nchunks + c) * H + hh) * 2]);
-    float den = 0.f, l_out;
+    float M = -INFINITY;
+    for (int c = tid; c < nchunks; c += 128)
+        M = fmaxf(M, ml[(int64_t)c * H * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0)
+        red[warp] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])), zs);
     const bool zero = zs == INFINITY || M == -INFINITY;
-    if (!zero) {
-        den = __expf(zs - M);
-        for (int c = 0; c < nchunks; c++) {
-            const float *ml = ws_ml + ((bt * nchunks + c) * H + hh) * 2;
-            if (ml[0] != -INFINITY)
-                den += ml[1] * __expf(ml[0] - M);
-        }
-        l_out = M + __logf(den);
-    } else {
-        l_out = zs == INFINITY ? INFINITY : -INFINITY;
+    float part = 0.f;
+    for (int c = tid; c < nchunks; c += 128) {
+        const float mc = ml[(int64_t)c * H * 2];
+        const float wc = (zero || mc == -INFINITY) ? 0.f : __expf(mc - M);
+        wt[c] = wc;
+        part += ml[(int64_t)c * H * 2 + 1] * wc;
     }
-    for (int d = threadIdx.x; d < DIM; d += blockDim.x) {
-        float o = 0.f;
-        if (!zero) {
-            for (int c = 0; c < nchunks; c++) {
-                const float mc = ws_ml[((bt * nchunks + c) * H + hh) * 2];
-                if (mc != -INFINITY)
-                    o += ws_o[((bt * nchunks + c) * H + hh) * DIM + d] * __expf(mc - M);
-            }
-            o /= den;
-        }
-        out[(bt * H + hh) * DIM + d] = __float2bfloat16_rn(o);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        part += __shfl_xor_sync(0xffffffffu, part, o);
+    __syncthreads();                       // red reused, wt complete
+    if (lane == 0)
+        red[warp] = part;
+    __syncthreads();
+    if (tid == 0) {
+        const float den = zero ? 0.f : red[0] + red[1] + red[2] + red[3] + __expf(zs - M);
+        s_den = den;
+        if (lse)
+            lse[bt * H + hh] = zero ? (zs == INFINITY ? INFINITY : -INFINITY) : M + __logf(den);
     }
-    if (threadIdx.x == 0 && lse)
-        lse[bt * H + hh] = l_out;
+    __syncthreads();
+    const float inv = zero ? 0.f : 1.f / s_den;
+    const float *op = ws_o + (bt * nchunks * H + hh) * (int64_t)DIM + tid * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int c = zero ? nchunks : 0;
+    for (; c + 8 <= nchunks; c += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++)
+            v[j] = __ldg((const float4 *)(op + (int64_t)(c + j) * H * DIM));
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const float wc = wt[c + j];
+            acc.x += v[j].x * wc;
+            acc.y += v[j].y * wc;
+            acc.z += v[j].z * wc;
+            acc.w += v[j].w * wc;
+        }
+    }
+    for (; c < nchunks; c++) {
+        const float4 v = __ldg((const float4 *)(op + (int64_t)c * H * DIM));
+        const float wc = wt[c];
+        acc.x += v.x * wc;
+        acc.y += v.y * wc;
+        acc.z += v.z * wc;
+        acc.w += v.w * wc;
+    }
+    __nv_bfloat162 o2[2] = {__floats2bfloat162_rn(acc.x * inv, acc.y * inv),
+                            __floats2bfloat162_rn(acc.z * inv, acc.w * inv)};
+    *(uint2 *)(out + (bt * H + hh) * DIM + tid * 4) = *(const uint2 *)o2;
 }
 
 // Split of each query's key tiles over work items when there are too few

@@ -174,22 +174,30 @@ topk_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
 // Long rows (many entries, few rows: decode): the row is cut into chunks of
 // kChunk entries handled by separate blocks, in four launches:
 //   1. per-chunk histograms of the top 12 key bits;
-//   2. per row: the bin b that holds the k-th largest key, and for each chunk
-//      the offset of its candidates (keys in bins >= b) in index order;
-//   3. per chunk: the candidates (key, index) compacted to those offsets;
-//   4. per row: the exact block radix select over the candidates.
-// Scratch (caller workspace): histograms, offsets and candidate lists.
+//   2. the row's bin totals, a slice of bins per block;
+//   3. per chunk: the bin b that holds the k-th largest key (from the totals,
+//      worked out again by every block), then the chunk's candidates (keys
+//      in bins >= b) compacted in index order into the chunk's own region;
+//   4. per row: the candidate lists joined in chunk order, then the exact
+//      block radix select over them.
+// Scratch (caller workspace): histograms, totals, counts and candidate lists.
 
 constexpr int64_t kChunk = 8192;
 constexpr int kBins = 4096;
 constexpr int64_t kMultiMinE = 65536;
+constexpr int kCollectThreads = 512;
 
 struct MultiWs {
     uint32_t *hist;      // [rows][nchunks][kBins]
-    uint32_t *off;       // [rows][nchunks + 2]: candidate offsets, total, threshold bin
-    uint32_t *ckey;      // [rows][E]
+    uint32_t *tot;       // [rows][kBins]
+    uint32_t *cnt;       // [rows][nchunks] candidates per chunk
+    uint32_t *ckey;      // [rows][E]  chunk c's candidates at c * kChunk
     int32_t *cidx;       // [rows][E]
+    uint32_t *jkey;      // [rows][E]  joined candidate lists
+    int32_t *jidx;       // [rows][E]
 };
+
+__host__ __device__ inline size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
 __host__ __device__ inline MultiWs multi_ws(void *base, int64_t rows, int64_t E)
 {
@@ -197,13 +205,27 @@ __host__ __device__ inline MultiWs multi_ws(void *base, int64_t rows, int64_t E)
     MultiWs w;
     char *p = (char *)base;
     w.hist = (uint32_t *)p;
-    p += rows * nchunks * kBins * sizeof(uint32_t);
-    w.off = (uint32_t *)p;
-    p += ((rows * (nchunks + 2) * sizeof(uint32_t) + 255) / 256) * 256;
+    p += align256(rows * nchunks * kBins * sizeof(uint32_t));
+    w.tot = (uint32_t *)p;
+    p += align256(rows * kBins * sizeof(uint32_t));
+    w.cnt = (uint32_t *)p;
+    p += align256(rows * nchunks * sizeof(uint32_t));
     w.ckey = (uint32_t *)p;
-    p += rows * E * sizeof(uint32_t);
+    p += align256(rows * E * sizeof(uint32_t));
     w.cidx = (int32_t *)p;
+    p += align256(rows * E * sizeof(int32_t));
+    w.jkey = (uint32_t *)p;
+    p += align256(rows * E * sizeof(uint32_t));
+    w.jidx = (int32_t *)p;
     return w;
+}
+
+__host__ __device__ inline size_t multi_ws_bytes(int64_t rows, int64_t E)
+{
+    const int64_t nchunks = (E + kChunk - 1) / kChunk;
+    return align256(rows * nchunks * kBins * sizeof(uint32_t)) +
+           align256(rows * kBins * sizeof(uint32_t)) + align256(rows * nchunks * sizeof(uint32_t)) +
+           4 * align256(rows * E * sizeof(uint32_t));
 }
 
 __global__ void __launch_bounds__(256)
@@ -229,140 +251,115 @@ topk_hist_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
         dst[b] = hist[b];
 }
 
-__global__ void __launch_bounds__(1024)
-topk_thresh_kernel(const int64_t *__restrict__ q_pos, int64_t E, int m, int k, int nchunks,
-                   MultiWs w)
+// Totals of a 256-bin slice of one row (grid: 16 slices x rows).
+__global__ void __launch_bounds__(256)
+topk_total_kernel(int nchunks, MultiWs w)
 {
-    __shared__ uint32_t tot[kBins];
-    __shared__ uint32_t wsum[32];
-    __shared__ int tbin;
-    const int64_t row = blockIdx.x;
-    const int64_t V = visible(q_pos[row], m, E);
-    uint32_t *off = w.off + row * (nchunks + 2);
-    if (V <= k)
-        return;
-    const uint32_t *h = w.hist + row * (int64_t)nchunks * kBins;
-    for (int b = threadIdx.x; b < kBins; b += blockDim.x) {
-        uint32_t t = 0;
-        for (int c = 0; c < nchunks; c++)
-            t += h[(int64_t)c * kBins + b];
-        tot[b] = t;
-    }
-    __syncthreads();
-    // descending bins: thread i owns bins 4095-4i .. 4092-4i
-    const int i = threadIdx.x;
-    uint32_t local = 0;
-#pragma unroll
-    for (int j = 0; j < 4; j++)
-        local += tot[kBins - 1 - 4 * i - j];
-    // block inclusive scan of `local` in thread order
-    uint32_t v = local;
-    const int lane = i & 31, wid = i >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t x = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o)
-            v += x;
-    }
-    if (lane == 31)
-        wsum[wid] = v;
-    __syncthreads();
-    if (wid == 0) {
-        uint32_t x = wsum[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o)
-                x += y;
-        }
-        wsum[lane] = x;
-    }
-    __syncthreads();
-    const uint32_t incl = v + (wid > 0 ? wsum[wid - 1] : 0u);
-    const uint32_t excl = incl - local;
-    if (excl < (uint32_t)k && (uint32_t)k <= incl) {
-        uint32_t cum = excl;
-        for (int j = 0; j < 4; j++) {
-            const int b = kBins - 1 - 4 * i - j;
-            cum += tot[b];
-            if (cum >= (uint32_t)k) {
-                tbin = b;
-                break;
-            }
-        }
-    }
-    __syncthreads();
-    const int b0 = tbin;
-    // candidates of each chunk (keys in bins >= b0): one warp per chunk sums
-    // its bins, then one warp turns the counts into offsets in chunk order
-    __shared__ uint32_t ccount[1024];
-    for (int c = wid; c < nchunks; c += 32) {
-        uint32_t cnt = 0;
-        for (int b = b0 + lane; b < kBins; b += 32)
-            cnt += h[(int64_t)c * kBins + b];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-        if (lane == 0)
-            ccount[c] = cnt;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        uint32_t run = 0;
-        for (int c0 = 0; c0 < nchunks; c0 += 32) {
-            const int c = c0 + lane;
-            const uint32_t cnt = c < nchunks ? ccount[c] : 0u;
-            uint32_t x = cnt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o)
-                    x += y;
-            }
-            if (c < nchunks)
-                off[c] = run + x - cnt;
-            run += __shfl_sync(0xffffffffu, x, 31);
-        }
-        if (lane == 0) {
-            off[nchunks] = run;
-            off[nchunks + 1] = (uint32_t)b0;
-        }
-    }
+    const int64_t row = blockIdx.y;
+    const int b = blockIdx.x * 256 + threadIdx.x;
+    const uint32_t *h = w.hist + row * (int64_t)nchunks * kBins + b;
+    uint32_t t = 0;
+    int c = 0;
+    for (; c + 4 <= nchunks; c += 4)
+        t += h[(int64_t)c * kBins] + h[(int64_t)(c + 1) * kBins] + h[(int64_t)(c + 2) * kBins] +
+             h[(int64_t)(c + 3) * kBins];
+    for (; c < nchunks; c++)
+        t += h[(int64_t)c * kBins];
+    w.tot[row * kBins + b] = t;
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kCollectThreads)
 topk_collect_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
                     const int64_t *__restrict__ q_pos, int m, int k, MultiWs w)
 {
-    __shared__ Shared sh;
+    constexpr int NW = kCollectThreads / 32;
+    constexpr int PER = kChunk / kCollectThreads;       // keys per thread (16)
+    __shared__ uint32_t wsum[NW];
+    __shared__ uint32_t s_b0;
     const int64_t row = blockIdx.y, c = blockIdx.x;
     const int nchunks = gridDim.x;
     const int64_t V = visible(q_pos[row], m, E);
     if (V <= k)
         return;
-    const uint32_t *off = w.off + row * (nchunks + 2);
-    const uint32_t b0 = off[nchunks + 1];
-    uint32_t base = off[c];
-    const float *src = scores + row * ld;
-    uint32_t *ck = w.ckey + row * E;
-    int32_t *ci = w.cidx + row * E;
-    const int64_t s1 = (c + 1) * kChunk < V ? (c + 1) * kChunk : V;
-    for (int64_t c0 = c * kChunk; c0 < s1; c0 += kThreads) {
-        const int64_t s = c0 + threadIdx.x;
-        uint32_t u = 0;
-        bool cand = false;
-        if (s < s1) {
-            u = float_key(src[s]);
-            cand = (u >> 20) >= b0;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    // the bin of the k-th largest key: thread i owns bins 4095-8i .. 4088-8i
+    {
+        const uint32_t *tot = w.tot + row * kBins;
+        uint32_t tb[8], local = 0;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            tb[j] = tot[kBins - 1 - 8 * tid - j];
+            local += tb[j];
         }
-        unsigned tot;
-        const unsigned pos = block_rank(cand, sh, &tot);
-        if (cand) {
-            ck[base + pos] = u;
-            ci[base + pos] = (int32_t)s;
+        uint32_t v = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o)
+                v += x;
         }
-        base += tot;
+        if (lane == 31)
+            wsum[wid] = v;
+        __syncthreads();
+        uint32_t before = 0;
+        for (int j = 0; j < wid; j++)
+            before += wsum[j];
+        const uint32_t incl = v + before, excl = incl - local;
+        if (excl < (uint32_t)k && (uint32_t)k <= incl) {
+            uint32_t cum = excl;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                cum += tb[j];
+                if (cum >= (uint32_t)k) {
+                    s_b0 = (uint32_t)(kBins - 1 - 8 * tid - j);
+                    break;
+                }
+            }
+        }
+        __syncthreads();
     }
+    const uint32_t b0 = s_b0;
+    // warp wid covers entries [c0 + 512 wid, +512) of the chunk, 32 at a time
+    const float *src = scores + row * ld;
+    const int64_t c0 = c * kChunk, s1 = c0 + kChunk < V ? c0 + kChunk : V;
+    const int64_t wbase = c0 + (int64_t)wid * (32 * PER);
+    uint32_t key[PER];
+    uint32_t mine = 0;
+#pragma unroll
+    for (int i = 0; i < PER; i++) {
+        const int64_t sidx = wbase + i * 32 + lane;
+        key[i] = sidx < s1 ? float_key(src[sidx]) : 0u;
+        mine += (sidx < s1 && (key[i] >> 20) >= b0) ? 1u : 0u;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        mine += __shfl_xor_sync(0xffffffffu, mine, o);
+    __syncthreads();                       // wsum reused
+    if (lane == 0)
+        wsum[wid] = mine;
+    __syncthreads();
+    uint32_t base = 0, total = 0;
+    for (int j = 0; j < NW; j++) {
+        base += j < wid ? wsum[j] : 0u;
+        total += wsum[j];
+    }
+    uint32_t *ck = w.ckey + row * E + c0;
+    int32_t *ci = w.cidx + row * E + c0;
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < PER; i++) {
+        const int64_t sidx = wbase + i * 32 + lane;
+        const bool cand = sidx < s1 && (key[i] >> 20) >= b0;
+        const unsigned bal = __ballot_sync(0xffffffffu, cand);
+        if (cand) {
+            const uint32_t pos = base + __popc(bal & lt);
+            ck[pos] = key[i];
+            ci[pos] = (int32_t)sidx;
+        }
+        base += __popc(bal);
+    }
+    if (tid == 0)
+        w.cnt[row * nchunks + c] = total;
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -371,6 +368,7 @@ topk_final_kernel(const int64_t *__restrict__ q_pos, int64_t E, int m, int k, in
 {
     extern __shared__ uint32_t keys[];
     __shared__ Shared sh;
+    __shared__ uint32_t offs[1025];
     const int64_t row = blockIdx.x;
     const int64_t V = visible(q_pos[row], m, E);
     int32_t *out = idx + row * k;
@@ -379,8 +377,43 @@ topk_final_kernel(const int64_t *__restrict__ q_pos, int64_t E, int m, int k, in
             out[j] = j < V ? j : -1;
         return;
     }
-    const int64_t C = w.off[row * (nchunks + 2) + nchunks];
-    RowCandidates src{w.ckey + row * E, w.cidx + row * E};
+    // join the chunks' lists in chunk order (so in index order): offsets by
+    // a warp scan over the counts, then one warp per chunk copies
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (wid == 0) {
+        uint32_t run = 0;
+        for (int c0 = 0; c0 < nchunks; c0 += 32) {
+            const int c = c0 + lane;
+            const uint32_t n = c < nchunks ? w.cnt[row * nchunks + c] : 0u;
+            uint32_t x = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o)
+                    x += y;
+            }
+            if (c < nchunks)
+                offs[c] = run + x - n;
+            run += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0)
+            offs[nchunks] = run;
+    }
+    __syncthreads();
+    const int64_t C = offs[nchunks];
+    uint32_t *jk = w.jkey + row * E;
+    int32_t *ji = w.jidx + row * E;
+    for (int c = wid; c < nchunks; c += kWarps) {
+        const uint32_t o = offs[c], n = offs[c + 1] - o;
+        const uint32_t *sk = w.ckey + row * E + (int64_t)c * kChunk;
+        const int32_t *si = w.cidx + row * E + (int64_t)c * kChunk;
+        for (uint32_t j = lane; j < n; j += 32) {
+            jk[o + j] = sk[j];
+            ji[o + j] = si[j];
+        }
+    }
+    __syncthreads();
+    RowCandidates src{jk, ji};
     block_select(src, C, k, out, keys, C <= kResident, sh);
 }
 
@@ -497,9 +530,7 @@ size_t topk_workspace_size(int64_t rows, int64_t E, int k)
     (void)k;
     if (E < kMultiMinE || rows > 65535 || rows <= 0 || (E + kChunk - 1) / kChunk > 1024)
         return 0;
-    const int64_t nchunks = (E + kChunk - 1) / kChunk;
-    return (size_t)rows * nchunks * kBins * 4 +
-           ((size_t)rows * (nchunks + 2) * 4 + 255) / 256 * 256 + (size_t)rows * E * 8;
+    return multi_ws_bytes(rows, E);
 }
 
 cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s)
@@ -527,8 +558,8 @@ cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s)
         const MultiWs w = multi_ws(a.ws, a.rows, a.E);
         topk_hist_kernel<<<dim3(nchunks, (unsigned)a.rows), 256, 0, s>>>(a.scores, a.E, a.ld,
                                                                          a.q_pos, a.m, a.k, w);
-        topk_thresh_kernel<<<(unsigned)a.rows, 1024, 0, s>>>(a.q_pos, a.E, a.m, a.k, nchunks, w);
-        topk_collect_kernel<<<dim3(nchunks, (unsigned)a.rows), kThreads, 0, s>>>(
+        topk_total_kernel<<<dim3(kBins / 256, (unsigned)a.rows), 256, 0, s>>>(nchunks, w);
+        topk_collect_kernel<<<dim3(nchunks, (unsigned)a.rows), kCollectThreads, 0, s>>>(
             a.scores, a.E, a.ld, a.q_pos, a.m, a.k, w);
         cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kResident * (int)sizeof(uint32_t));
