@@ -1,14 +1,16 @@
 // topk.cu -- top-k selector (Eq. 17): radix select over the visible scores.
 //
-// One block per score row. Scores are mapped to order-preserving 32-bit keys
-// (larger float -> larger key, -0 folded onto +0). Four 8-bit digit passes,
-// most significant first, find the key T of the k-th largest element and how
-// many elements equal to T must be taken (ties prefer lower indices). A final
-// pass in index order writes every element with key > T and the first
-// `need` elements with key == T, so each row comes out in ascending index
-// order. When the visible row fits, its keys are staged once in shared
-// memory and every pass reads them from there; longer rows are re-read from
-// global memory (L2) on each pass.
+// Scores are mapped to order-preserving 32-bit keys (larger float -> larger
+// key, -0 folded onto +0). Radix digits, most significant first, find the key
+// T of the k-th largest element and how many elements equal to T must be
+// taken (ties prefer lower indices). A final pass in index order writes every
+// element with key > T and the first `need` elements with key == T, so each
+// row comes out in ascending index order. Three layouts of the work:
+//  * short rows (<= 2048 visible): one warp per row, keys in registers;
+//  * rows up to 64 K: one block per row, keys staged once in shared memory
+//    when they fit (re-read from L2 otherwise), 12 + 12 + 8-bit digits;
+//  * longer rows (decode): chunks of the row over many blocks, then one block
+//    per row over the candidates of the threshold bin.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -21,38 +23,56 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kResident = 40960;   // keys staged in shared memory (160 KB)
 
 struct Shared {
-    unsigned hist[256];
+    unsigned hist[4096];                 // digit histogram (12 or 8 bits)
     unsigned warp_tot[kWarps];
+    unsigned warp_cnt[2][kWarps];
     unsigned bin, need;
 };
-
-// Exclusive block-wide prefix count of a per-thread flag; returns the
-// thread's rank and writes the block total to *total.
-__device__ __forceinline__ unsigned block_rank(bool flag, Shared &sh, unsigned *total)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned ballot = __ballot_sync(0xffffffffu, flag);
-    const unsigned in_warp = __popc(ballot & ((1u << lane) - 1u));
-    __syncthreads();                       // warp_tot free for reuse
-    if (lane == 0)
-        sh.warp_tot[warp] = __popc(ballot);
-    __syncthreads();
-    unsigned before = 0, tot = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; w++) {
-        const unsigned v = sh.warp_tot[w];
-        before += (w < warp) ? v : 0u;
-        tot += v;
-    }
-    *total = tot;
-    return before + in_warp;
-}
 
 // Source of one row: order-preserving key and the index it reports.
 struct RowScores {
     const float *src;
     __device__ __forceinline__ uint32_t key(int64_t p) const { return float_key(src[p]); }
     __device__ __forceinline__ int32_t index(int64_t p) const { return (int32_t)p; }
+    // keys of [0, V) into shared memory with 16-byte loads, 4 in flight per
+    // thread (a row is read from HBM once; one scalar load at a time would
+    // pay the memory latency for every 2 KB of the row)
+    __device__ __forceinline__ void stage(uint32_t *keys, int64_t V) const
+    {
+        int64_t head = 0;
+        if (((uintptr_t)src & 15u) != 0)
+            head = V < 4 - (int64_t)(((uintptr_t)src & 15u) >> 2) ? V
+                                                                    : 4 - (int64_t)(((uintptr_t)src & 15u) >> 2);
+        for (int64_t s = threadIdx.x; s < head; s += kThreads)
+            keys[s] = key(s);
+        const float4 *v4 = (const float4 *)(src + head);
+        const int64_t n4 = (V - head) >> 2;
+        int64_t i = threadIdx.x;
+        for (; i + 3 * kThreads < n4; i += 4 * kThreads) {
+            float4 f[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                f[j] = __ldg(v4 + i + j * kThreads);
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                uint32_t *d = keys + head + 4 * (i + j * kThreads);
+                d[0] = float_key(f[j].x);
+                d[1] = float_key(f[j].y);
+                d[2] = float_key(f[j].z);
+                d[3] = float_key(f[j].w);
+            }
+        }
+        for (; i < n4; i += kThreads) {
+            const float4 f = __ldg(v4 + i);
+            uint32_t *d = keys + head + 4 * i;
+            d[0] = float_key(f.x);
+            d[1] = float_key(f.y);
+            d[2] = float_key(f.z);
+            d[3] = float_key(f.w);
+        }
+        for (int64_t s = head + 4 * n4 + threadIdx.x; s < V; s += kThreads)
+            keys[s] = key(s);
+    }
 };
 
 struct RowCandidates {
@@ -60,95 +80,144 @@ struct RowCandidates {
     const int32_t *idx;
     __device__ __forceinline__ uint32_t key(int64_t p) const { return keys[p]; }
     __device__ __forceinline__ int32_t index(int64_t p) const { return idx[p]; }
+    __device__ __forceinline__ void stage(uint32_t *dst, int64_t V) const
+    {
+        for (int64_t s = threadIdx.x; s < V; s += kThreads)
+            dst[s] = keys[s];
+    }
 };
+
+// Bin of the digit histogram hist[0..nb) (descending) where the count from
+// the top reaches `need`; writes sh.bin and sh.need (what is still needed
+// inside that bin). Thread t owns bins nb-1-t*per .. nb-per-t*per.
+__device__ __forceinline__ void find_bin(Shared &sh, int nb, unsigned need)
+{
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int per = nb >= kThreads ? nb / kThreads : 1;
+    const int hi = nb - 1 - tid * per;                 // first (highest) owned bin
+    unsigned local = 0;
+    if (hi >= 0)
+        for (int j = 0; j < per; j++)
+            local += sh.hist[hi - j];
+    unsigned incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += y;
+    }
+    if (lane == 31)
+        sh.warp_tot[wid] = incl;
+    __syncthreads();
+    unsigned before = 0;
+    for (int w = 0; w < wid; w++)
+        before += sh.warp_tot[w];
+    incl += before;
+    const unsigned excl = incl - local;
+    if (hi >= 0 && excl < need && need <= incl) {
+        unsigned cum = excl;
+        for (int j = 0; j < per; j++) {
+            const unsigned hb = sh.hist[hi - j];
+            if (cum + hb >= need) {
+                sh.bin = (unsigned)(hi - j);
+                sh.need = need - cum;
+                break;
+            }
+            cum += hb;
+        }
+    }
+    __syncthreads();
+}
 
 // Top-k of positions [0, V) of `src` (V > k) by (key descending, position
 // ascending), written to out[0..k) in position order. Positions must be in
 // ascending order of the index they report, so ties go to lower indices.
+// The k-th largest key T is found with three radix digits (12, 12 and 8
+// bits, most significant first); each histogram adds the lanes of a warp that
+// fall in one bin with a single atomic. The compaction gives every warp one
+// contiguous segment of positions: the counts of keys above T and equal to T
+// per segment decide, after one barrier, where each warp writes and how many
+// of the keys equal to T it may still take.
 template <typename Src>
 __device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restrict__ out,
                              uint32_t *keys, bool res, Shared &sh)
 {
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (res) {
-        for (int64_t s = threadIdx.x; s < V; s += kThreads)
-            keys[s] = src.key(s);
+        src.stage(keys, V);
         __syncthreads();
     }
+    const int64_t Vr = (V + 31) & ~(int64_t)31;        // whole warps in every loop
 
     uint32_t prefix = 0, pmask = 0;
     unsigned need = (unsigned)k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int b = threadIdx.x; b < 256; b += kThreads)
+#pragma unroll 1
+    for (int p = 0; p < 3; p++) {
+        const int shift = p == 0 ? 20 : (p == 1 ? 8 : 0);
+        const int nb = p < 2 ? 4096 : 256;
+        for (int b = tid; b < nb; b += kThreads)
             sh.hist[b] = 0;
-        if (threadIdx.x == 0) {
-            sh.bin = 0;
-            sh.need = need;
+        __syncthreads();
+        for (int64_t s = tid; s < Vr; s += kThreads) {
+            uint32_t u = 0;
+            if (s < V)
+                u = res ? keys[s] : src.key(s);
+            const bool in = s < V && (u & pmask) == prefix;
+            const unsigned b = (u >> shift) & (unsigned)(nb - 1);
+            const unsigned same = __match_any_sync(0xffffffffu, in ? b : 0xffffffffu);
+            if (in && lane == __ffs(same) - 1)
+                atomicAdd(&sh.hist[b], (unsigned)__popc(same));
         }
         __syncthreads();
-        for (int64_t s = threadIdx.x; s < V; s += kThreads) {
-            const uint32_t u = res ? keys[s] : src.key(s);
-            if ((u & pmask) == prefix)
-                atomicAdd(&sh.hist[(u >> shift) & 255u], 1u);
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            // lane l owns bins 255-8l .. 248-8l (descending); find the bin
-            // where the count from the top reaches `need`.
-            const int lane = threadIdx.x;
-            unsigned local = 0;
-#pragma unroll
-            for (int j = 0; j < 8; j++)
-                local += sh.hist[255 - 8 * lane - j];
-            unsigned incl = local;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const unsigned v = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off)
-                    incl += v;
-            }
-            const unsigned excl = incl - local;
-            if (excl < need && need <= incl) {
-                unsigned cum = excl;
-                for (int j = 0; j < 8; j++) {
-                    const int b = 255 - 8 * lane - j;
-                    const unsigned hb = sh.hist[b];
-                    if (cum + hb >= need) {
-                        sh.bin = (unsigned)b;
-                        sh.need = need - cum;
-                        break;
-                    }
-                    cum += hb;
-                }
-            }
-        }
-        __syncthreads();
+        find_bin(sh, nb, need);
         prefix |= sh.bin << shift;
-        pmask |= 255u << shift;
+        pmask |= (unsigned)(nb - 1) << shift;
         need = sh.need;
-        __syncthreads();
+        __syncthreads();                                // sh.bin / sh.need reused
     }
-
-    // compaction in position order
     const uint32_t T = prefix;
-    unsigned base = 0, eq_seen = 0;
-    for (int64_t c0 = 0; c0 < V; c0 += kThreads) {
-        const int64_t s = c0 + threadIdx.x;
+
+    // compaction in position order, one contiguous segment per warp
+    const int64_t seg = ((V + kWarps - 1) / kWarps + 31) & ~(int64_t)31;
+    const int64_t w0 = (int64_t)wid * seg, w1 = w0 + seg < V ? w0 + seg : V;
+    unsigned ngt = 0, neq = 0;
+    for (int64_t s0 = w0; s0 < w1; s0 += 32) {
+        const int64_t s = s0 + lane;
         uint32_t u = 0;
-        if (s < V)
+        if (s < w1)
             u = res ? keys[s] : src.key(s);
-        const bool gt = s < V && u > T;
-        const bool eq = s < V && u == T;
-        unsigned eq_tot, take_tot;
-        const unsigned eq_rank = block_rank(eq, sh, &eq_tot);
-        const bool take = gt || (eq && eq_seen + eq_rank < need);
-        const unsigned pos = block_rank(take, sh, &take_tot);
-        if (take && base + pos < (unsigned)k)
-            out[base + pos] = src.index(s);
-        base += take_tot;
-        eq_seen += eq_tot;
+        ngt += __popc(__ballot_sync(0xffffffffu, s < w1 && u > T));
+        neq += __popc(__ballot_sync(0xffffffffu, s < w1 && u == T));
     }
-    for (int j = (int)base + threadIdx.x; j < k; j += kThreads)
-        out[j] = -1;
+    if (lane == 0) {
+        sh.warp_cnt[0][wid] = ngt;
+        sh.warp_cnt[1][wid] = neq;
+    }
+    __syncthreads();
+    unsigned gt_before = 0, eq_before = 0;
+    for (int w = 0; w < wid; w++) {
+        gt_before += sh.warp_cnt[0][w];
+        eq_before += sh.warp_cnt[1][w];
+    }
+    unsigned base = gt_before + (eq_before < need ? eq_before : need);
+    unsigned eq_seen = eq_before;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int64_t s0 = w0; s0 < w1; s0 += 32) {
+        const int64_t s = s0 + lane;
+        uint32_t u = 0;
+        if (s < w1)
+            u = res ? keys[s] : src.key(s);
+        const bool gt = s < w1 && u > T;
+        const bool eq = s < w1 && u == T;
+        const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+        const bool take = gt || (eq && eq_seen + __popc(eqb & lt) < need);
+        const unsigned tb = __ballot_sync(0xffffffffu, take);
+        const unsigned pos = base + __popc(tb & lt);
+        if (take && pos < (unsigned)k)
+            out[pos] = src.index(s);
+        base += __popc(tb);
+        eq_seen += __popc(eqb);
+    }
 }
 
 __global__ void __launch_bounds__(kThreads)

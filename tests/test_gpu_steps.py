@@ -188,6 +188,21 @@ def test_topk_long_rows_resident_and_streamed():
     _topk_case(3, 262144, 1024, 4, [4 * 262144 - 1] * 3, 23)
 
 
+def test_topk_block_rows_streamed_and_ties():
+    # one block per row past the shared-memory stage (rows re-read from L2)
+    _topk_case(4, 50000, 1000, 1, [49999, 41000, 900, 45000], 25)
+    # ties straddling the k-th value in every radix digit: five distinct scores
+    rows, E, k = 3, 20000, 777
+    rng = np.random.default_rng(26)
+    sc = torch.as_tensor(rng.integers(0, 5, size=(rows, E)).astype(np.float32) * 0.5 - 1.0)
+    q_pos = torch.tensor([E - 1, 15000, E - 1], dtype=torch.int64)
+    idx = torch.empty(rows, k, device=DEV, dtype=torch.int32)
+    abi.csa_topk(sc.to(DEV), q_pos.to(DEV), 1, k, idx, E)
+    abi.csa_get_error()
+    ref = oracle.topk(sc.double().numpy(), q_pos.numpy(), 1, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+
+
 def test_topk_long_rows_split_over_blocks():
     # rows past 65536 entries go through the four-launch chunked path with a
     # caller workspace: candidates of the threshold bin across chunk borders,
