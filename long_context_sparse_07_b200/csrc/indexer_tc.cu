@@ -10,10 +10,12 @@
 // its registers: I[t][s] = kscale[s] * sum_h w'[t][h] * ReLU(D[s][(t, h)]),
 // with w' = wI * qI_scale (scales are positive, so they commute with ReLU).
 //
-// Warp roles (192 threads): warp 0 issues TMA loads (query tile once, then a
-// ring of key-tile stages), warp 1 owns TMEM and issues the MMAs into two
-// accumulator buffers, warps 2-5 drain the accumulators (one lane quarter
-// each) and write score rows, overlapping the next tile's MMAs. Key tiles
+// Warp roles: warp 0 issues TMA loads (query tile once, then a ring of
+// key-tile stages), warp 1 owns TMEM and issues the MMAs into two
+// accumulator buffers, warps 2.. drain the accumulators and write score rows,
+// overlapping the next tile's MMAs: four warps per TMEM lane quarter when a
+// tile holds 4 or more tokens (each takes a quarter of the tokens), since the
+// head reduction costs more than the MMAs that feed it. Key tiles
 // past the causal bound of every token of the tile are never loaded; score
 // entries s >= V_t are not written. Every wait is bounded; on expiry the
 // block records CSA_ERR_TIMEOUT, drains its own copies and returns.
@@ -38,11 +40,13 @@ struct TcArgs {
     unsigned *err;
 };
 
-constexpr int kThreads = 192;
-
 template <bool FP8, int HI, int NT>
 struct Cfg {
     static constexpr int N = NT * HI;
+    // epilogue warps per TMEM lane quarter; each drains NT / SPLIT tokens
+    static constexpr int SPLIT = NT >= 4 ? 4 : NT;
+    static constexpr int TPW = NT / SPLIT;
+    static constexpr int THREADS = 32 * (2 + 4 * SPLIT);
     static constexpr int STAGES = FP8 ? 6 : 4;
     static constexpr int TMEM_COLS = (2 * N) < 32 ? 32 : 2 * N;
     static constexpr uint32_t IDESC = FP8 ? tc::idesc_e4m3(128, N) : tc::idesc_bf16(128, N);
@@ -53,7 +57,7 @@ struct Cfg {
 };
 
 template <bool FP8, int HI, int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<FP8, HI, NT>::THREADS, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmq,
                   const TcArgs a)
 {
@@ -106,7 +110,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         tc::mbar_init(bfull, 1);
         for (int i = 0; i < 2; i++) {
             tc::mbar_init(&accf[i], 1);
-            tc::mbar_init(&acce[i], 4);
+            tc::mbar_init(&acce[i], 4 * C::SPLIT);
         }
         tc::mbar_init(done, 1);
         tc::fence_mbar_init();
@@ -118,7 +122,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         tc::tmem_relinquish();
     }
     if (warp >= 2) {
-        for (int col = threadIdx.x - 64; col < N; col += 128) {
+        for (int col = threadIdx.x - 64; col < N; col += C::THREADS - 64) {
             const int tt = col / HI, hh = col % HI;
             const int64_t t = t0 + tt;
             float wv = 0.f;
@@ -211,8 +215,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             static_cast<void>(tc::mbar_wait(done, 0, &never, 200000000ull));
         }
     } else {
-        // ---------------- epilogue: warps 2..5, lane quarter = warp % 4
+        // ---------------- epilogue: warps 2.., lane quarter = warp % 4, tokens
+        // part * TPW .. part * TPW + TPW - 1 of the tile
         const int q4 = warp & 3;
+        const int part = (warp - 2) >> 2;
         const int row = q4 * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
         for (int i = 0; i < ntiles; i++) {
@@ -229,18 +235,20 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 ks = s < a.E ? a.kI_scale[(int64_t)b * a.E + s] : 0.f;
             const uint32_t base = lane_addr + (uint32_t)(buf * N);
 #pragma unroll
-            for (int tt = 0; tt < NT; tt++) {
+            for (int u = 0; u < C::TPW; u++) {
+                const int tt = part * C::TPW + u;
                 float sacc = 0.f;
                 if constexpr (HI >= 32) {
+                    uint32_t r[HI / 32][32];
 #pragma unroll
-                    for (int cc = 0; cc < HI / 32; cc++) {
-                        uint32_t r[32];
-                        tc::tmem_ld32(base + (uint32_t)(tt * HI + cc * 32), r);
-                        tc::tmem_ld_wait();
+                    for (int cc = 0; cc < HI / 32; cc++)
+                        tc::tmem_ld32(base + (uint32_t)(tt * HI + cc * 32), r[cc]);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int cc = 0; cc < HI / 32; cc++)
 #pragma unroll
                         for (int j = 0; j < 32; j++)
-                            sacc += wsm[tt * HI + cc * 32 + j] * fmaxf(__uint_as_float(r[j]), 0.f);
-                    }
+                            sacc += wsm[tt * HI + cc * 32 + j] * fmaxf(__uint_as_float(r[cc][j]), 0.f);
                 } else {
                     uint32_t r[16];
                     tc::tmem_ld16(base + (uint32_t)(tt * HI), r);
@@ -311,7 +319,7 @@ cudaError_t launch_one(const IndexerArgs &a, unsigned *err, cudaStream_t s)
     if (e != cudaSuccess)
         return e;
     dim3 grid((unsigned)(ttiles * t.nchunks), (unsigned)a.B);
-    indexer_tc_kernel<FP8, HI, NT><<<grid, kThreads, smem, s>>>(tmk, tmq, t);
+    indexer_tc_kernel<FP8, HI, NT><<<grid, C::THREADS, smem, s>>>(tmk, tmq, t);
     return cudaGetLastError();
 }
 
