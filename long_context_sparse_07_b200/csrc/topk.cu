@@ -22,11 +22,14 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kResident = 40960;   // keys staged in shared memory (160 KB)
 
+constexpr int kCand = 4096;          // keys of the first threshold bin kept aside
+
 struct Shared {
     unsigned hist[4096];                 // digit histogram (12 or 8 bits)
+    uint32_t cand[kCand];                // keys of the first threshold bin
     unsigned warp_tot[kWarps];
     unsigned warp_cnt[2][kWarps];
-    unsigned bin, need;
+    unsigned bin, need, ncand;
 };
 
 // Source of one row: order-preserving key and the index it reports.
@@ -36,15 +39,18 @@ struct RowScores {
     __device__ __forceinline__ int32_t index(int64_t p) const { return (int32_t)p; }
     // keys of [0, V) into shared memory with 16-byte loads, 4 in flight per
     // thread (a row is read from HBM once; one scalar load at a time would
-    // pay the memory latency for every 2 KB of the row)
-    __device__ __forceinline__ void stage(uint32_t *keys, int64_t V) const
+    // pay the memory latency for every 2 KB of the row), counted into the
+    // histogram of their top 12 bits on the way
+    __device__ __forceinline__ void stage(uint32_t *keys, int64_t V, unsigned *hist) const
     {
         int64_t head = 0;
         if (((uintptr_t)src & 15u) != 0)
             head = V < 4 - (int64_t)(((uintptr_t)src & 15u) >> 2) ? V
                                                                     : 4 - (int64_t)(((uintptr_t)src & 15u) >> 2);
-        for (int64_t s = threadIdx.x; s < head; s += kThreads)
+        for (int64_t s = threadIdx.x; s < head; s += kThreads) {
             keys[s] = key(s);
+            atomicAdd(&hist[keys[s] >> 20], 1u);
+        }
         const float4 *v4 = (const float4 *)(src + head);
         const int64_t n4 = (V - head) >> 2;
         int64_t i = threadIdx.x;
@@ -56,22 +62,36 @@ struct RowScores {
 #pragma unroll
             for (int j = 0; j < 4; j++) {
                 uint32_t *d = keys + head + 4 * (i + j * kThreads);
-                d[0] = float_key(f[j].x);
-                d[1] = float_key(f[j].y);
-                d[2] = float_key(f[j].z);
-                d[3] = float_key(f[j].w);
+                const uint32_t k0 = float_key(f[j].x), k1 = float_key(f[j].y);
+                const uint32_t k2 = float_key(f[j].z), k3 = float_key(f[j].w);
+                d[0] = k0;
+                d[1] = k1;
+                d[2] = k2;
+                d[3] = k3;
+                atomicAdd(&hist[k0 >> 20], 1u);
+                atomicAdd(&hist[k1 >> 20], 1u);
+                atomicAdd(&hist[k2 >> 20], 1u);
+                atomicAdd(&hist[k3 >> 20], 1u);
             }
         }
         for (; i < n4; i += kThreads) {
             const float4 f = __ldg(v4 + i);
             uint32_t *d = keys + head + 4 * i;
-            d[0] = float_key(f.x);
-            d[1] = float_key(f.y);
-            d[2] = float_key(f.z);
-            d[3] = float_key(f.w);
+            const uint32_t k0 = float_key(f.x), k1 = float_key(f.y);
+            const uint32_t k2 = float_key(f.z), k3 = float_key(f.w);
+            d[0] = k0;
+            d[1] = k1;
+            d[2] = k2;
+            d[3] = k3;
+            atomicAdd(&hist[k0 >> 20], 1u);
+            atomicAdd(&hist[k1 >> 20], 1u);
+            atomicAdd(&hist[k2 >> 20], 1u);
+            atomicAdd(&hist[k3 >> 20], 1u);
         }
-        for (int64_t s = head + 4 * n4 + threadIdx.x; s < V; s += kThreads)
+        for (int64_t s = head + 4 * n4 + threadIdx.x; s < V; s += kThreads) {
             keys[s] = key(s);
+            atomicAdd(&hist[keys[s] >> 20], 1u);
+        }
     }
 };
 
@@ -80,10 +100,13 @@ struct RowCandidates {
     const int32_t *idx;
     __device__ __forceinline__ uint32_t key(int64_t p) const { return keys[p]; }
     __device__ __forceinline__ int32_t index(int64_t p) const { return idx[p]; }
-    __device__ __forceinline__ void stage(uint32_t *dst, int64_t V) const
+    __device__ __forceinline__ void stage(uint32_t *dst, int64_t V, unsigned *hist) const
     {
-        for (int64_t s = threadIdx.x; s < V; s += kThreads)
-            dst[s] = keys[s];
+        for (int64_t s = threadIdx.x; s < V; s += kThreads) {
+            const uint32_t u = keys[s];
+            dst[s] = u;
+            atomicAdd(&hist[u >> 20], 1u);
+        }
     }
 };
 
@@ -133,8 +156,10 @@ __device__ __forceinline__ void find_bin(Shared &sh, int nb, unsigned need)
 // ascending), written to out[0..k) in position order. Positions must be in
 // ascending order of the index they report, so ties go to lower indices.
 // The k-th largest key T is found with three radix digits (12, 12 and 8
-// bits, most significant first); each histogram adds the lanes of a warp that
-// fall in one bin with a single atomic. The compaction gives every warp one
+// bits, most significant first). The first histogram is built while the row
+// is staged; the keys of its threshold bin are then set aside (when there are
+// at most kCand) so that the other two digits scan only them. The compaction
+// gives every warp one
 // contiguous segment of positions: the counts of keys above T and equal to T
 // per segment decide, after one barrier, where each warp writes and how many
 // of the keys equal to T it may still take.
@@ -143,30 +168,53 @@ __device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restri
                              uint32_t *keys, bool res, Shared &sh)
 {
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    // digit 1 (top 12 bits): histogram while the row is staged (or read)
+    for (int b = tid; b < 4096; b += kThreads)
+        sh.hist[b] = 0;
+    if (tid == 0)
+        sh.ncand = 0;
+    __syncthreads();
     if (res) {
-        src.stage(keys, V);
-        __syncthreads();
+        src.stage(keys, V, sh.hist);
+    } else {
+        for (int64_t s = tid; s < V; s += kThreads)
+            atomicAdd(&sh.hist[src.key(s) >> 20], 1u);
     }
-    const int64_t Vr = (V + 31) & ~(int64_t)31;        // whole warps in every loop
-
-    uint32_t prefix = 0, pmask = 0;
-    unsigned need = (unsigned)k;
+    __syncthreads();
+    find_bin(sh, 4096, (unsigned)k);
+    uint32_t prefix = sh.bin << 20, pmask = 0xfff00000u;
+    unsigned need = sh.need;
+    const unsigned c1 = sh.hist[sh.bin];
+    __syncthreads();                                    // sh.bin / sh.need reused
+    // digits 2 and 3 (12 and 8 bits) over the keys of that bin only: kept
+    // aside when there are few of them, else re-read from the row
+    const bool few = c1 <= (unsigned)kCand;
+    if (few) {
+        for (int64_t s = tid; s < V; s += kThreads) {
+            const uint32_t u = res ? keys[s] : src.key(s);
+            if ((u & pmask) == prefix)
+                sh.cand[atomicAdd(&sh.ncand, 1u)] = u;
+        }
+    }
 #pragma unroll 1
-    for (int p = 0; p < 3; p++) {
-        const int shift = p == 0 ? 20 : (p == 1 ? 8 : 0);
-        const int nb = p < 2 ? 4096 : 256;
+    for (int p = 1; p < 3; p++) {
+        const int shift = p == 1 ? 8 : 0;
+        const int nb = p == 1 ? 4096 : 256;
         for (int b = tid; b < nb; b += kThreads)
             sh.hist[b] = 0;
         __syncthreads();
-        for (int64_t s = tid; s < Vr; s += kThreads) {
-            uint32_t u = 0;
-            if (s < V)
-                u = res ? keys[s] : src.key(s);
-            const bool in = s < V && (u & pmask) == prefix;
-            const unsigned b = (u >> shift) & (unsigned)(nb - 1);
-            const unsigned same = __match_any_sync(0xffffffffu, in ? b : 0xffffffffu);
-            if (in && lane == __ffs(same) - 1)
-                atomicAdd(&sh.hist[b], (unsigned)__popc(same));
+        if (few) {
+            for (int j = tid; j < (int)c1; j += kThreads) {
+                const uint32_t u = sh.cand[j];
+                if ((u & pmask) == prefix)
+                    atomicAdd(&sh.hist[(u >> shift) & (unsigned)(nb - 1)], 1u);
+            }
+        } else {
+            for (int64_t s = tid; s < V; s += kThreads) {
+                const uint32_t u = res ? keys[s] : src.key(s);
+                if ((u & pmask) == prefix)
+                    atomicAdd(&sh.hist[(u >> shift) & (unsigned)(nb - 1)], 1u);
+            }
         }
         __syncthreads();
         find_bin(sh, nb, need);
