@@ -18,7 +18,7 @@ namespace csa {
 
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kResident = 40960;   // keys staged in shared memory (160 KB)
 
