@@ -433,12 +433,19 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--n", type=int, default=None,
+                    help="run the workload on a shorter sequence of n tokens (small profiling cases)")
     ap.add_argument("--graph", default="auto", choices=["auto", "on", "off"],
                     help="replay the timed step from a CUDA graph (auto: decode only)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     w = W.WORKLOADS[args.workload]
+    if args.n is not None:
+        # a shorter sequence of the same workload (profiling captures), named as such
+        if args.n % w.m or args.n <= 0:
+            sys.exit("--n must be a positive multiple of m = %d" % w.m)
+        w = W.scaled(w, n=args.n, name="%s@n%d" % (w.name, args.n))
     if args.impl == "reference":
         run_reference(args, w)
     else:
