@@ -111,9 +111,30 @@ class ClockSampler:
 # --------------------------------------------------------------------------- our arm
 
 
+def rank_workload(w, rank):
+    """The workload of one rank: every rank runs its own independent sequence
+    (same shapes, seed + 1000 * rank), so no data crosses ranks."""
+    return W.scaled(w, seed=w.seed + 1000 * rank) if rank else w
+
+
+def max_over_ranks(x, dist, device):
+    """x reduced with max over the ranks of `dist` (the value itself without it)."""
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(local_ms, units_per_rank, world, dist, device):
+    """Whole-job throughput: the units of all ranks over the slowest rank's
+    mean step time. Returns (rate per second, that time in ms)."""
+    ms = max_over_ranks(local_ms, dist, device)
+    return units_per_rank * world / (ms * 1e-3), ms
+
+
 def build_path(w, rank):
     from long_context_sparse_07_b200 import path
-    wr = W.scaled(w, seed=w.seed + 1000 * rank) if rank else w
+    wr = rank_workload(w, rank)
     if w.kind == "csa":
         return path.CsaPrefill(wr, W.csa_operands(wr))
     if w.kind == "hca":
@@ -304,21 +325,13 @@ def run_ours(args, w):
     barrier()
     abi.csa_get_error()
     mean_ms = sum(step_ms) / len(step_ms)
-    t = torch.tensor([mean_ms], device="cuda", dtype=torch.float64)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    units = units_per_step(w) * world
-    value = units / (ms * 1e-3)
+    value, ms = job_rate(mean_ms, units_per_step(w), world, dist, "cuda")
 
     # end to end through the public API with host buffers
     e2e_steps = max(3, min(args.steps, 20))
     p.step(stream)
     e_ms, h2d, d2h = time_e2e(p, e2e_steps, stream)
-    te = torch.tensor([sum(e_ms) / len(e_ms)], device="cuda", dtype=torch.float64)
-    if dist:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = units / (float(te.item()) * 1e-3)
+    e2e_value, _ = job_rate(sum(e_ms) / len(e_ms), units_per_step(w), world, dist, "cuda")
 
     # roofline of the dominant kernel
     pk = peaks()
