@@ -179,6 +179,28 @@ __device__ __forceinline__ const __nv_bfloat16 *key_row(const TcAttn &a, const Q
     return nullptr;
 }
 
+// The selection index read by key slot j (only slots j < nsel of a sparse
+// selection read one), and whether slot j holds a key, given that index: the
+// same decision as key_row, split so that the load can be issued early.
+__device__ __forceinline__ int32_t slot_index(const TcAttn &a, const QInfo &q, int64_t bt,
+                                              int64_t j)
+{
+    return (!a.dense && j < q.nsel) ? __ldg(a.idx + bt * a.k + j) : 0;
+}
+
+__device__ __forceinline__ bool slot_valid(const TcAttn &a, const QInfo &q, int64_t j, int32_t s)
+{
+    if (j < q.nsel) {
+        const int64_t e = a.dense ? j : (int64_t)s;
+        return e >= 0 && e < q.V;
+    }
+    if (j >= q.wbeg && j < q.nk) {
+        const int64_t wr = q.w0 + (j - q.wbeg) - q.wp0;
+        return wr >= 0 && wr < a.win_rows;
+    }
+    return false;
+}
+
 // 16 e4m3 codes times one scale -> 16 bf16 in two 16-byte chunks.
 __device__ __forceinline__ void decode16(const uint4 &cw, float sc, uint4 *lo, uint4 *hi)
 {
@@ -541,7 +563,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const uint32_t lane_tm = tmem + ((uint32_t)(q4 * 32) << 16);
         float *xg = sX + g * (8 * 128);                 // [8][128] partial logits handed over
         uint32_t t = 0, qctr = 0;
-        bool ok = true;
+        bool ok = true, stale = false;
         for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++qctr) {
             const int64_t bt = w / a.nchunks;
             const QInfo q = query_info(a, bt, (int)(w % a.nchunks));
@@ -549,16 +571,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int u = 0; u < 8; u++)
                 lpart[u] = 0.f;
+            // the selection index of this thread's key slot, loaded one tile
+            // ahead so that its latency overlaps the softmax of the tile before
+            int32_t s_next =
+                q.ntiles > 0 ? slot_index(a, q, bt, (int64_t)q.tile0 * KT + kidx) : 0;
             for (int i = 0; i < q.ntiles; ++i, ++t) {
-                int64_t er;
-                const bool valid =
-                    key_row<KV8>(a, q, bt, (int64_t)(q.tile0 + i) * KT + kidx, false, &er) != nullptr ||
-                    er >= 0;
-                const bool got = tc::mbar_wait(&sfull[t & 1], (t >> 1) & 1, abortv);
-                if (tc::named_bar_or(gbar, 128, !got)) {
-                    ok = false;
-                    break;
-                }
+                const int64_t jslot = (int64_t)(q.tile0 + i) * KT + kidx;
+                const int32_t s_cur = s_next;
+                if (i + 1 < q.ntiles)
+                    s_next = slot_index(a, q, bt, jslot + KT);
+                const bool valid = slot_valid(a, q, jslot, s_cur);
+                // a wait that gives up marks this thread stale; the group agrees
+                // on it at its next barrier (the exchange below, or the end of
+                // the item), so no barrier is spent on the waits themselves
+                stale |= !tc::mbar_wait(&sfull[t & 1], (t >> 1) & 1, abortv);
                 tc::fence_after();
                 float z[8];
                 {
@@ -569,7 +595,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                     for (int j = 0; j < 8; j++)
                         xg[j * 128 + r] = __uint_as_float(half ? rr[j] : rr[8 + j]);
-                    tc::named_bar_sync(gbar, 128);
+                    if (tc::named_bar_or(gbar, 128, stale)) {
+                        ok = false;
+                        break;
+                    }
 #pragma unroll
                     for (int j = 0; j < 8; j++) {
                         const float mine = __uint_as_float(half ? rr[8 + j] : rr[j]);
@@ -658,13 +687,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     lpart[j + 1] += pr.y;
                 }
                 // P^T is free once the O^T product of the previous tile is done
-                if (t > 0 && !o_waited) {
-                    const bool od = tc::mbar_wait(odone, (t - 1) & 1, abortv);
-                    if (tc::named_bar_or(gbar, 128, !od)) {
-                        ok = false;
-                        break;
-                    }
-                }
+                if (t > 0 && !o_waited)
+                    stale |= !tc::mbar_wait(odone, (t - 1) & 1, abortv);
                 {
                     // P^T rows hk..hk+7 (one per head, 64 keys, 128-byte swizzle)
                     uint8_t *pbase = sP + (kidx & 7) * 2;
@@ -692,7 +716,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (lane == 0)
                     red[q4 * H + hk + j] = v;
             }
-            tc::named_bar_sync(gbar, 128);
+            if (tc::named_bar_or(gbar, 128, stale)) {
+                ok = false;
+                break;
+            }
             // one thread per head: the output factor (alpha_s is free here)
             if (et < 16) {
                 const int hh = h0 + et;
@@ -819,7 +846,7 @@ combine_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_ml, 
 {
     __shared__ float wt[kMaxChunks];
     __shared__ float red[4];
-    __shared__ float s_M, s_den;
+    __shared__ float s_den;
     const int64_t bt = blockIdx.x;
     const int hh = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
