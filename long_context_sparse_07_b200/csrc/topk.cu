@@ -41,19 +41,19 @@ struct RowScores {
     // thread (a row is read from HBM once; one scalar load at a time would
     // pay the memory latency for every 2 KB of the row), counted into the
     // histogram of their top 12 bits on the way
-    __device__ __forceinline__ void stage(uint32_t *keys, int64_t V, unsigned *hist) const
+    __device__ __forceinline__ void stage(uint32_t *keys, int V, unsigned *hist) const
     {
-        int64_t head = 0;
+        int head = 0;
         if (((uintptr_t)src & 15u) != 0)
-            head = V < 4 - (int64_t)(((uintptr_t)src & 15u) >> 2) ? V
-                                                                    : 4 - (int64_t)(((uintptr_t)src & 15u) >> 2);
-        for (int64_t s = threadIdx.x; s < head; s += kThreads) {
+            head = V < 4 - (int)(((uintptr_t)src & 15u) >> 2) ? V
+                                                                : 4 - (int)(((uintptr_t)src & 15u) >> 2);
+        for (int s = threadIdx.x; s < head; s += kThreads) {
             keys[s] = key(s);
             atomicAdd(&hist[keys[s] >> 20], 1u);
         }
         const float4 *v4 = (const float4 *)(src + head);
-        const int64_t n4 = (V - head) >> 2;
-        int64_t i = threadIdx.x;
+        const int n4 = (V - head) >> 2;
+        int i = threadIdx.x;
         for (; i + 3 * kThreads < n4; i += 4 * kThreads) {
             float4 f[4];
 #pragma unroll
@@ -88,7 +88,7 @@ struct RowScores {
             atomicAdd(&hist[k2 >> 20], 1u);
             atomicAdd(&hist[k3 >> 20], 1u);
         }
-        for (int64_t s = head + 4 * n4 + threadIdx.x; s < V; s += kThreads) {
+        for (int s = head + 4 * n4 + threadIdx.x; s < V; s += kThreads) {
             keys[s] = key(s);
             atomicAdd(&hist[keys[s] >> 20], 1u);
         }
@@ -100,9 +100,9 @@ struct RowCandidates {
     const int32_t *idx;
     __device__ __forceinline__ uint32_t key(int64_t p) const { return keys[p]; }
     __device__ __forceinline__ int32_t index(int64_t p) const { return idx[p]; }
-    __device__ __forceinline__ void stage(uint32_t *dst, int64_t V, unsigned *hist) const
+    __device__ __forceinline__ void stage(uint32_t *dst, int V, unsigned *hist) const
     {
-        for (int64_t s = threadIdx.x; s < V; s += kThreads) {
+        for (int s = threadIdx.x; s < V; s += kThreads) {
             const uint32_t u = keys[s];
             dst[s] = u;
             atomicAdd(&hist[u >> 20], 1u);
@@ -163,21 +163,22 @@ __device__ __forceinline__ void find_bin(Shared &sh, int nb, unsigned need)
 // contiguous segment of positions: the counts of keys above T and equal to T
 // per segment decide, after one barrier, where each warp writes and how many
 // of the keys equal to T it may still take.
-template <typename Src>
-__device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restrict__ out,
-                             uint32_t *keys, bool res, Shared &sh)
+template <bool RES, typename Src>
+__device__ void block_select_t(const Src &src, int V, int k, int32_t *__restrict__ out,
+                               uint32_t *keys, Shared &sh)
 {
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    auto key_at = [&](int s) -> uint32_t { return RES ? keys[s] : src.key(s); };
     // digit 1 (top 12 bits): histogram while the row is staged (or read)
     for (int b = tid; b < 4096; b += kThreads)
         sh.hist[b] = 0;
     if (tid == 0)
         sh.ncand = 0;
     __syncthreads();
-    if (res) {
+    if (RES) {
         src.stage(keys, V, sh.hist);
     } else {
-        for (int64_t s = tid; s < V; s += kThreads)
+        for (int s = tid; s < V; s += kThreads)
             atomicAdd(&sh.hist[src.key(s) >> 20], 1u);
     }
     __syncthreads();
@@ -190,8 +191,8 @@ __device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restri
     // aside when there are few of them, else re-read from the row
     const bool few = c1 <= (unsigned)kCand;
     if (few) {
-        for (int64_t s = tid; s < V; s += kThreads) {
-            const uint32_t u = res ? keys[s] : src.key(s);
+        for (int s = tid; s < V; s += kThreads) {
+            const uint32_t u = key_at(s);
             if ((u & pmask) == prefix)
                 sh.cand[atomicAdd(&sh.ncand, 1u)] = u;
         }
@@ -210,8 +211,8 @@ __device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restri
                     atomicAdd(&sh.hist[(u >> shift) & (unsigned)(nb - 1)], 1u);
             }
         } else {
-            for (int64_t s = tid; s < V; s += kThreads) {
-                const uint32_t u = res ? keys[s] : src.key(s);
+            for (int s = tid; s < V; s += kThreads) {
+                const uint32_t u = key_at(s);
                 if ((u & pmask) == prefix)
                     atomicAdd(&sh.hist[(u >> shift) & (unsigned)(nb - 1)], 1u);
             }
@@ -226,16 +227,18 @@ __device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restri
     const uint32_t T = prefix;
 
     // compaction in position order, one contiguous segment per warp
-    const int64_t seg = ((V + kWarps - 1) / kWarps + 31) & ~(int64_t)31;
-    const int64_t w0 = (int64_t)wid * seg, w1 = w0 + seg < V ? w0 + seg : V;
-    unsigned ngt = 0, neq = 0;
-    for (int64_t s0 = w0; s0 < w1; s0 += 32) {
-        const int64_t s = s0 + lane;
-        uint32_t u = 0;
-        if (s < w1)
-            u = res ? keys[s] : src.key(s);
-        ngt += __popc(__ballot_sync(0xffffffffu, s < w1 && u > T));
-        neq += __popc(__ballot_sync(0xffffffffu, s < w1 && u == T));
+    const int seg = ((V + kWarps - 1) / kWarps + 31) & ~31;
+    const int w0 = wid * seg, w1 = w0 + seg < V ? w0 + seg : V;
+    unsigned ngt = 0, neq = 0;                          // per lane, summed below
+    for (int s = w0 + lane; s < w1; s += 32) {
+        const uint32_t u = key_at(s);
+        ngt += u > T;
+        neq += u == T;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ngt += __shfl_xor_sync(0xffffffffu, ngt, o);
+        neq += __shfl_xor_sync(0xffffffffu, neq, o);
     }
     if (lane == 0) {
         sh.warp_cnt[0][wid] = ngt;
@@ -250,11 +253,9 @@ __device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restri
     unsigned base = gt_before + (eq_before < need ? eq_before : need);
     unsigned eq_seen = eq_before;
     const unsigned lt = (1u << lane) - 1u;
-    for (int64_t s0 = w0; s0 < w1; s0 += 32) {
-        const int64_t s = s0 + lane;
-        uint32_t u = 0;
-        if (s < w1)
-            u = res ? keys[s] : src.key(s);
+    for (int s0 = w0; s0 < w1; s0 += 32) {
+        const int s = s0 + lane;
+        const uint32_t u = s < w1 ? key_at(s) : 0u;
         const bool gt = s < w1 && u > T;
         const bool eq = s < w1 && u == T;
         const unsigned eqb = __ballot_sync(0xffffffffu, eq);
@@ -266,6 +267,16 @@ __device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restri
         base += __popc(tb);
         eq_seen += __popc(eqb);
     }
+}
+
+template <typename Src>
+__device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restrict__ out,
+                             uint32_t *keys, bool res, Shared &sh)
+{
+    if (res)
+        block_select_t<true>(src, (int)V, k, out, keys, sh);
+    else
+        block_select_t<false>(src, (int)V, k, out, keys, sh);
 }
 
 __global__ void __launch_bounds__(kThreads)
