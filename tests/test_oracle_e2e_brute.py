@@ -11,7 +11,9 @@ the path (entries and index scores rounded to float32) and shares nothing with
 than V} cover the cases where a composition slip (visibility off by one, the
 window start, the sink in the max, an index-order mistake) would show. The
 HCA brute force does the same with non-overlapping blocks (Eq. 20-23) and
-every visible entry (Eq. 24-26).
+every visible entry (Eq. 24-26); the decode one reads the fp8 caches (codes
+decoded by torch, times their group scales, then the bf16 RoPE dims; Module F)
+and the window buffer by position.
 """
 import math
 
@@ -144,3 +146,89 @@ def test_hca_prefill_matches_brute_force(m):
     np.testing.assert_allclose(res["entries"], ent, rtol=0, atol=1e-12)
     np.testing.assert_allclose(res["out"], out, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(res["lse"], lse, rtol=1e-12, atol=1e-12)
+
+
+def e4m3(codes):
+    """e4m3 codes (uint8 tensor) to float64 values by torch's own decoder."""
+    import torch
+    return codes.contiguous().view(torch.float8_e4m3fn).to(torch.float64).numpy().tolist()
+
+
+def attend_bf(q, keys, zs, scale):
+    z = [scale * sum(qx * kx for qx, kx in zip(q, key)) for key in keys]
+    M = max(z + [zs])
+    e = [math.exp(v - M) for v in z]
+    den = sum(e) + math.exp(zs - M)
+    c = len(q)
+    return [sum(e[j] * keys[j][x] for j in range(len(keys))) / den for x in range(c)], \
+        M + math.log(den)
+
+
+def brute_decode(ops, w):
+    scale = 1.0 / math.sqrt(w.c)
+    G = w.scale_group
+    sink = ops["sink"].double().tolist()
+    res = {"idx": [], "out": [], "lse": [], "hca_out": [], "hca_lse": [], "scores": []}
+    for b in range(w.batch):
+        t = int(ops["q_pos"][b, 0])
+        qI_c, kI_c = e4m3(ops["qI"][b, 0]), e4m3(ops["kI"][b])
+        qs, ks = ops["qI_scale"][b, 0].double().tolist(), ops["kI_scale"][b].double().tolist()
+        wI = ops["wI"][b, 0].double().tolist()
+        E = len(kI_c)
+        V = visible(t, w.m, E)
+        sc = []
+        for s in range(V):
+            acc = 0.0
+            for hh in range(w.hI):
+                dot = sum(qI_c[hh][x] * qs[hh] * kI_c[s][x] * ks[s] for x in range(w.cI))
+                acc += wI[hh] * max(0.0, dot)
+            sc.append(f32(acc))
+        order = sorted(range(V), key=lambda s: (-sc[s], s))
+        sel = sorted(order[:min(w.k, V)])
+        res["scores"].append(sc)
+        res["idx"].append(sel + [-1] * (w.k - len(sel)))
+
+        def entry(pre, s):
+            body = e4m3(ops[pre + "_nope"][b, s])
+            scl = ops[pre + "_scale"][b, s].double().tolist()
+            return [body[x] * scl[x // G] for x in range(len(body))] + \
+                ops[pre + "_rope"][b, s].double().tolist()
+
+        p0 = int(ops["win_pos0"][b])
+        win = [ops["kwin"][b, p - p0].double().tolist() for p in range(max(0, t - w.n_win + 1), t + 1)]
+        q = ops["q"][b, 0].double().tolist()
+        keys = [entry("kv", s) for s in sel] + win
+        Eh = ops["hca_nope"].shape[1]
+        hkeys = [entry("hca", s) for s in range(visible(t, w.m_hca, Eh))] + win
+        o, l, ho, hl = [], [], [], []
+        for hh in range(w.h):
+            oo, ll = attend_bf(q[hh], keys, sink[hh], scale)
+            o.append(oo)
+            l.append(ll)
+            oo, ll = attend_bf(q[hh], hkeys, sink[hh], scale)
+            ho.append(oo)
+            hl.append(ll)
+        res["out"].append([o])
+        res["lse"].append([l])
+        res["hca_out"].append([ho])
+        res["hca_lse"].append([hl])
+    return res
+
+
+def test_decode_matches_brute_force():
+    # two sequences of 64 tokens: 16 CSA entries (k = 4 of them), 8 HCA
+    # entries (m' = 8), a 4-row window, fp8 split-layout caches
+    w = W.scaled(W.WORKLOADS["decode_b8_ctx1m"], n=64, batch=2, hI=2, cI=32, k=4, n_win=4,
+                 h=2, m_hca=8, seed=41)
+    ops = W.decode_operands(w)
+    bf = brute_decode(ops, w)
+    res = pipeline.decode(ops, w)
+    for b in range(w.batch):
+        V = len(bf["scores"][b])
+        # both round a float64 sum to float32; the sums may differ in their
+        # last bits (summation order), so allow one float32 step
+        np.testing.assert_allclose(res["scores"][b, :V], bf["scores"][b], rtol=2 ** -23, atol=0)
+    np.testing.assert_array_equal(res["idx"], np.array(bf["idx"]))
+    for key in ("out", "lse", "hca_out", "hca_lse"):
+        np.testing.assert_allclose(np.asarray(res[key]), np.array(bf[key]), rtol=1e-12,
+                                   atol=1e-12, err_msg=key)
