@@ -6,8 +6,11 @@ Selections: where the oracle's k-th and (k+1)-th scores are separated by more
 than the score tolerance the selected set is unique and must match exactly;
 elsewhere the GPU's set must be a valid top-k within that tolerance (every
 chosen entry scores at least the oracle's k-th score minus the tolerance). The
-share of such near-tie rows is bounded, and attention outputs are compared on
-every row whose selection matches the oracle's.
+share of such near-tie rows is bounded. First, the oracle's top-k over the
+GPU's own float32 scores must be the GPU's selection exactly. Attention
+outputs are compared with the oracle's on every row whose selection matches
+the oracle's, and on every sampled row with the oracle's attention over the
+GPU's own selection.
 """
 import math
 
@@ -67,11 +70,22 @@ def run_csa(w, rows, seed_rows_note=""):
         close.append((d <= SCORE_REL * S[r]).mean() if V[r] else 1.0)
     assert np.mean(close) > 0.99
     gidx = p.idx[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+    # selection, first level: the oracle's top-k over the GPU's own float32
+    # score rows is the GPU's selection exactly (same values, same tie rule)
+    np.testing.assert_array_equal(gidx, oracle.topk(sc, rows, w.m, w.k))
+    # second level: against the oracle's float64 scores, differences are near ties
     same = check_selection(gidx, ref["idx"], ref["scores"], V, w.k, 5e-3 * S)
     out = p.out[0][torch.as_tensor(rows, device="cuda")]
     assert_close_out(to_np(out)[same], ref["out"][same], w.dtype, "out")
     lse = p.lse[0][torch.as_tensor(rows, device="cuda")].cpu().double().numpy()
     np.testing.assert_allclose(lse[same], ref["lse"][same], rtol=1e-3, atol=1e-3)
+    # every sampled row against the oracle's attention over the GPU's own
+    # selection, so that a tolerated near tie cannot hide an output error
+    o2, l2 = oracle.attend(oracle.f64(ops["q"][rows])[None], ref["entries"][None], gidx, w.k,
+                           w.m, oracle.f64(ops["Ca"])[None], [0], w.n_win,
+                           np.asarray(rows).reshape(1, -1), ops["sink"], 1.0 / math.sqrt(w.c))
+    assert_close_out(to_np(out), o2[0], w.dtype, "out (GPU selection)")
+    np.testing.assert_allclose(lse, l2[0], rtol=1e-3, atol=1e-3)
 
 
 def test_csa_fp32_n256_all_rows():
@@ -119,8 +133,15 @@ def test_decode_b8_ctx1m():
     for b in range(B):
         assert (np.abs(sc[b] - ref["scores"][b]) <= SCORE_REL * S[b]).all()
     V = np.full(B, p.E)
-    same = check_selection(p.idx.cpu().numpy(), ref["idx"], ref["scores"], V, w.k,
+    gidx = p.idx.cpu().numpy()
+    np.testing.assert_array_equal(gidx, oracle.topk(sc, ops["q_pos"].numpy().reshape(B), w.m,
+                                                    w.k))
+    same = check_selection(gidx, ref["idx"], ref["scores"], V, w.k,
                            SCORE_REL * S, max_tie_share=0.5)
     assert_close_out(to_np(p.out)[same], ref["out"][same], "bf16", "csa out")
+    ent = pipeline.split_entries(ops["kv_nope"], ops["kv_scale"], ops["kv_rope"], w.scale_group)
+    o2, _ = oracle.attend(ops["q"], ent, gidx, w.k, w.m, ops["kwin"], ops["win_pos0"], w.n_win,
+                          ops["q_pos"].numpy(), ops["sink"], 1.0 / math.sqrt(w.c))
+    assert_close_out(to_np(p.out), o2, "bf16", "csa out (GPU selection)")
     assert_close_out(to_np(p.hout), ref["hca_out"], "bf16", "hca out")
     np.testing.assert_allclose(p.hlse.cpu().double().numpy(), ref["hca_lse"], rtol=1e-3)
