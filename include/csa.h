@@ -108,7 +108,8 @@ const char *csa_last_message(void);
  *                   scale_group dividing c - rope_dims (per-group scale =
  *                   max(amax / 448, 2^-126), codes rounded to nearest even
  *                   and saturated; rope channels stored as bf16).
- * Requirements: c % 8 == 0 (bf16) or c % 4 == 0 (f32), 1 <= m <= 1024,
+ * Requirements: c / 8 (bf16) or c / 4 (f32) a power of two of at most 256,
+ *   1 <= m <= 1024,
  *   all buffers 16-byte aligned.
  */
 csa_status csa_compress_kv(const void *Ca, const void *Cb, const void *Za, const void *Zb,
@@ -149,8 +150,10 @@ csa_status csa_indexer_scores(const void *qI, const float *qI_scale, const float
  *   q_pos     [rows] int64.
  *   idx       [rows, k] int32 output.
  *   workspace, ws_bytes   device scratch of at least
- *             csa_topk_workspace_size(rows, E, k) bytes (may be NULL when that
- *             size is 0).
+ *             csa_topk_workspace_size(rows, E, k) bytes, 256-byte aligned
+ *             (may be NULL when that size is 0; it is nonzero for rows of
+ *             65536 entries or more, which are split over many blocks).
+ *             The caller owns it; nothing in it must be initialised.
  * Requirements: 1 <= k <= 4096.
  */
 csa_status csa_topk(const float *scores, int64_t rows, int64_t E, int64_t ld,
