@@ -1,28 +1,37 @@
 #!/usr/bin/env python
 """Throughput of the CSA / HCA hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-per-workload] [--no-cpu-baseline]
 
 One step = one pass of the whole path over one synthetic sequence (CSA:
 compress KV, compress indexer keys, indexer scores, top-k, sparse attention;
 HCA: compress, dense attention; decode: indexer, top-k, sparse and HCA
-attention over a batch of long caches). With N GPUs (one process per GPU,
-launched by torchrun) every rank runs its own sequence: the units are
+attention over a batch of long caches). The default workload is the largest
+prefill that fits one GPU: a 131072-token CSA prefill with an e4m3 indexer
+(64 indexer heads, top-1024, 64 query heads). With N GPUs (one process per
+GPU, launched by torchrun) every rank runs its own sequence: the units are
 independent, so there is no data-path collective and scaling is weak.
 
-Printed by rank 0: one JSON line (see the keys below). ``value`` is tokens/s
-(prefill) or queries/s (decode) over all ranks, from CUDA-event time with
-inputs resident in HBM and L2 flushed between steps; ``e2e`` is the same
-metric with the step's inputs copied from pinned host memory and its output
-read back inside the timed region; ``roofline`` describes the dominant kernel;
-``cpu_baseline`` is the float64 CPU oracle on a bounded sample.
+Printed by rank 0: one JSON line. ``value`` is tokens/s (prefill) or
+queries/s (decode) over all ranks, from CUDA-event time with inputs resident
+in HBM and L2 flushed between steps; ``e2e`` is the same metric with the
+step's inputs copied from pinned host memory and its output read back inside
+the timed region; ``roofline`` describes the dominant kernel of the default
+workload; ``per_workload`` times every workload of the suite in the same run
+(step time, per-kernel times and roofline fractions, and for decode the HBM
+fraction of the CSA step); ``cpu_baseline`` is the float64 CPU oracle on a
+bounded sample, timed on inputs converted to float64 beforehand.
+
+``--impl reference`` times that same oracle sample as the reference arm.
 """
 from __future__ import annotations
 
 import argparse
 import datetime
-import json
 import hashlib
+import json
+import math
 import os
 import statistics
 import sys
@@ -39,19 +48,32 @@ from long_context_sparse_07_b200 import workloads as W  # noqa: E402
 from long_context_sparse_07_b200 import work  # noqa: E402
 
 METRIC = "CSA/HCA tokens/s (prefill), queries/s (decode) and % of roofline on 1 B200"
-DEFAULT_WORKLOAD = "csa_bf16_n4096"
+DEFAULT_WORKLOAD = "csa_fp8idx_n131072"
+SUITE = ("csa_fp32_n256", "csa_bf16_n4096", "hca_bf16_n65536", "csa_fp8idx_n131072",
+         "decode_b8_ctx1m")
 L2_FLUSH_BYTES = 512 << 20
+# query rows of the oracle's bounded sample, per workload (prefill: the
+# quadratic steps run on these rows, stratified over the sequence)
+ORACLE_ROWS = {"csa_fp32_n256": 256, "csa_bf16_n4096": 256, "hca_bf16_n65536": 64,
+               "csa_fp8idx_n131072": 32}
 
 
 def peaks():
+    """Roofline denominators: measured HBM copy bandwidth and dense bf16
+    throughput when present; e4m3 contractions take twice the bf16 figure
+    (the nominal dense fp8 : bf16 ratio of B200) until fp8 is measured."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as fh:
             d = json.load(fh)
-        return {"hbm": d["hbm_gbs"], "bf16": d["bf16_tflops"],
-                "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+        bf16 = d["bf16_tflops"]
+        return {"hbm": d["hbm_gbs"], "bf16": bf16,
+                "bf16_sustained": d.get("bf16_tflops_sustained", bf16),
+                "fp8": d.get("fp8_tflops", 2.0 * bf16),
+                "fp8_source": "measured" if "fp8_tflops" in d else "nominal-ratio (2 x measured bf16)",
                 "source": "measured"}
-    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "fp8": 3180.0,
+            "fp8_source": "nominal-ratio (2 x fallback bf16)", "source": "fallback"}
 
 
 # --------------------------------------------------------------------------- clocks
@@ -108,7 +130,7 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-# --------------------------------------------------------------------------- our arm
+# --------------------------------------------------------------------------- host logic
 
 
 def rank_workload(w, rank):
@@ -132,18 +154,38 @@ def job_rate(local_ms, units_per_rank, world, dist, device):
     return units_per_rank * world / (ms * 1e-3), ms
 
 
-def build_path(w, rank):
+def units_per_step(w):
+    return w.batch if w.kind == "decode" else w.n
+
+
+def unit_of(w):
+    return "queries/s" if w.kind == "decode" else "tokens/s"
+
+
+def config_of(w, world=1):
+    """The workload description both arms print (same keys, same values)."""
+    return {"workload": w.name, "n": w.n, "c": w.c, "m": w.m, "k": w.k, "h": w.h,
+            "hI": w.hI, "cI": w.cI, "n_win": w.n_win, "dtype": w.dtype,
+            "indexer_dtype": w.idx_dtype, "batch_per_gpu": w.batch,
+            "l2": "flushed between timed steps (512 MiB write)",
+            "parallelism": "dp%d (independent sequences)" % world}
+
+
+def build_path(w, rank, keep_ops=False):
+    """The device-resident step of rank `rank` (and, with keep_ops, the host
+    operands it was built from)."""
     from long_context_sparse_07_b200 import path
     wr = rank_workload(w, rank)
     if w.kind == "csa":
-        return path.CsaPrefill(wr, W.csa_operands(wr))
-    if w.kind == "hca":
-        return path.HcaPrefill(wr, W.hca_operands(wr))
-    return path.Decode(wr, W.decode_operands(wr))
-
-
-def units_per_step(w):
-    return w.batch if w.kind == "decode" else w.n
+        ops = W.csa_operands(wr)
+        p = path.CsaPrefill(wr, ops)
+    elif w.kind == "hca":
+        ops = W.hca_operands(wr)
+        p = path.HcaPrefill(wr, ops)
+    else:
+        ops = W.decode_operands(wr)
+        p = path.Decode(wr, ops)
+    return (p, ops) if keep_ops else p
 
 
 def algorithmic(w, p):
@@ -154,28 +196,54 @@ def algorithmic(w, p):
     return work.decode(w, p.E, p.E_hca)
 
 
-# DRAM bytes (read + write) per launch of the dominant kernel from one ncu capture
+def kernel_roofline(w, name, a, ms, pk):
+    """Roofline of one kernel from its algorithmic work `a` ({"flops",
+    "bytes"}) and its mean launch time: bound = the slower of the tensor-core
+    time (at the peak of its operand dtype) and the HBM time; frac = that
+    ideal time over the measured one."""
+    if w.dtype == "f32":
+        # CUDA-core float32 path of the parity-sized workload: no tensor peak
+        # applies; report against HBM only
+        tensor_peak, pdt = None, None
+    elif name == "indexer" and w.idx_dtype == "e4m3":
+        tensor_peak, pdt = pk["fp8"], "e4m3"
+    else:
+        tensor_peak, pdt = pk["bf16"], "bf16"
+    t_hbm = a["bytes"] / (pk["hbm"] * 1e9)
+    t_ten = a["flops"] / (tensor_peak * 1e12) if tensor_peak and a["flops"] else 0.0
+    sec = ms * 1e-3
+    if t_ten > t_hbm:
+        r = {"bound": "tensor", "achieved": a["flops"] / sec / 1e12, "peak": tensor_peak,
+             "unit": "TFLOP/s", "peak_dtype": pdt}
+    else:
+        r = {"bound": "hbm", "achieved": a["bytes"] / sec / 1e9, "peak": pk["hbm"],
+             "unit": "GB/s"}
+    r["frac"] = r["achieved"] / r["peak"]
+    r["ideal_ms"] = max(t_ten, t_hbm) * 1e3
+    return r
+
+
+# DRAM bytes (read + write) per launch of a kernel from one ncu capture
 # (summarised under profiles/), keyed by workload and kernel; each entry holds the
-# SHA-1 of the kernel source it was taken on and counts only while that source is
-# unchanged.
-MEASURED_TRAFFIC = {
-    ("csa_bf16_n4096", "attend"): ("attend_tc.cu", "7eeca1bf5e32ae25532dfa810103adaea4c2bcfc",
-                                   143.875840e6 + 95.943936e6),
-}
+# SHA-1 of the kernel source it was taken on and the number of launches it covers
+# scaled to a full launch, and counts only while that source is unchanged.
+MEASURED_TRAFFIC = {}
 
 
 def measured_traffic(workload, kernel):
     ent = MEASURED_TRAFFIC.get((workload, kernel))
     if ent is None:
         return None
-    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "long_context_sparse_07_b200",
-                       "csrc", ent[0])
+    src = os.path.join(ROOT, "long_context_sparse_07_b200", "csrc", ent[0])
     try:
         with open(src, "rb") as f:
             digest = hashlib.sha1(f.read()).hexdigest()
     except OSError:
         return None
     return ent[2] if digest == ent[1] else None
+
+
+# --------------------------------------------------------------------------- timing
 
 
 def time_steps(p, steps, flush, stream):
@@ -248,46 +316,196 @@ def time_e2e(p, steps, stream):
         b.record(stream)
         times.append((a, b))
     torch.cuda.synchronize()
+    del host_in, host_out
     return [a.elapsed_time(b) for a, b in times], h2d, d2h
 
 
-def cpu_baseline(w, p_rows=None):
-    """The oracle as it stands on a bounded sample, extrapolated linearly."""
-    import oracle
-    from oracle import pipeline
-    cores = os.cpu_count()
-    if w.kind == "decode":
-        wd = W.scaled(w, batch=1)
-        ops = W.decode_operands(wd)
-        t0 = time.perf_counter()
-        pipeline.decode(ops, wd)
-        dt = time.perf_counter() - t0
-        return {"value": 1.0 / dt, "unit": "queries/s", "cores": cores, "kind": "oracle",
-                "sample": "1 of %d decode queries (full cache), scaled per query" % w.batch}
-    ops = W.csa_operands(w) if w.kind == "csa" else W.hca_operands(w)
-    rows = p_rows or 128
-    sel = np.random.default_rng(0).choice(w.n, size=rows, replace=False)
-    # compression is linear in tokens: time it on the first n/8 tokens
-    ns = max(w.m, (w.n // 8) // w.m * w.m)
-    t0 = time.perf_counter()
-    if w.kind == "csa":
-        oracle.compress(ops["Ca"][:ns], ops["Cb"][:ns], ops["Za"][:ns], ops["Zb"][:ns],
-                        ops["Ba"], ops["Bb"], w.m, True)
-        oracle.compress(ops["CIa"][:ns], ops["CIb"][:ns], ops["ZIa"][:ns], ops["ZIb"][:ns],
-                        ops["BIa"], ops["BIb"], w.m, True)
+def measure(p, w, steps, warmup, graph, flush, stream, barrier, clk=None):
+    """Warm-up, then `steps` timed steps; returns (mean step ms, mean kernel
+    ms by name, whether a graph was replayed)."""
+    from long_context_sparse_07_b200 import abi
+    for _ in range(warmup):
+        p.step(stream)
+    torch.cuda.synchronize()
+    abi.csa_get_error()
+    barrier()
+    use_graph = graph == "on" or (graph == "auto" and w.kind == "decode")
+    if clk is not None:
+        with clk:
+            f = time_steps_graph if use_graph else time_steps
+            step_ms, kern_ms = f(p, steps, flush, stream)
     else:
-        oracle.compress(ops["C"][:ns], None, ops["Z"][:ns], None, ops["B"], None, w.m, False)
-    t_comp = (time.perf_counter() - t0) * (w.n / ns)
-    fn = pipeline.csa_prefill if w.kind == "csa" else pipeline.hca_prefill
-    t0 = time.perf_counter()
-    fn(ops, w, sel)
-    t_all = time.perf_counter() - t0
-    # the pipeline call also compresses the whole sequence once: subtract it
-    t_rows = max(t_all - t_comp, 1e-3)
-    total = t_comp + t_rows * (w.n / rows)
-    return {"value": w.n / total, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": "compression on %d of %d tokens and %d of %d query rows, extrapolated "
-                      "linearly" % (ns, w.n, rows, w.n)}
+        f = time_steps_graph if use_graph else time_steps
+        step_ms, kern_ms = f(p, steps, flush, stream)
+    barrier()
+    abi.csa_get_error()
+    kavg = {n: sum(v) / len(v) for n, v in kern_ms.items()}
+    return sum(step_ms) / len(step_ms), kavg, use_graph
+
+
+def workload_summary(w, p, step_ms, kavg, use_graph, pk, steps):
+    """Per-kernel rooflines and the whole step's fraction of its ideal time
+    (sum of the kernels' ideal times over the measured step time)."""
+    alg = algorithmic(w, p)
+    kernels = {n: kernel_roofline(w, n, alg[n], kavg[n], pk) for n in kavg}
+    ideal = sum(r["ideal_ms"] for r in kernels.values())
+    out = {"ms_per_step": step_ms, "value": units_per_step(w) / (step_ms * 1e-3),
+           "unit": unit_of(w), "steps": steps,
+           "launch": "CUDA graph replay" if use_graph else "eager",
+           "kernel_ms": {n: round(v, 5) for n, v in kavg.items()},
+           "kernels": {n: {k: (round(v, 4) if isinstance(v, float) else v)
+                           for k, v in r.items()} for n, r in kernels.items()},
+           "step_frac": ideal / step_ms if w.dtype != "f32" else None,
+           "dominant": max(kavg, key=kavg.get)}
+    if w.kind == "decode":
+        names = ("indexer", "topk", "attend")
+        ms = sum(kavg[n] for n in names)
+        by = sum(alg[n]["bytes"] for n in names)
+        out["csa_step"] = {"kernels": list(names), "ms": ms, "bytes": by,
+                           "achieved": by / (ms * 1e-3) / 1e9, "peak": pk["hbm"],
+                           "unit": "GB/s", "frac": by / (ms * 1e-3) / 1e9 / pk["hbm"]}
+    return out
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+
+def stratified_rows(n, count, seed):
+    """`count` query positions, one uniform pick in each of `count` equal
+    strata of [0, n) (all positions when count >= n)."""
+    if count >= n:
+        return np.arange(n, dtype=np.int64)
+    g = np.random.default_rng(seed)
+    lo = (np.arange(count) * n) // count
+    hi = ((np.arange(count) + 1) * n) // count
+    return (lo + np.floor(g.random(count) * (hi - lo))).astype(np.int64)
+
+
+class OracleSample:
+    """A bounded sample of one workload for the float64 CPU oracle, with
+    every input converted to float64 before any timing.
+
+    Prefill: the linear compression steps run over the whole sequence, the
+    quadratic steps (indexer, top-k, attention) over `rows` stratified query
+    positions; the whole workload's time is estimated as
+    t_compress + t_rows * n / rows. Decode: one query (sequence 0) over its
+    full cache, every step of the decode path; the batch takes B times that.
+    """
+
+    def __init__(self, w, seed=0, ops=None):
+        import oracle
+        from oracle import pipeline
+        self.oracle, self.pipeline, self.w = oracle, pipeline, w
+        f64 = oracle.f64
+        if w.kind == "decode":
+            ws = W.scaled(w, batch=1)
+            if ops is None:
+                ops = W.decode_operands(ws)
+            else:
+                # sequence 0 of a batch: every operand but the sink is batched
+                ops = {k: (v if k == "sink" else v[:1]) for k, v in ops.items()}
+            self.rows = 1
+            self.qI = oracle.dequantize(ops["qI"], ops["qI_scale"].reshape(1, 1, w.hI, 1), w.cI)
+            self.kI = oracle.dequantize(ops["kI"], ops["kI_scale"].reshape(1, -1, 1), w.cI)
+            self.ent = pipeline.split_entries(ops["kv_nope"], ops["kv_scale"], ops["kv_rope"],
+                                              w.scale_group)
+            self.hent = pipeline.split_entries(ops["hca_nope"], ops["hca_scale"],
+                                               ops["hca_rope"], w.scale_group)
+            self.wI, self.q, self.kwin = f64(ops["wI"]), f64(ops["q"]), f64(ops["kwin"])
+            self.sink = f64(ops["sink"])
+            self.pos = ops["q_pos"].numpy()
+            self.win_pos0 = ops["win_pos0"].numpy()
+            self.sample = ("1 of %d decode queries (sequence 0 over its full %d-token cache: "
+                           "indexer, top-k, CSA and HCA attention), caches decoded to float64 "
+                           "before timing; batch time = %d x that"
+                           % (w.batch, w.n, w.batch))
+            return
+        self.rows = stratified_rows(w.n, ORACLE_ROWS.get(w.name, 64), seed)
+        R = self.rows
+        if w.kind == "csa":
+            ops = W.csa_operands(w) if ops is None else ops
+            self.kv = [f64(ops[k]) for k in ("Ca", "Cb", "Za", "Zb", "Ba", "Bb")]
+            self.ki = [f64(ops[k]) for k in ("CIa", "CIb", "ZIa", "ZIb", "BIa", "BIb")]
+            self.qI, self.wI = pipeline._indexer_operands(ops, R, w)
+            self.win = self.kv[0]
+        else:
+            ops = W.hca_operands(w) if ops is None else ops
+            self.kv = [f64(ops[k]) for k in ("C", "Z", "B")]
+            self.win = self.kv[0]
+        self.q = f64(ops["q"][torch.as_tensor(R)])
+        self.sink = f64(ops["sink"])
+        self.sample = ("compression over all %d tokens; indexer, top-k and attention over %d "
+                       "stratified query rows of %d; whole-sequence time = t_compress + "
+                       "t_rows x n / rows; inputs converted to float64 before timing"
+                       % (w.n, len(R), w.n) if len(R) < w.n else
+                       "the whole workload (all %d query rows)" % w.n)
+
+    def run(self):
+        """Times one pass of the sample; returns the estimated seconds of the
+        whole workload (one step) and the seconds actually spent."""
+        o, pl, w = self.oracle, self.pipeline, self.w
+        scale = 1.0 / math.sqrt(w.c)
+        t0 = time.perf_counter()
+        if w.kind == "decode":
+            sc = o.indexer(self.qI, self.wI, self.kI, self.pos, w.m)
+            sel = o.topk(sc.reshape(1, -1).astype(np.float32), self.pos.reshape(1), w.m, w.k)
+            o.attend(self.q, self.ent, sel, w.k, w.m, self.kwin, self.win_pos0, w.n_win,
+                     self.pos, self.sink, scale)
+            o.attend(self.q, self.hent, None, 0, w.m_hca, self.kwin, self.win_pos0, w.n_win,
+                     self.pos, self.sink, scale)
+            dt = time.perf_counter() - t0
+            return dt * w.batch, dt
+        R = self.rows
+        pos = R.reshape(1, -1)
+        if w.kind == "csa":
+            ent = pl.store(o.compress(*self.kv, w.m, True), w.dtype)
+            k64 = o.compress(*self.ki, w.m, True)
+            if w.idx_dtype == "e4m3":
+                codes, scales = o.quantize_e4m3(k64, w.cI)
+                kI = o.dequantize(codes, scales, w.cI)
+            else:
+                kI = pl.store(k64, w.idx_dtype)
+            t1 = time.perf_counter()
+            sc = o.indexer(self.qI[None], self.wI[None], kI[None], pos, w.m)[0]
+            sel = o.topk(sc.astype(np.float32), R, w.m, w.k)
+            o.attend(self.q[None], ent[None], sel, w.k, w.m, self.win[None], [0], w.n_win, pos,
+                     self.sink, scale)
+        else:
+            C, Z, B = self.kv
+            ent = pl.store(o.compress(C, None, Z, None, B, None, w.m, False), w.dtype)
+            t1 = time.perf_counter()
+            o.attend(self.q[None], ent[None], None, 0, w.m, self.win[None], [0], w.n_win, pos,
+                     self.sink, scale)
+        t2 = time.perf_counter()
+        return (t1 - t0) + (t2 - t1) * w.n / len(R), t2 - t0
+
+
+def oracle_cores():
+    """Threads the oracle's OpenMP loops use."""
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v and v.isdigit() else os.cpu_count()
+
+
+def host_operands(w):
+    """The workload's operands on the host (decode: sequence 0 only, the
+    part the oracle sample reads)."""
+    if w.kind == "csa":
+        return W.csa_operands(w)
+    if w.kind == "hca":
+        return W.hca_operands(w)
+    return W.decode_operands(W.scaled(w, batch=1))
+
+
+def cpu_baseline(w, ops=None):
+    """The oracle as it stands on a bounded sample (OracleSample)."""
+    s = OracleSample(w, ops=ops)
+    s.run()                                   # first pass: page-in, thread start-up
+    est, spent = s.run()
+    return {"value": units_per_step(w) / est, "unit": unit_of(w), "cores": oracle_cores(),
+            "kind": "oracle", "sample": s.sample, "sample_s": round(spent, 3)}
+
+
+# --------------------------------------------------------------------------- our arm
 
 
 def run_ours(args, w):
@@ -302,77 +520,80 @@ def run_ours(args, w):
                                 device_id=torch.device("cuda", local))
     from long_context_sparse_07_b200 import abi
     abi.load()
-    p = build_path(w, rank)
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    for _ in range(args.warmup):
-        p.step(stream)
-    torch.cuda.synchronize()
-    abi.csa_get_error()
+    pk = peaks()
 
     def barrier():
         if dist:
             dist.barrier()
         torch.cuda.synchronize()
 
-    barrier()
-    graph = args.graph == "on" or (args.graph == "auto" and w.kind == "decode")
-    with ClockSampler(local) as clk:
-        if graph:
-            step_ms, kern_ms = time_steps_graph(p, args.steps, flush, stream)
-        else:
-            step_ms, kern_ms = time_steps(p, args.steps, flush, stream)
-    barrier()
-    abi.csa_get_error()
-    mean_ms = sum(step_ms) / len(step_ms)
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    p, host_ops = build_path(w, rank, keep_ops=True)
+    if not want_cpu:
+        host_ops = None
+    clk = ClockSampler(local)
+    mean_ms, kavg, use_graph = measure(p, w, args.steps, args.warmup, args.graph, flush, stream,
+                                       barrier, clk)
     value, ms = job_rate(mean_ms, units_per_step(w), world, dist, "cuda")
+    summ = workload_summary(w, p, mean_ms, kavg, use_graph, pk, args.steps)
 
     # end to end through the public API with host buffers
-    e2e_steps = max(3, min(args.steps, 20))
-    p.step(stream)
+    e2e_steps = max(3, min(args.steps, 20 if units_per_step(w) * w.h * w.c < (1 << 30) else 3))
     e_ms, h2d, d2h = time_e2e(p, e2e_steps, stream)
     e2e_value, _ = job_rate(sum(e_ms) / len(e_ms), units_per_step(w), world, dist, "cuda")
 
-    # roofline of the dominant kernel
-    pk = peaks()
-    alg = algorithmic(w, p)
-    kavg = {n: sum(v) / len(v) for n, v in kern_ms.items()}
-    dom = max(kavg, key=kavg.get)
-    a = alg[dom]
-    if a["flops"] > 0 and a["flops"] / pk["bf16"] > a["bytes"] / (pk["hbm"] * 1e9 / 1e12):
-        achieved = a["flops"] / (kavg[dom] * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s"}
-    else:
-        achieved = a["bytes"] / (kavg[dom] * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+    dom = summ["dominant"]
+    roof = dict(summ["kernels"][dom])
+    roof.pop("ideal_ms", None)
     roof["traffic"] = measured_traffic(w.name, dom)
     roof["kernel"] = dom
-    roof["peak_source"] = pk["source"]
-    roof["kernel_ms"] = {n: round(v, 5) for n, v in kavg.items()}
+    roof["peak_source"] = pk["source"] if roof.get("peak_dtype") != "e4m3" else pk["fp8_source"]
+    roof["kernel_ms"] = summ["kernel_ms"]
+    launches = p.launches_per_step * args.steps
+    del p
+    torch.cuda.empty_cache()
+
+    # every other workload of the suite, each on its own (rank-local) inputs
+    per = {}
+    if not args.no_per_workload and args.n is None:
+        for name in SUITE:
+            if name == w.name:
+                per[name] = summ
+                continue
+            wn = W.WORKLOADS[name]
+            pn = build_path(wn, rank)
+            steps_n = max(3, min(args.steps, 10))
+            m_n, k_n, g_n = measure(pn, wn, steps_n, args.warmup, args.graph, flush, stream,
+                                    barrier)
+            per[name] = workload_summary(wn, pn, m_n, k_n, g_n, pk, steps_n)
+            launches += pn.launches_per_step * steps_n
+            del pn
+            torch.cuda.empty_cache()
 
     if rank == 0:
-        unit = "queries/s" if w.kind == "decode" else "tokens/s"
         line = {
-            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+            "metric": METRIC, "value": value, "unit": unit_of(w), "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32",
             "data": "synthetic (seeded generators; random-init projection outputs)",
-            "config": {"workload": w.name, "n": w.n, "c": w.c, "m": w.m, "k": w.k,
-                       "h": w.h, "hI": w.hI, "cI": w.cI, "n_win": w.n_win,
-                       "indexer_dtype": w.idx_dtype, "batch_per_gpu": w.batch,
-                       "l2": "flushed between timed steps (512 MiB write)",
-                       "launch": "CUDA graph replay" if graph else "eager",
-                       "parallelism": "dp%d (independent sequences)" % world},
-            "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": p.launches_per_step * args.steps,
+            "config": config_of(w, world),
+            "launch": "CUDA graph replay" if use_graph else "eager",
+            "e2e": {"value": e2e_value, "unit": unit_of(w), "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches,
             "roofline": roof,
+            "step_frac": summ["step_frac"],
             "clocks": clk.summary(),
+            "peaks": {k: pk[k] for k in ("hbm", "bf16", "bf16_sustained", "fp8", "source",
+                                         "fp8_source")},
         }
+        if per:
+            line["per_workload"] = per
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(w)
+            line["cpu_baseline"] = cpu_baseline(w, host_ops)
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -383,56 +604,34 @@ def run_ours(args, w):
 
 
 def run_reference(args, w):
-    """The CPU oracle timed as the reference arm (bounded sample per step)."""
+    """The CPU oracle timed as the reference arm: each step is one pass of the
+    same bounded sample as ``cpu_baseline`` (new stratified rows per step)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    import oracle
-    from oracle import pipeline
-    cores = os.cpu_count()
-    total_steps = args.steps + args.warmup
-    budget = 90.0 / max(total_steps, 1)          # seconds of CPU work per step
-    if w.kind == "decode":
-        raise SystemExit("reference arm: decode workload not wired")
-    ops = W.csa_operands(w) if w.kind == "csa" else W.hca_operands(w)
-    fn = pipeline.csa_prefill if w.kind == "csa" else pipeline.hca_prefill
-    # calibrate: one row costs about this much (compression included once)
-    g = np.random.default_rng(0)
-    t0 = time.perf_counter()
-    fn(ops, w, g.choice(w.n, size=8, replace=False))
-    t_cal = time.perf_counter() - t0
-    ns = max(w.m, min(w.n, int(w.n * min(1.0, budget / max(t_cal, 1e-3) / 4))) // w.m * w.m)
-    rows = 4
-    times = []
-    for i in range(total_steps):
-        sel = g.choice(w.n, size=rows, replace=False)
-        t0 = time.perf_counter()
-        if w.kind == "csa":
-            oracle.compress(ops["Ca"][:ns], ops["Cb"][:ns], ops["Za"][:ns], ops["Zb"][:ns],
-                            ops["Ba"], ops["Bb"], w.m, True)
-        else:
-            oracle.compress(ops["C"][:ns], None, ops["Z"][:ns], None, ops["B"], None, w.m,
-                            False)
-        t1 = time.perf_counter()
-        fn(ops, w, sel)
-        t2 = time.perf_counter()
+    ops = host_operands(w)
+    samples = [OracleSample(w, seed=s, ops=ops) for s in range(2)]
+    del ops
+    est, spent = [], []
+    for i in range(args.steps + args.warmup):
+        e, s = samples[i % 2].run()
         if i >= args.warmup:
-            t_comp = (t1 - t0) * w.n / ns
-            t_rows = max((t2 - t1) - t_comp, 1e-4) * w.n / rows
-            times.append(t_comp + t_rows)
-    ms = 1e3 * sum(times) / len(times)
-    value = w.n / (ms * 1e-3)
-    unit = "tokens/s"
+            est.append(e)
+            spent.append(s)
+    t_est = sum(est) / len(est)
+    value = units_per_step(w) / t_est
+    unit = unit_of(w)
+    cores = oracle_cores()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit,
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(spent) / len(spent),
+            "ms_per_workload_estimated": 1e3 * t_est,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic (seeded generators)",
-            "config": {"workload": w.name, "n": w.n, "c": w.c, "m": w.m, "k": w.k,
-                       "h": w.h},
+            "config": config_of(w, world),
             "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
-                             "sample": "per step: compression on %d of %d tokens and %d query "
-                                       "rows, extrapolated linearly" % (ns, w.n, rows)},
+                             "sample": samples[0].sample},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -441,11 +640,13 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="time only the selected workload")
     ap.add_argument("--n", type=int, default=None,
                     help="run the workload on a shorter sequence of n tokens (small profiling cases)")
     ap.add_argument("--graph", default="auto", choices=["auto", "on", "off"],

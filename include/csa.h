@@ -220,7 +220,7 @@ size_t csa_mqa_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys
  * allocation may cause). The method on the reference pages has no
  * counterpart of this call: it only changes where the scratch lives.
  *   Scratch (the split-key partial results) comes from one file-scope device
- *   array of csa_noalloc_scratch_bytes() bytes (16 MiB) that every GPU loading
+ *   array of csa_noalloc_scratch_bytes() bytes (32 MiB) that every GPU loading
  *   the library holds until the process exits. The call allocates nothing.
  *   Every other argument, the results and the error behaviour are those of
  *   csa_sparse_mqa. A shape whose scratch (csa_mqa_workspace_size) exceeds the
@@ -228,6 +228,11 @@ size_t csa_mqa_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys
  *   csa_last_message().
  *   The first call on a device looks up the array's device address (with
  *   that device current); make it before capturing the stream into a graph.
+ *   The address is kept for the life of the process and does not survive a
+ *   device reset (cudaDeviceReset): do not call this entry point on a device
+ *   after resetting it in the same process.
+ *   The 32 MiB cover a decode step of 8 queries, 64 heads of width 512, 1024
+ *   selected entries and a 128-row window.
  *   All calls share the one array and each call overwrites the part it uses
  *   before reading it, so nothing needs clearing; but calls that may overlap
  *   on the GPU (different streams, or different host threads on one device)
@@ -239,6 +244,18 @@ csa_status csa_sparse_mqa_noalloc(const void *q, csa_dtype q_dt, csa_entries kv,
                                   const float *sink, int B, int64_t n_q, int h, float scale,
                                   void *out, float *lse, void *stream);
 size_t csa_noalloc_scratch_bytes(void);
+
+/*
+ * csa_debug_wait_probe -- checks the device-side failure path. Launches one
+ * thread that waits, through the same bounded mbarrier wait every pipeline
+ * kernel uses, on a barrier that nothing completes; after limit_ns
+ * nanoseconds (1e3 .. 1e9) the wait gives up and the device error word
+ * records CSA_ERR_TIMEOUT, which the next csa_get_error returns (and clears).
+ * Nothing is left in flight and the device stays usable. The method has no
+ * counterpart of this call: it exists so that tests can make a device wait
+ * expire without faulting or hanging the GPU.
+ */
+csa_status csa_debug_wait_probe(uint64_t limit_ns, void *stream);
 
 /*
  * csa_get_error -- synchronises the current device, reads and clears its

@@ -28,7 +28,7 @@ STATUS = {0: "CSA_OK", -1: "CSA_ERR_INVALID_ARG", -2: "CSA_ERR_UNSUPPORTED",
 EXPORTS = ("csa_abi_version", "csa_status_string", "csa_last_message", "csa_compress_kv",
            "csa_indexer_scores", "csa_topk", "csa_topk_workspace_size", "csa_sparse_mqa",
            "hca_dense_mqa", "csa_mqa_workspace_size", "csa_sparse_mqa_noalloc",
-           "csa_noalloc_scratch_bytes", "csa_get_error")
+           "csa_noalloc_scratch_bytes", "csa_debug_wait_probe", "csa_get_error")
 
 
 class CsaError(RuntimeError):
@@ -85,6 +85,8 @@ def load(path: str = LIB_PATH):
                                          _P, _I, _I64, _I, _F, _P, _P, _P]
     L.csa_noalloc_scratch_bytes.restype = _S
     L.csa_noalloc_scratch_bytes.argtypes = []
+    L.csa_debug_wait_probe.restype = _I
+    L.csa_debug_wait_probe.argtypes = [ctypes.c_uint64, _P]
     L.csa_get_error.restype = _I
     L.csa_get_error.argtypes = [ctypes.c_char_p, _S]
     _lib = L
@@ -211,6 +213,12 @@ def hca_dense_mqa(q, kv: Entries, E: int, m: int, kwin, win_pos0, n_win: int, q_
                                 win_rows, _ptr(win_pos0), n_win, _ptr(q_pos), _ptr(sink), B,
                                 n_q, h, scale, _ptr(out), _ptr(lse), _ptr(workspace), ws,
                                 _stream(stream)))
+
+
+def csa_debug_wait_probe(limit_ns: int, stream=None):
+    """Launch one bounded device wait that nothing completes; the next
+    csa_get_error() reports CSA_ERR_TIMEOUT."""
+    _check(load().csa_debug_wait_probe(int(limit_ns), _stream(stream)))
 
 
 def csa_get_error() -> int:

@@ -213,13 +213,15 @@ size_t csa_mqa_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys
     return csa::attend_workspace_size(B, n_q, h, c, max_keys);
 }
 
-static csa_status attend_common(const char *w, const void *q, csa_dtype q_dt, csa_entries kv,
-                                int64_t E, int dense, const int32_t *idx, int k, int m,
-                                const void *kwin,
-                                int64_t win_rows, const int64_t *win_pos0, int n_win,
-                                const int64_t *q_pos, const float *sink, int B, int64_t n_q,
-                                int h, float scale, void *out, float *lse, void *workspace,
-                                size_t ws_bytes, void *stream)
+}  // extern "C"
+
+namespace csa {
+
+// Host-side checks of an attention call, workspace excluded (see csa.h).
+csa_status check_attend(const char *w, const void *q, csa_dtype q_dt, const csa_entries &kv,
+                        int64_t E, const int32_t *idx, int k, int m, const void *kwin,
+                        int64_t win_rows, int n_win, const int64_t *q_pos, const float *sink,
+                        int B, int64_t n_q, int h, void *out)
 {
     REQUIRE(q && out && q_pos && sink, CSA_ERR_INVALID_ARG,
             "%s: q, out, q_pos and sink are required", w);
@@ -244,6 +246,26 @@ static csa_status attend_common(const char *w, const void *q, csa_dtype q_dt, cs
             "%s: a window needs a 16-byte aligned kwin with win_rows >= 1", w);
     REQUIRE(aligned16(q) && aligned16(out), CSA_ERR_INVALID_ARG,
             "%s: q and out must be 16-byte aligned", w);
+    return CSA_OK;
+}
+
+}  // namespace csa
+
+extern "C" {
+
+static csa_status attend_common(const char *w, const void *q, csa_dtype q_dt, csa_entries kv,
+                                int64_t E, int dense, const int32_t *idx, int k, int m,
+                                const void *kwin,
+                                int64_t win_rows, const int64_t *win_pos0, int n_win,
+                                const int64_t *q_pos, const float *sink, int B, int64_t n_q,
+                                int h, float scale, void *out, float *lse, void *workspace,
+                                size_t ws_bytes, void *stream)
+{
+    csa_status st = csa::check_attend(w, q, q_dt, kv, E, idx, k, m, kwin, win_rows, n_win,
+                                      q_pos, sink, B, n_q, h, out);
+    if (st != CSA_OK)
+        return st;
+    const int c = kv.c;
     const size_t need = csa::attend_workspace_size(B, n_q, h, c, (dense ? E : k) + n_win);
     REQUIRE(ws_bytes >= need && (need == 0 || workspace), CSA_ERR_INVALID_ARG,
             "%s: workspace of %zu bytes required", w, need);
@@ -277,6 +299,16 @@ csa_status hca_dense_mqa(const void *q, csa_dtype q_dt, csa_entries kv, int64_t 
     return attend_common("hca_dense_mqa", q, q_dt, kv, E, 1, nullptr, 0, m, kwin, win_rows,
                          win_pos0, n_win, q_pos, sink, B, n_q, h, scale, out, lse, workspace,
                          ws_bytes, stream);
+}
+
+csa_status csa_debug_wait_probe(uint64_t limit_ns, void *stream)
+{
+    const char *w = "csa_debug_wait_probe";
+    REQUIRE(limit_ns >= 1000u && limit_ns <= 1000000000u, CSA_ERR_INVALID_ARG,
+            "%s: limit_ns = %llu out of [1e3, 1e9]", w, (unsigned long long)limit_ns);
+    unsigned *err = err_word();
+    REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
+    return launched(csa::launch_wait_probe(limit_ns, err, (cudaStream_t)stream), w);
 }
 
 csa_status csa_get_error(char *buf, size_t len)

@@ -68,6 +68,16 @@ struct AttendArgs {
 };
 cudaError_t launch_attend(const AttendArgs &a, unsigned *err, cudaStream_t s);
 
+// Host-side checks of an attention call (everything but the workspace);
+// CSA_OK or the status the call returns, with csa_last_message() set.
+csa_status check_attend(const char *what, const void *q, csa_dtype q_dt, const csa_entries &kv,
+                        int64_t E, const int32_t *idx, int k, int m, const void *kwin,
+                        int64_t win_rows, int n_win, const int64_t *q_pos, const float *sink,
+                        int B, int64_t n_q, int h, void *out);
+
+// One bounded wait that nothing completes (csa_debug_wait_probe).
+cudaError_t launch_wait_probe(uint64_t limit_ns, unsigned *err, cudaStream_t s);
+
 // Sets the text that csa_last_message() returns on this thread.
 void set_last_message(const char *msg);
 size_t attend_workspace_size(int B, int64_t n_q, int h, int c, int64_t max_keys);

@@ -16,7 +16,10 @@
 
 namespace {
 
-constexpr size_t kScratchBytes = 16u << 20;     // 16 MiB per GPU
+// 32 MiB per GPU: enough for an 8-query decode step with 64 heads of width
+// 512 over 1024 selected entries and a 128-row window (18 key chunks per
+// query, 18.9 MB of partial results).
+constexpr size_t kScratchBytes = 32u << 20;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -26,7 +29,9 @@ std::mutex g_scratch_mutex;
 
 // Device address of this GPU's scratch array. In host code the array's name
 // only stands in for the symbol, so the address is looked up once per device,
-// with that device current.
+// with that device current, and kept for the life of the process: it does
+// not survive a reset of the device (cudaDeviceReset), after which this entry
+// point must not be called again in the same process.
 cudaError_t scratch_address(void **out)
 {
     int dev = 0;
@@ -59,9 +64,11 @@ csa_status csa_sparse_mqa_noalloc(const void *q, csa_dtype q_dt, csa_entries kv,
                                   const float *sink, int B, int64_t n_q, int h, float scale,
                                   void *out, float *lse, void *stream)
 {
-    if (B < 0 || n_q < 0 || k < 0 || n_win < 0)
-        return csa_sparse_mqa(q, q_dt, kv, E, m, idx, k, kwin, win_rows, win_pos0, n_win, q_pos,
-                              sink, B, n_q, h, scale, out, lse, nullptr, 0, stream);
+    // the arguments are checked before the scratch is sized from them
+    const csa_status st = csa::check_attend("csa_sparse_mqa_noalloc", q, q_dt, kv, E, idx, k, m,
+                                            kwin, win_rows, n_win, q_pos, sink, B, n_q, h, out);
+    if (st != CSA_OK)
+        return st;
     const size_t need = csa_mqa_workspace_size(B, n_q, h, kv.c, (int64_t)k + n_win);
     if (need > kScratchBytes) {
         char msg[200];

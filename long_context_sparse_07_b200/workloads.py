@@ -23,6 +23,8 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Dict, Iterable, Optional
 
 import numpy as np
@@ -134,21 +136,46 @@ def _gen(seed: int, tid: int, chunk: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(ss))
 
 
+_POOL: Optional[ThreadPoolExecutor] = None
+
+
+def _pool() -> ThreadPoolExecutor:
+    global _POOL
+    if _POOL is None:
+        _POOL = ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1))
+    return _POOL
+
+
 def _rows(seed: int, name: str, rows: int, cols: int, draw, lo: int = 0,
-          hi: Optional[int] = None, dtype=np.float32) -> np.ndarray:
-    """Rows [lo, hi) of a [rows, cols] array drawn chunk by chunk."""
+          hi: Optional[int] = None, dtype=np.float32, out=None):
+    """Rows [lo, hi) of a [rows, cols] array drawn chunk by chunk. Chunks are
+    independent streams, so they are drawn on a thread pool (numpy's
+    generators release the GIL); the values do not depend on the pool.
+    With ``out`` (a torch tensor [hi - lo, cols]) each drawn chunk is cast
+    into it (RNE, element by element) instead of returning float32 rows."""
     hi = rows if hi is None else hi
     tid = _TENSOR_IDS[name]
-    out = np.empty((hi - lo, cols), dtype=dtype)
+    if out is None:
+        out = np.empty((hi - lo, cols), dtype=dtype)
     c0 = lo // ROW_CHUNK
     c1 = (hi + ROW_CHUNK - 1) // ROW_CHUNK
-    for ch in range(c0, c1):
+
+    def one(ch):
         r0 = ch * ROW_CHUNK
         r1 = min(rows, r0 + ROW_CHUNK)
         block = draw(_gen(seed, tid, ch), (r1 - r0, cols))
         a = max(lo, r0)
         b = min(hi, r1)
-        out[a - lo:b - lo] = block[a - r0:b - r0]
+        if isinstance(out, torch.Tensor):
+            out[a - lo:b - lo] = torch.from_numpy(block[a - r0:b - r0]).to(out.dtype)
+        else:
+            out[a - lo:b - lo] = block[a - r0:b - r0]
+
+    if c1 - c0 > 1:
+        list(_pool().map(one, range(c0, c1)))
+    else:
+        for ch in range(c0, c1):
+            one(ch)
     return out
 
 
@@ -156,6 +183,18 @@ def normal(seed, name, rows, cols, std, lo=0, hi=None) -> np.ndarray:
     def draw(g, shape):
         return (g.standard_normal(shape, dtype=np.float32) * np.float32(std))
     return _rows(seed, name, rows, cols, draw, lo, hi)
+
+
+def normal_as(seed, name, rows, cols, std, dtype: str, lo=0, hi=None) -> torch.Tensor:
+    """``to_storage(normal(...), dtype)`` with the cast done chunk by chunk
+    (same bits, without the whole float32 array in host memory)."""
+    hi = rows if hi is None else hi
+    out = torch.empty((hi - lo, cols), dtype={"f32": torch.float32, "bf16": torch.bfloat16}[dtype])
+
+    def draw(g, shape):
+        return (g.standard_normal(shape, dtype=np.float32) * np.float32(std))
+    _rows(seed, name, rows, cols, draw, lo, hi, out=out)
+    return out
 
 
 def uniform(seed, name, rows, cols, lo=0, hi=None) -> np.ndarray:
@@ -223,8 +262,8 @@ def csa_operands(w: Workload, lo: int = 0, hi: Optional[int] = None,
                                    w.idx_dtype).view(hi - lo, w.hI, w.cI)
         out["wI"] = to_storage(normal(s, "wI", n, w.hI, w.std_w, lo, hi), "f32")
     if "query" in parts:
-        out["q"] = to_storage(normal(s, "q", n, w.h * w.c, w.std_q, lo, hi),
-                              w.dtype).view(hi - lo, w.h, w.c)
+        out["q"] = normal_as(s, "q", n, w.h * w.c, w.std_q, w.dtype, lo,
+                             hi).view(hi - lo, w.h, w.c)
         out["sink"] = to_storage(normal(s, "sink", 1, w.h, 1.0), "f32").view(w.h)
     return out
 
@@ -242,8 +281,8 @@ def hca_operands(w: Workload, lo: int = 0, hi: Optional[int] = None,
         out["Z"] = to_storage(normal(s, "Z", n, w.c, w.std_proj, lo, hi), w.dtype)
         out["B"] = to_storage(normal(s, "B", w.m, w.c, w.std_bias), "f32")
     if "query" in parts:
-        out["q"] = to_storage(normal(s, "q", n, w.h * w.c, w.std_q, lo, hi),
-                              w.dtype).view(hi - lo, w.h, w.c)
+        out["q"] = normal_as(s, "q", n, w.h * w.c, w.std_q, w.dtype, lo,
+                             hi).view(hi - lo, w.h, w.c)
         out["sink"] = to_storage(normal(s, "sink", 1, w.h, 1.0), "f32").view(w.h)
     return out
 

@@ -106,3 +106,17 @@ def test_product_path_does_not_touch_the_oracle():
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
                 assert "csa_oracle" not in src, f
+
+
+def test_wait_probe_rejects_limits_outside_its_range(lib):
+    assert lib.csa_debug_wait_probe(10, None) == -1
+    assert b"limit_ns" in lib.csa_last_message()
+    assert lib.csa_debug_wait_probe(5 * 10 ** 9, None) == -1
+
+
+def test_no_alloc_validates_before_touching_the_device(lib):
+    P = 0x10000
+    kv = _entries(c=512)
+    st = lib.csa_sparse_mqa_noalloc(P, abi.CSA_BF16, kv, 10, 4, None, 5, P, 10, None, 4, P, P, 1,
+                                    4, 8, 0.1, P, None, None)
+    assert st == -1 and b"idx" in lib.csa_last_message()

@@ -2,15 +2,17 @@
 (through the C ABI) against the oracle's own chain of steps, each side starting
 from the same generated operands.
 
-Selections: where the oracle's k-th and (k+1)-th scores are separated by more
-than the score tolerance the selected set is unique and must match exactly;
-elsewhere the GPU's set must be a valid top-k within that tolerance (every
-chosen entry scores at least the oracle's k-th score minus the tolerance). The
-share of such near-tie rows is bounded. First, the oracle's top-k over the
-GPU's own float32 scores must be the GPU's selection exactly. Attention
+Scores: the oracle's indexer over the GPU's own indexer keys must match every
+visible GPU score to SCORE_REL of the row scale (only the accumulation order
+differs); against the oracle's own keys (which may sit one storage code away)
+a looser bound holds. Selections, first level: the oracle's top-k over the
+GPU's own float32 scores must be the GPU's selection exactly. Second level:
+against the oracle's float64 scores, every entry the two sides disagree on
+must sit at the selection boundary, within twice the row's measured score
+error of the k-th score (or 1e-6 of it); the gaps are printed. Attention
 outputs are compared with the oracle's on every row whose selection matches
-the oracle's, and on every sampled row with the oracle's attention over the
-GPU's own selection.
+the oracle's chain, and on every sampled row with the oracle's attention over
+the GPU's own selection.
 """
 import math
 
@@ -26,25 +28,41 @@ from helpers import assert_close_out, sample_rows, score_scale, to_np, SCORE_REL
 pytestmark = pytest.mark.gpu
 
 
-def check_selection(gpu_idx, ref_idx, ref_scores, V, k, tol, max_tie_share=0.05):
-    """Returns the rows whose selection equals the oracle's."""
+def check_selection(gpu_idx, ref_idx, ref_scores, gpu_scores, V, k, what):
+    """Second-level selection check against the oracle's float64 scores.
+
+    Returns the rows whose selection equals the oracle's. On a row that
+    differs, every entry the two sides disagree on must sit at the selection
+    boundary: its float64 score lies within `band` of the oracle's k-th
+    score, band = max(1e-6 |kth|, 2 err), err = the row's largest
+    |GPU score - float64 score| over its visible entries (the GPU selects
+    exactly on its own scores, checked at the first level, so a swap needs a
+    gap no larger than twice the score error). The relative gap of each
+    differing row is printed."""
     same = np.zeros(len(V), dtype=bool)
     for r in range(len(V)):
         g, o = gpu_idx[r], ref_idx[r]
         if np.array_equal(g, o):
             same[r] = True
             continue
-        assert V[r] > k, "row %d: short row must select everything" % r
+        assert V[r] > k, "%s row %d: short row must select everything" % (what, r)
         sel = g[g >= 0]
         assert len(sel) == k and len(np.unique(sel)) == k and sel.max() < V[r], r
         row = ref_scores[r, :V[r]]
         kth = np.sort(row)[::-1][k - 1]
-        assert (row[sel] >= kth - 2 * tol[r]).all(), "row %d: invalid selection" % r
-    assert (~same).mean() <= max_tie_share, "near-tie rows %.3f" % (~same).mean()
+        err = np.abs(gpu_scores[r, :V[r]] - row).max()
+        diff = np.setxor1d(sel, o[o >= 0])
+        gap = np.abs(row[diff] - kth).max()
+        band = max(1e-6 * abs(kth), 2 * err)
+        print("%s row %d: %d entries swapped at the boundary; max |score - kth| = %.3g "
+              "(%.3g of |kth|), row score error %.3g (%.3g of |kth|)"
+              % (what, r, len(diff) // 2, gap, gap / abs(kth), err, err / abs(kth)))
+        assert gap <= band, "%s row %d: swap beyond the score error" % (what, r)
+    print("%s: %d of %d rows select exactly the oracle's set" % (what, same.sum(), len(V)))
     return same
 
 
-def run_csa(w, rows, seed_rows_note=""):
+def run_csa(w, rows):
     ops = W.csa_operands(w)
     p = path.CsaPrefill(w, ops)
     p.step()
@@ -52,32 +70,55 @@ def run_csa(w, rows, seed_rows_note=""):
     ref = pipeline.csa_prefill(ops, w, rows)
     # compressed KV entries (full)
     assert_close_out(to_np(p.entries.body), ref["entries"], w.dtype, "entries")
-    # indexer keys
+    # indexer keys: the GPU's float32 compressor output may round to the
+    # neighbouring bf16 value or e4m3 code of the oracle's (one e4m3 code is
+    # up to 2^-3 relative, hence the loose relative bound here)
     if w.idx_dtype == "e4m3":
         kI = oracle.dequantize(p.kI.body.cpu(), p.kI.scale.cpu().view(-1, 1), w.cI)
     else:
         kI = to_np(p.kI.body)
     np.testing.assert_allclose(kI, ref["kI"], rtol=0.13, atol=1e-2)
-    # scores on the sampled rows
     qv, wv = pipeline._indexer_operands(ops, rows, w)
-    S = score_scale(qv, wv, np.abs(ref["kI"]).max())
-    sc = p.scores[0][torch.as_tensor(rows, device="cuda")].cpu().double().numpy()
+    sel_rows = torch.as_tensor(rows, device="cuda")
+    sc = p.scores[0][sel_rows].cpu().double().numpy()
     V = np.array([oracle.visible(t, w.m, w.E) for t in rows])
-    close = []
+    pos = np.asarray(rows).reshape(1, -1)
+    # scores on exactly the GPU's inputs: the oracle's indexer over the GPU's
+    # own keys; only the float32 accumulation order differs, so every visible
+    # score is held to SCORE_REL * S_t
+    own = oracle.indexer(qv[None], wv[None], kI[None], pos, w.m)[0]
+    S = score_scale(qv, wv, np.abs(kI).max())
+    worst = 0.0
+    for r in range(len(rows)):
+        if not V[r]:
+            continue
+        d = np.abs(sc[r, :V[r]] - own[r, :V[r]])
+        worst = max(worst, d.max() / S[r])
+        assert (d <= SCORE_REL * S[r] + 1e-30).all(), "row %d: score error %.3g S_t" % (
+            r, d.max() / S[r])
+    print("%s: largest score error over the GPU's own keys %.3g S_t" % (w.name, worst))
+    # scores against the oracle's whole chain (its own keys): a key one
+    # storage code away moves a score by at most sum_h |w| |qI_h . dk|, which
+    # stays under 5e-3 S_t for these operand laws
+    Sref = score_scale(qv, wv, np.abs(ref["kI"]).max())
     for r in range(len(rows)):
         d = np.abs(sc[r, :V[r]] - ref["scores"][r, :V[r]])
-        assert (d <= 5e-3 * S[r] + 1e-30).all()
-        close.append((d <= SCORE_REL * S[r]).mean() if V[r] else 1.0)
-    assert np.mean(close) > 0.99
-    gidx = p.idx[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+        assert (d <= 5e-3 * Sref[r] + 1e-30).all()
+    gidx = p.idx[sel_rows].cpu().numpy()
     # selection, first level: the oracle's top-k over the GPU's own float32
     # score rows is the GPU's selection exactly (same values, same tie rule)
     np.testing.assert_array_equal(gidx, oracle.topk(sc, rows, w.m, w.k))
-    # second level: against the oracle's float64 scores, differences are near ties
-    same = check_selection(gidx, ref["idx"], ref["scores"], V, w.k, 5e-3 * S)
-    out = p.out[0][torch.as_tensor(rows, device="cuda")]
+    # second level, on the GPU's keys: the oracle's float64 selection over the
+    # same keys differs only at the boundary, within the score error
+    own_idx = oracle.topk(own.astype(np.float32).astype(np.float64), rows, w.m, w.k)
+    check_selection(gidx, own_idx, own, sc, V, w.k, w.name + " (GPU keys)")
+    # against the oracle's whole chain: rows with the same selection compare
+    # outputs directly
+    same = np.array([np.array_equal(gidx[r], ref["idx"][r]) for r in range(len(rows))])
+    print("%s: %d of %d rows select the oracle chain's set" % (w.name, same.sum(), len(rows)))
+    out = p.out[0][sel_rows]
     assert_close_out(to_np(out)[same], ref["out"][same], w.dtype, "out")
-    lse = p.lse[0][torch.as_tensor(rows, device="cuda")].cpu().double().numpy()
+    lse = p.lse[0][sel_rows].cpu().double().numpy()
     np.testing.assert_allclose(lse[same], ref["lse"][same], rtol=1e-3, atol=1e-3)
     # every sampled row against the oracle's attention over the GPU's own
     # selection, so that a tolerated near tie cannot hide an output error
@@ -100,7 +141,7 @@ def test_csa_bf16_n4096_sampled():
 
 def test_csa_fp8idx_n131072_sampled():
     w = W.WORKLOADS["csa_fp8idx_n131072"]
-    run_csa(w, sample_rows(w.n, w.m, 48, 5))
+    run_csa(w, sample_rows(w.n, w.m, 512, 5))
 
 
 def test_hca_bf16_n65536_sampled():
@@ -136,8 +177,7 @@ def test_decode_b8_ctx1m():
     gidx = p.idx.cpu().numpy()
     np.testing.assert_array_equal(gidx, oracle.topk(sc, ops["q_pos"].numpy().reshape(B), w.m,
                                                     w.k))
-    same = check_selection(gidx, ref["idx"], ref["scores"], V, w.k,
-                           SCORE_REL * S, max_tie_share=0.5)
+    same = check_selection(gidx, ref["idx"], ref["scores"], sc, V, w.k, "decode")
     assert_close_out(to_np(p.out)[same], ref["out"][same], "bf16", "csa out")
     ent = pipeline.split_entries(ops["kv_nope"], ops["kv_scale"], ops["kv_rope"], w.scale_group)
     o2, _ = oracle.attend(ops["q"], ent, gidx, w.k, w.m, ops["kwin"], ops["win_pos0"], w.n_win,

@@ -81,8 +81,32 @@ def test_no_alloc_matches_workspace_call_twice_in_a_row():
     assert not torch.equal(got1, got2)
 
 
+def test_no_alloc_serves_the_8_query_decode_step():
+    """The decode step of the 1M-token workload (8 queries, 64 heads, 1024
+    selected entries, 128 window rows) fits the fixed scratch."""
+    abi.csa_get_error()
+    cs = _case(64, B=8, E=8192, k=1024, n_win=128)
+    ref, lref = _with_workspace(cs)
+    got, lgot = _no_alloc(cs)
+    abi.csa_get_error()
+    assert_close_out(to_np(got), to_np(ref), "bf16", "no-alloc vs workspace (B=8)")
+    np.testing.assert_allclose(lgot.cpu().numpy(), lref.cpu().numpy(), rtol=0, atol=2.0 ** -8)
+
+
+def test_no_alloc_checks_arguments_before_sizing_its_scratch():
+    cs = _case(65, B=2, E=1024)
+    bad = Entries(cs["kv"].body, 4096, scale=cs["kv"].scale, rope=cs["kv"].rope, rope_dims=64,
+                  scale_group=64)
+    out = torch.empty_like(cs["q"])
+    with pytest.raises(abi.CsaError) as ei:
+        abi.csa_sparse_mqa_noalloc(cs["q"], bad, cs["E"], cs["m"], cs["idx"], cs["k"],
+                                   cs["kwin"], cs["win_pos0"], cs["n_win"], cs["q_pos"],
+                                   cs["sink"], cs["scale"], out)
+    assert ei.value.status in (-1, -2) and "scratch" not in str(ei.value)
+
+
 def test_no_alloc_refuses_shapes_beyond_its_scratch():
-    cs = _case(63, B=8, E=20000, k=4096)
+    cs = _case(63, B=16, E=20000, k=4096)
     B, n_q, h, c = cs["q"].shape
     assert abi.csa_mqa_workspace_size(B, n_q, h, c, cs["k"] + cs["n_win"]) > \
         abi.csa_noalloc_scratch_bytes()
