@@ -44,6 +44,8 @@ _TENSOR_IDS = {
     "kv_nope": 21, "kv_scale": 22, "kv_rope": 23, "kI": 24, "kI_scale": 25,
     "kwin": 26, "hca_nope": 27, "hca_scale": 28, "hca_rope": 29,
     "scores": 30, "idx_u": 31, "entries": 32, "kwin_step": 33,
+    "H": 40, "W_aKV": 41, "W_bKV": 42, "W_aZ": 43, "W_bZ": 44, "W_aKI": 45, "W_bKI": 46,
+    "W_aZI": 47, "W_bZI": 48, "W_DQ": 49, "W_IUQ": 50, "W_w": 51, "W_UQ": 52,
 }
 
 
@@ -120,6 +122,57 @@ WORKLOADS: Dict[str, Workload] = {
         std_proj=1.0, std_bias=0.0, std_q=1.0, std_w=1.0, batch=8,
         m_hca=128, rope_dims=64, scale_group=64),
 }
+
+
+@dataclasses.dataclass(frozen=True)
+class Layer:
+    """Hidden size d and query latent width d_c of a workload's layer, and the
+    law of its weights: std_w (None: 1/sqrt(fan_in)) and of its biases."""
+    d: int
+    dc: int
+    std_w: Optional[float]
+    std_bias: float
+
+
+# The whole-layer form of the two small CSA workloads: the operands of the
+# path are projections of a hidden state H ~ N(0, 1) (the 256-token fp32 case:
+# d = 128, weights N(0, 1/fan_in), no low-rank query stated, so the latent is
+# full width d_c = d; the 4096-token bf16 case: d = 2048, low-rank query of
+# rank 256, weights and biases N(0, 0.02^2)).
+LAYERS: Dict[str, Layer] = {
+    "csa_fp32_n256": Layer(d=128, dc=128, std_w=None, std_bias=math.sqrt(1.0 / 128)),
+    "csa_bf16_n4096": Layer(d=2048, dc=256, std_w=0.02, std_bias=0.02),
+}
+
+
+def layer_draws(w: Workload, layer: Optional[Layer] = None) -> Dict[str, np.ndarray]:
+    """Hidden state and weights of one CSA layer (float32 draws, no arithmetic
+    of the method): H [n, d]; KV compressor W_aKV, W_bKV, W_aZ, W_bZ [d, c]
+    and biases Ba, Bb [m, c]; indexer-key compressor W_aKI, W_bKI, W_aZI,
+    W_bZI [d, cI] and BIa, BIb [m, cI]; query latent W_DQ [d, dc]; indexer
+    query W_IUQ [dc, hI * cI] and head weights W_w [d, hI]; attention query
+    W_UQ [dc, h * c]; sink [h]."""
+    L = LAYERS[w.name.split("@")[0]] if layer is None else layer
+    s, d, dc = w.seed, L.d, L.dc
+
+    def wstd(fan_in):
+        return L.std_w if L.std_w is not None else math.sqrt(1.0 / fan_in)
+
+    out = {"H": normal(s, "H", w.n, d, 1.0)}
+    for nm in ("W_aKV", "W_bKV", "W_aZ", "W_bZ"):
+        out[nm] = normal(s, nm, d, w.c, wstd(d))
+    for nm in ("W_aKI", "W_bKI", "W_aZI", "W_bZI"):
+        out[nm] = normal(s, nm, d, w.cI, wstd(d))
+    out["W_DQ"] = normal(s, "W_DQ", d, dc, wstd(d))
+    out["W_IUQ"] = normal(s, "W_IUQ", dc, w.hI * w.cI, wstd(dc))
+    out["W_w"] = normal(s, "W_w", d, w.hI, wstd(d))
+    out["W_UQ"] = normal(s, "W_UQ", dc, w.h * w.c, wstd(dc))
+    for nm in ("Ba", "Bb"):
+        out[nm] = normal(s, nm, w.m, w.c, L.std_bias)
+    for nm in ("BIa", "BIb"):
+        out[nm] = normal(s, nm, w.m, w.cI, L.std_bias)
+    out["sink"] = normal(s, "sink", 1, w.h, 1.0).reshape(w.h)
+    return out
 
 
 def scaled(w: Workload, **changes) -> Workload:

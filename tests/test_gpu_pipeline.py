@@ -62,12 +62,14 @@ def check_selection(gpu_idx, ref_idx, ref_scores, gpu_scores, V, k, what):
     return same
 
 
-def run_csa(w, rows):
-    ops = W.csa_operands(w)
+def run_csa(w, rows, ops=None, ref=None):
+    """GPU path on `ops` (default: the workload's drawn operands) against the
+    oracle's chain `ref` (default: the chain over the same operands)."""
+    ops = W.csa_operands(w) if ops is None else ops
     p = path.CsaPrefill(w, ops)
     p.step()
     abi.csa_get_error()
-    ref = pipeline.csa_prefill(ops, w, rows)
+    ref = pipeline.csa_prefill(ops, w, rows) if ref is None else ref
     # compressed KV entries (full)
     assert_close_out(to_np(p.entries.body), ref["entries"], w.dtype, "entries")
     # indexer keys: the GPU's float32 compressor output may round to the
@@ -142,6 +144,53 @@ def test_csa_bf16_n4096_sampled():
 def test_csa_fp8idx_n131072_sampled():
     w = W.WORKLOADS["csa_fp8idx_n131072"]
     run_csa(w, sample_rows(w.n, w.m, 512, 5))
+
+
+def harness_projections(draws, w):
+    """The projections before the path (Eq. 9-10, 13-15, 18), computed on the
+    test harness's side with float64 torch matmuls on the GPU, rounded to
+    float32 and then to the storage dtype: the same definition the oracle's
+    layer computes with numpy, done independently."""
+    dev = torch.device("cuda")
+    t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev, torch.float64)
+         for k, v in draws.items()}
+    H = t["H"]
+    n = H.shape[0]
+
+    def store(x, dt):
+        x = x.to(torch.float32)
+        return (x.to(torch.bfloat16) if dt == "bf16" else x).cpu()
+
+    ops = {}
+    for a, b in (("Ca", "W_aKV"), ("Cb", "W_bKV"), ("Za", "W_aZ"), ("Zb", "W_bZ")):
+        ops[a] = store(H @ t[b], w.dtype)
+    for a, b in (("CIa", "W_aKI"), ("CIb", "W_bKI"), ("ZIa", "W_aZI"), ("ZIb", "W_bZI")):
+        ops[a] = store(H @ t[b], w.idx_dtype)
+    cQ = H @ t["W_DQ"]
+    ops["qI"] = store(cQ @ t["W_IUQ"], w.idx_dtype).view(n, w.hI, w.cI)
+    ops["wI"] = store(H @ t["W_w"], "f32")
+    ops["q"] = store(cQ @ t["W_UQ"], w.dtype).view(n, w.h, w.c)
+    for k in ("Ba", "Bb", "BIa", "BIb", "sink"):
+        ops[k] = torch.from_numpy(np.ascontiguousarray(draws[k], dtype=np.float32))
+    return ops
+
+
+@pytest.mark.parametrize("name,count", [("csa_fp32_n256", None), ("csa_bf16_n4096", 256)])
+def test_whole_layer_from_hidden_state(name, count):
+    """The path on operands projected from one hidden state H (correlated as
+    in a real layer) against the oracle's whole layer from the same H."""
+    from oracle import layer
+    w = W.WORKLOADS[name]
+    draws = W.layer_draws(w)
+    ops = harness_projections(draws, w)
+    rows = np.arange(w.n) if count is None else sample_rows(w.n, w.m, count, 8)
+    ref = layer.csa_layer(draws, w, rows)
+    moved = sum(int((ops[k].double() != ref["ops"][k].double()).sum()) for k in ops)
+    total = sum(v.numel() for v in ops.values())
+    print("%s: %d of %d projected inputs round differently on the two sides" % (
+        name, moved, total))
+    assert moved <= total * 1e-6
+    run_csa(w, rows, ops=ops, ref=ref)
 
 
 def test_hca_bf16_n65536_sampled():
