@@ -8,17 +8,25 @@
 // K = c_I (bf16: kind::f16, 16 per MMA; e4m3: kind::f8f6f4, 32 per MMA).
 // The epilogue thread that owns a key lane then reduces over heads inside
 // its registers: I[t][s] = kscale[s] * sum_h w'[t][h] * ReLU(D[s][(t, h)]),
-// with w' = wI * qI_scale (scales are positive, so they commute with ReLU).
+// with w' = wI * qI_scale (scales are positive, so they commute with ReLU);
+// pairs of heads go through one packed fp32 FMA (fma.rn.f32x2).
+//
+// A block owns NSUB x NT tokens: every key tile in shared memory feeds NSUB
+// MMAs of N = NT x HI (one per group of NT tokens), so a key tile is read
+// from L2 once per NSUB x NT tokens. The accumulators of consecutive
+// (key tile, token group) pairs alternate between two TMEM buffers, so the
+// epilogue of one overlaps the MMA of the next.
 //
 // Warp roles: warp 0 issues TMA loads (query tile once, then a ring of
-// key-tile stages), warp 1 owns TMEM and issues the MMAs into two
-// accumulator buffers, warps 2.. drain the accumulators and write score rows,
-// overlapping the next tile's MMAs: four warps per TMEM lane quarter when a
-// tile holds 4 or more tokens (each takes a quarter of the tokens), since the
-// head reduction costs more than the MMAs that feed it. Key tiles
-// past the causal bound of every token of the tile are never loaded; score
-// entries s >= V_t are not written. Every wait is bounded; on expiry the
-// block records CSA_ERR_TIMEOUT, drains its own copies and returns.
+// key-tile stages), warp 1 owns TMEM and issues the MMAs, warps 2.. drain the
+// accumulators and write score rows: four warps per TMEM lane quarter when a
+// token group holds 4 or more tokens (each takes a quarter of the tokens),
+// since the head reduction costs more than the MMAs that feed it. Key tiles
+// past the causal bound of every token of the block are never loaded; score
+// entries s >= V_t are not written. Token blocks are launched longest first
+// (the causal triangle makes the last tokens' rows the longest). Every wait
+// is bounded; on expiry the block records CSA_ERR_TIMEOUT, drains its own
+// copies and returns.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -40,50 +48,81 @@ struct TcArgs {
     unsigned *err;
 };
 
-template <bool FP8, int HI, int NT>
+template <bool FP8, int HI, int NT, int NSUB>
 struct Cfg {
-    static constexpr int N = NT * HI;
+    static constexpr int N = NT * HI;          // columns of one accumulator
+    static constexpr int TT = NT * NSUB;       // tokens of a block
+    static constexpr int QROWS = TT * HI;      // query rows (token, head) of a block
     // epilogue warps per TMEM lane quarter; each drains NT / SPLIT tokens
     static constexpr int SPLIT = NT >= 4 ? 4 : NT;
     static constexpr int TPW = NT / SPLIT;
     static constexpr int THREADS = 32 * (2 + 4 * SPLIT);
-    static constexpr int STAGES = FP8 ? 6 : 4;
+    static constexpr int STAGES = FP8 ? (NSUB > 1 ? 4 : 6) : 4;
     static constexpr int TMEM_COLS = (2 * N) < 32 ? 32 : 2 * N;
     static constexpr uint32_t IDESC = FP8 ? tc::idesc_e4m3(128, N) : tc::idesc_bf16(128, N);
     static size_t smem_bytes(int kb)
     {
-        return 1024 + (size_t)kb * N * 128 + (size_t)STAGES * kb * 16384 + 256 + N * 4 + NT * 8;
+        return 1024 + (size_t)kb * QROWS * 128 + (size_t)STAGES * kb * 16384 + 256 + QROWS * 4 +
+               TT * 8;
     }
 };
 
-template <bool FP8, int HI, int NT>
-__global__ void __launch_bounds__(Cfg<FP8, HI, NT>::THREADS, 1)
+// sum_h w[h] * max(x[h], 0) over HI heads (x: raw TMEM words), two heads per
+// packed fp32 FMA, two independent accumulator pairs.
+template <int HI>
+__device__ __forceinline__ float relu_dot(const uint32_t *x, const float *w)
+{
+    uint64_t acc0 = 0, acc1 = 0;           // (+0.f, +0.f)
+#pragma unroll
+    for (int j = 0; j < HI; j += 4) {
+        const float4 wv = *(const float4 *)(w + j);
+        uint64_t xa, xb, wa, wb;
+        asm("mov.b64 %0, {%1, %2};" : "=l"(xa) : "f"(fmaxf(__uint_as_float(x[j]), 0.f)),
+            "f"(fmaxf(__uint_as_float(x[j + 1]), 0.f)));
+        asm("mov.b64 %0, {%1, %2};" : "=l"(xb) : "f"(fmaxf(__uint_as_float(x[j + 2]), 0.f)),
+            "f"(fmaxf(__uint_as_float(x[j + 3]), 0.f)));
+        asm("mov.b64 %0, {%1, %2};" : "=l"(wa) : "f"(wv.x), "f"(wv.y));
+        asm("mov.b64 %0, {%1, %2};" : "=l"(wb) : "f"(wv.z), "f"(wv.w));
+        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc0) : "l"(xa), "l"(wa));
+        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc1) : "l"(xb), "l"(wb));
+    }
+    asm("add.rn.f32x2 %0, %0, %1;" : "+l"(acc0) : "l"(acc1));
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc0));
+    return lo + hi;
+}
+
+template <bool FP8, int HI, int NT, int NSUB>
+__global__ void __launch_bounds__(Cfg<FP8, HI, NT, NSUB>::THREADS, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmq,
                   const TcArgs a)
 {
-    using C = Cfg<FP8, HI, NT>;
+    using C = Cfg<FP8, HI, NT, NSUB>;
     constexpr int N = C::N;
+    constexpr int TT = C::TT;
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int KB = a.kb;
     uint8_t *sB = smem;
-    uint8_t *sA = sB + (size_t)KB * N * 128;
+    uint8_t *sA = sB + (size_t)KB * C::QROWS * 128;
     uint64_t *bars = (uint64_t *)(sA + (size_t)S * KB * 16384);
     uint64_t *full = bars, *empty = bars + S, *bfull = bars + 2 * S;
     uint64_t *accf = bfull + 1, *acce = accf + 2, *done = acce + 2;
     uint32_t *tmem_slot = (uint32_t *)(done + 1);
     int *abort_flag = (int *)(tmem_slot + 1);
     float *wsm = (float *)(bars + 32);
-    int64_t *vt = (int64_t *)(wsm + N);
+    int64_t *vt = (int64_t *)(wsm + C::QROWS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.y;
-    const int64_t tile = blockIdx.x / a.nchunks;
+    const int64_t ttiles = (a.n_q + TT - 1) / TT;
+    // longest rows first: token block (ttiles - 1) is launched first
+    const int64_t tile = ttiles - 1 - blockIdx.x / a.nchunks;
     const int chunk = blockIdx.x % a.nchunks;
-    const int64_t t0 = tile * NT;
+    const int64_t t0 = tile * TT;
 
-    if (threadIdx.x < NT) {
+    if (threadIdx.x < TT) {
         const int64_t t = t0 + threadIdx.x;
         vt[threadIdx.x] = t < a.n_q ? visible(a.q_pos[(int64_t)b * a.n_q + t], a.m, a.E) : 0;
     }
@@ -92,7 +131,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     __syncthreads();
     int64_t vmax = 0;
 #pragma unroll
-    for (int tt = 0; tt < NT; tt++)
+    for (int tt = 0; tt < TT; tt++)
         vmax = vt[tt] > vmax ? vt[tt] : vmax;
     const int64_t s_begin = (int64_t)chunk * a.key_chunk;
     int64_t s_end = s_begin + a.key_chunk;
@@ -122,7 +161,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         tc::tmem_relinquish();
     }
     if (warp >= 2) {
-        for (int col = threadIdx.x - 64; col < N; col += C::THREADS - 64) {
+        for (int col = threadIdx.x - 64; col < C::QROWS; col += C::THREADS - 64) {
             const int tt = col / HI, hh = col % HI;
             const int64_t t = t0 + tt;
             float wv = 0.f;
@@ -144,12 +183,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         if (lane == 0) {
             // ---------------- producer
             const int xstep = FP8 ? 128 : 64;    // elements per 128-byte block
+            constexpr int QBOX = C::QROWS < 256 ? C::QROWS : 256;
             int issued = 0;
             bool ok = true;
-            tc::mbar_arrive_expect_tx(bfull, (uint32_t)(KB * N * 128));
+            tc::mbar_arrive_expect_tx(bfull, (uint32_t)(KB * C::QROWS * 128));
             for (int kb = 0; kb < KB; kb++)
-                tc::tma_load_2d(sB + (size_t)kb * N * 128, &tmq, bfull, kb * xstep,
-                                (int)(((int64_t)b * a.n_q + t0) * HI));
+                for (int r0 = 0; r0 < C::QROWS; r0 += QBOX)
+                    tc::tma_load_2d(sB + ((size_t)kb * C::QROWS + r0) * 128, &tmq, bfull,
+                                    kb * xstep, (int)(((int64_t)b * a.n_q + t0) * HI + r0));
             for (int i = 0; i < ntiles && ok; i++) {
                 const int st = i % S;
                 if (i >= S && !tc::mbar_wait(&empty[st], ((i / S) - 1) & 1, abort_flag)) {
@@ -174,36 +215,42 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // ---------------- MMA issuer
+            // ---------------- MMA issuer: for each key tile, one MMA group per
+            // token group into the next accumulator buffer
             bool ok = tc::mbar_wait(bfull, 0, abort_flag);
             const uint32_t sBa = tc::smem_u32(sB);
             for (int i = 0; i < ntiles && ok; i++) {
-                const int st = i % S, buf = i & 1;
-                if (i >= 2 && !tc::mbar_wait(&acce[buf], ((i / 2) - 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
+                const int st = i % S;
                 if (!tc::mbar_wait(&full[st], (i / S) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                tc::fence_after();
-                const uint32_t d = tmem + (uint32_t)(buf * N);
                 const uint32_t sAa = tc::smem_u32(sA + (size_t)st * KB * 16384);
 #pragma unroll 1
-                for (int kb = 0; kb < KB; kb++) {
-#pragma unroll
-                    for (int kk = 0; kk < 4; kk++) {
-                        const uint64_t ad = tc::sdesc_sw128(sAa + kb * 16384 + kk * 32);
-                        const uint64_t bd = tc::sdesc_sw128(sBa + kb * N * 128 + kk * 32);
-                        if (FP8)
-                            tc::mma_f8(d, ad, bd, C::IDESC, (kb | kk) != 0);
-                        else
-                            tc::mma_f16(d, ad, bd, C::IDESC, (kb | kk) != 0);
+                for (int j = 0; j < NSUB && ok; j++) {
+                    const int g = i * NSUB + j, buf = g & 1;
+                    if (g >= 2 && !tc::mbar_wait(&acce[buf], ((g / 2) - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
                     }
+                    tc::fence_after();
+                    const uint32_t d = tmem + (uint32_t)(buf * N);
+#pragma unroll 1
+                    for (int kb = 0; kb < KB; kb++) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; kk++) {
+                            const uint64_t ad = tc::sdesc_sw128(sAa + kb * 16384 + kk * 32);
+                            const uint64_t bd = tc::sdesc_sw128(
+                                sBa + ((uint32_t)kb * C::QROWS + (uint32_t)j * N) * 128 + kk * 32);
+                            if (FP8)
+                                tc::mma_f8(d, ad, bd, C::IDESC, (kb | kk) != 0);
+                            else
+                                tc::mma_f16(d, ad, bd, C::IDESC, (kb | kk) != 0);
+                        }
+                    }
+                    tc::mma_commit(&accf[buf]);
                 }
                 tc::mma_commit(&empty[st]);
-                tc::mma_commit(&accf[buf]);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -215,56 +262,58 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             static_cast<void>(tc::mbar_wait(done, 0, &never, 200000000ull));
         }
     } else {
-        // ---------------- epilogue: warps 2.., lane quarter = warp % 4, tokens
-        // part * TPW .. part * TPW + TPW - 1 of the tile
+        // ---------------- epilogue: warps 2.., lane quarter = warp % 4; in each
+        // token group, tokens part * TPW .. part * TPW + TPW - 1
         const int q4 = warp & 3;
         const int part = (warp - 2) >> 2;
         const int row = q4 * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
-        for (int i = 0; i < ntiles; i++) {
-            const int buf = i & 1;
-            if (!tc::mbar_wait(&accf[buf], (i / 2) & 1, abort_flag)) {
-                *abort_flag = 1;
-                report(a.err, CSA_ERR_TIMEOUT, K_INDEXER_TC, blockIdx.x, 2);
-                break;
-            }
-            tc::fence_after();
+        bool ok = true;
+        for (int i = 0; i < ntiles && ok; i++) {
             const int64_t s = s_begin + (int64_t)i * 128 + row;
+            // the key's scale is requested before the wait for its accumulator
             float ks = 1.f;
             if (FP8)
-                ks = s < a.E ? a.kI_scale[(int64_t)b * a.E + s] : 0.f;
-            const uint32_t base = lane_addr + (uint32_t)(buf * N);
-#pragma unroll
-            for (int u = 0; u < C::TPW; u++) {
-                const int tt = part * C::TPW + u;
-                float sacc = 0.f;
-                if constexpr (HI >= 32) {
-                    uint32_t r[HI / 32][32];
-#pragma unroll
-                    for (int cc = 0; cc < HI / 32; cc++)
-                        tc::tmem_ld32(base + (uint32_t)(tt * HI + cc * 32), r[cc]);
-                    tc::tmem_ld_wait();
-#pragma unroll
-                    for (int cc = 0; cc < HI / 32; cc++)
-#pragma unroll
-                        for (int j = 0; j < 32; j++)
-                            sacc += wsm[tt * HI + cc * 32 + j] * fmaxf(__uint_as_float(r[cc][j]), 0.f);
-                } else {
-                    uint32_t r[16];
-                    tc::tmem_ld16(base + (uint32_t)(tt * HI), r);
-                    tc::tmem_ld_wait();
-#pragma unroll
-                    for (int j = 0; j < 16; j++)
-                        sacc += wsm[tt * HI + j] * fmaxf(__uint_as_float(r[j]), 0.f);
+                ks = s < a.E ? __ldg(a.kI_scale + (int64_t)b * a.E + s) : 0.f;
+#pragma unroll 1
+            for (int j = 0; j < NSUB; j++) {
+                const int g = i * NSUB + j, buf = g & 1;
+                if (!tc::mbar_wait(&accf[buf], (g / 2) & 1, abort_flag)) {
+                    *abort_flag = 1;
+                    report(a.err, CSA_ERR_TIMEOUT, K_INDEXER_TC, blockIdx.x, 2);
+                    ok = false;
+                    break;
                 }
-                const int64_t t = t0 + tt;
-                if (t < a.n_q && s < vt[tt])
-                    a.scores[((int64_t)b * a.n_q + t) * a.ld + s] = sacc * ks;
+                tc::fence_after();
+                const uint32_t base = lane_addr + (uint32_t)(buf * N);
+#pragma unroll
+                for (int u = 0; u < C::TPW; u++) {
+                    const int tl = part * C::TPW + u;      // token inside the group
+                    const int tt = j * NT + tl;            // token inside the block
+                    float sacc;
+                    if constexpr (HI >= 32) {
+                        uint32_t r[HI];
+#pragma unroll
+                        for (int cc = 0; cc < HI / 32; cc++)
+                            tc::tmem_ld32(base + (uint32_t)(tl * HI + cc * 32),
+                                          *reinterpret_cast<uint32_t(*)[32]>(r + cc * 32));
+                        tc::tmem_ld_wait();
+                        sacc = relu_dot<HI>(r, wsm + tt * HI);
+                    } else {
+                        uint32_t r[16];
+                        tc::tmem_ld16(base + (uint32_t)(tl * HI), r);
+                        tc::tmem_ld_wait();
+                        sacc = relu_dot<16>(r, wsm + tt * HI);
+                    }
+                    const int64_t t = t0 + tt;
+                    if (t < a.n_q && s < vt[tt])
+                        a.scores[((int64_t)b * a.n_q + t) * a.ld + s] = sacc * ks;
+                }
+                tc::fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    tc::mbar_arrive(&acce[buf]);
             }
-            tc::fence_before();
-            __syncwarp();
-            if (lane == 0)
-                tc::mbar_arrive(&acce[buf]);
         }
     }
     tc::fence_before();
@@ -275,16 +324,17 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     }
 }
 
-template <bool FP8, int HI, int NT>
+template <bool FP8, int HI, int NT, int NSUB>
 cudaError_t launch_one(const IndexerArgs &a, unsigned *err, cudaStream_t s)
 {
-    using C = Cfg<FP8, HI, NT>;
+    using C = Cfg<FP8, HI, NT, NSUB>;
     const int esize = FP8 ? 1 : 2;
     CUtensorMap tmk, tmq;
     const CUtensorMapDataType dt =
         FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!make_tmap_2d(&tmk, a.kI.body, dt, esize, (uint64_t)a.B * a.E, a.cI, 128) ||
-        !make_tmap_2d(&tmq, a.qI, dt, esize, (uint64_t)a.B * a.n_q * HI, a.cI, C::N))
+        !make_tmap_2d(&tmq, a.qI, dt, esize, (uint64_t)a.B * a.n_q * HI, a.cI,
+                      C::QROWS < 256 ? C::QROWS : 256))
         return cudaErrorInvalidValue;
     TcArgs t;
     t.wI = a.wI;
@@ -295,7 +345,7 @@ cudaError_t launch_one(const IndexerArgs &a, unsigned *err, cudaStream_t s)
     t.E = a.E;
     t.m = a.m;
     t.kb = a.cI * esize / 128;
-    const int64_t ttiles = (a.n_q + NT - 1) / NT;
+    const int64_t ttiles = (a.n_q + C::TT - 1) / C::TT;
     // few token tiles: split the keys of each tile over several blocks, sized
     // so that all blocks run in one wave (two resident blocks per SM)
     int dev = 0, sms = 148;
@@ -314,22 +364,37 @@ cudaError_t launch_one(const IndexerArgs &a, unsigned *err, cudaStream_t s)
     t.ld = a.ld;
     t.err = err;
     const size_t smem = C::smem_bytes(t.kb);
-    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<FP8, HI, NT>,
+    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<FP8, HI, NT, NSUB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
     dim3 grid((unsigned)(ttiles * t.nchunks), (unsigned)a.B);
-    indexer_tc_kernel<FP8, HI, NT><<<grid, C::THREADS, smem, s>>>(tmk, tmq, t);
+    indexer_tc_kernel<FP8, HI, NT, NSUB><<<grid, C::THREADS, smem, s>>>(tmk, tmq, t);
     return cudaGetLastError();
 }
 
 template <bool FP8>
 cudaError_t dispatch_heads(const IndexerArgs &a, unsigned *err, cudaStream_t s, bool few)
 {
+    // prefill: a block takes 16 tokens (e4m3) or one group of N = 256 (bf16,
+    // whose key tiles are twice the size); decode: one token per block
     switch (a.hI) {
-    case 16: return few ? launch_one<FP8, 16, 1>(a, err, s) : launch_one<FP8, 16, 16>(a, err, s);
-    case 32: return few ? launch_one<FP8, 32, 1>(a, err, s) : launch_one<FP8, 32, 8>(a, err, s);
-    case 64: return few ? launch_one<FP8, 64, 1>(a, err, s) : launch_one<FP8, 64, 4>(a, err, s);
+    case 16:
+        return few ? launch_one<FP8, 16, 1, 1>(a, err, s) : launch_one<FP8, 16, 16, 1>(a, err, s);
+    case 32:
+        if (few)
+            return launch_one<FP8, 32, 1, 1>(a, err, s);
+        if constexpr (FP8)
+            return launch_one<FP8, 32, 8, 2>(a, err, s);
+        else
+            return launch_one<FP8, 32, 8, 1>(a, err, s);
+    case 64:
+        if (few)
+            return launch_one<FP8, 64, 1, 1>(a, err, s);
+        if constexpr (FP8)
+            return launch_one<FP8, 64, 4, 4>(a, err, s);
+        else
+            return launch_one<FP8, 64, 4, 1>(a, err, s);
     }
     return cudaErrorInvalidValue;
 }
