@@ -50,7 +50,8 @@ constexpr int KT = 64;               // keys per tile
 constexpr float kLazy2 = 11.5f;      // lazy-rescale margin, base-2 units (about e^8)
 constexpr int kMmaWarp = 4;
 constexpr int kSoftWarp0 = 5;
-constexpr int kGatherBar = 5;        // named barrier of the 4 gather warps (1..4: head groups)
+constexpr int kGatherBar = 5;        // named barrier of the 4 gather warps (1..4: head groups;
+                                     // 6, 7: the two gather groups)
 
 struct TcAttn {
     const __nv_bfloat16 *ent, *kwin;
@@ -101,8 +102,8 @@ struct Lay {
     static constexpr size_t Q_OFF = 2 * 65536;                      // 4 pairs x 2H x 128
     static constexpr size_t P_OFF = Q_OFF + 8 * H * 128;            // H x 128 (64 keys)
     static constexpr size_t X_OFF = P_OFF + H * 128;                // NG x 8 x 128 floats
-    static constexpr size_t PTR_OFF = X_OFF + NG * 8 * 128 * 4;     // 64 row pointers
-    static constexpr size_t ROW_OFF = PTR_OFF + KT * 8;             // 64 fp8 entry rows
+    static constexpr size_t PTR_OFF = X_OFF + NG * 8 * 128 * 4;     // 2 x 64 row pointers
+    static constexpr size_t ROW_OFF = PTR_OFF + 2 * KT * 8;         // 64 fp8 entry rows
     static constexpr size_t F_OFF = ROW_OFF + KT * 8;               // 8 x H floats
     static constexpr size_t BAR_OFF = F_OFF + ((8 * H * 4 + 63) / 64) * 64;
     static constexpr size_t TOTAL = BAR_OFF + 256;
@@ -155,6 +156,39 @@ __device__ __forceinline__ const __nv_bfloat16 *key_row(const TcAttn &a, const Q
     *entry_row = -1;
     if (j < q.nsel) {
         const int64_t s = a.dense ? j : (int64_t)a.idx[bt * a.k + j];
+        if (s < 0)
+            return nullptr;
+        if (s < q.V) {
+            if (KV8) {
+                *entry_row = q.b * a.E + s;
+                return nullptr;
+            }
+            return a.ent + (q.b * a.E + s) * DIM;
+        }
+        if (report_bad)
+            report(a.err, CSA_ERR_BOUNDS, K_ATTEND_TC, (unsigned)bt, (unsigned)s);
+        return nullptr;
+    }
+    if (j >= q.wbeg && j < q.nk) {
+        const int64_t p = q.w0 + (j - q.wbeg);
+        const int64_t wr = p - q.wp0;
+        if (wr >= 0 && wr < a.win_rows)
+            return a.kwin + (q.b * a.win_rows + wr) * DIM;
+        if (report_bad)
+            report(a.err, CSA_ERR_BOUNDS, K_ATTEND_TC, (unsigned)bt, (unsigned)p);
+    }
+    return nullptr;
+}
+
+// key_row with the selection index of slot j already loaded (slot_index).
+template <bool KV8>
+__device__ __forceinline__ const __nv_bfloat16 *key_row_s(const TcAttn &a, const QInfo &q,
+                                                          int64_t bt, int64_t j, int32_t sidx,
+                                                          bool report_bad, int64_t *entry_row)
+{
+    *entry_row = -1;
+    if (j < q.nsel) {
+        const int64_t s = a.dense ? j : (int64_t)sidx;
         if (s < 0)
             return nullptr;
         if (s < q.V) {
@@ -252,7 +286,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int i = 0; i < 2; i++) {
-            tc::mbar_init(&kfull[i], 128);
+            tc::mbar_init(&kfull[i], KV8 ? 128 : 64);    // one arrival per gather thread of the group
             tc::mbar_init(&kfree[i], 1);
             tc::mbar_init(&sfull[i], 1);
         }
@@ -285,7 +319,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     if (warp < 4) {
         // ------------------------------------------------------------ gather
+        // bf16 entries: two groups of two warps take alternate tiles (group g
+        // fills buffer g), so that one group's copies are in flight while the
+        // other waits for its buffer; fp8 entries: one group of four warps.
+        // The selection indices of a group's next tile are loaded while its
+        // current tile is copied.
+        constexpr int NGRP = KV8 ? 1 : 2;
+        constexpr int GT = 128 / NGRP;               // threads of a group
         const int gt = tid;                          // 0..127
+        const int grp = gt / GT, lt = gt % GT;
+        const int gbar = kGatherBar + 1 + grp;       // the group's own named barrier
+        const __nv_bfloat16 **gptr = kptr + grp * KT;
         const void *zero_src = KV8 ? (a.kwin ? (const void *)a.kwin : (const void *)a.ent8)
                                    : (a.E > 0 ? (const void *)a.ent : (const void *)a.kwin);
         uint32_t t = 0, qctr = 0;
@@ -305,8 +349,18 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     tc::tma_load_2d(sQ + (kb & 3) * (2 * H * 128) + (kb >> 2) * (H * 128), &tm_q,
                                     qfull, kb * 64, (int)(bt * H));
             }
-            for (int i = 0; i < q.ntiles; ++i, ++t) {
-                const int b = t & 1;
+            const uint32_t t_item = t;
+            // this group's first tile of the item
+            int i = (int)((grp - (int)(t_item % NGRP) + NGRP) % NGRP);
+            int32_t s_own = 0, s_first = 0;
+            if (i < q.ntiles && lt < KT) {
+                const int64_t j0 = (int64_t)(q.tile0 + i) * KT;
+                s_own = slot_index(a, q, bt, j0 + lt);
+                s_first = slot_index(a, q, bt, j0);
+            }
+            for (; i < q.ntiles; i += NGRP) {
+                const uint32_t tt = t_item + (uint32_t)i;
+                const int b = tt & 1;
                 uint8_t *kbuf = sK + b * 65536;
                 const int64_t jt0 = (int64_t)(q.tile0 + i) * KT;
                 // A tile whose 64 rows are consecutive rows of one bf16 source
@@ -316,31 +370,37 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 bool run = true;
                 int64_t row0 = 0;
                 const bool src_ent = jt0 < q.nsel;
-                if (gt < KT) {
+                if (lt < KT) {
                     int64_t er, er0;
-                    const __nv_bfloat16 *kp = key_row<KV8>(a, q, bt, jt0 + gt, true, &er);
-                    kptr[gt] = kp;
-                    krow[gt] = er;
-                    const __nv_bfloat16 *p0 = key_row<KV8>(a, q, bt, jt0, false, &er0);
+                    const __nv_bfloat16 *kp = key_row_s<KV8>(a, q, bt, jt0 + lt, s_own, true, &er);
+                    gptr[lt] = kp;
+                    if (KV8)
+                        krow[lt] = er;
+                    const __nv_bfloat16 *p0 = key_row_s<KV8>(a, q, bt, jt0, s_first, false, &er0);
                     const bool src_win = jt0 >= q.wbeg;
-                    const bool same = (jt0 + gt < q.nsel) == src_ent && (jt0 + gt >= q.wbeg) == src_win;
-                    run = p0 != nullptr && same && kp == p0 + (int64_t)gt * DIM;
+                    const bool same = (jt0 + lt < q.nsel) == src_ent && (jt0 + lt >= q.wbeg) == src_win;
+                    run = p0 != nullptr && same && kp == p0 + (int64_t)lt * DIM;
                     const __nv_bfloat16 *base = src_ent ? a.ent : a.kwin;
                     row0 = p0 ? (p0 - base) / DIM : 0;
                     run = run && row0 <= 0x7fffffff - KT && (src_ent ? a.tma_ent : a.tma_win);
                 }
-                const bool all_run = !tc::named_bar_or(kGatherBar, 128, !run);
-                // buffer b is free once the O^T product of tile t - 2 is done
-                // (the row pointers above are worked out before waiting)
-                if (t >= 2) {
-                    const bool fr = tc::mbar_wait(&kfree[b], ((t - 2) >> 1) & 1, abortv);
-                    if (tc::named_bar_or(kGatherBar, 128, !fr)) {
+                const bool all_run = !tc::named_bar_or(gbar, GT, !run);
+                // the group's next tile: its indices are requested now
+                if (i + NGRP < q.ntiles && lt < KT) {
+                    const int64_t jn = jt0 + (int64_t)NGRP * KT;
+                    s_own = slot_index(a, q, bt, jn + lt);
+                    s_first = slot_index(a, q, bt, jn);
+                }
+                // buffer b is free once the O^T product of tile tt - 2 is done
+                if (tt >= 2) {
+                    const bool fr = tc::mbar_wait(&kfree[b], ((tt - 2) >> 1) & 1, abortv);
+                    if (tc::named_bar_or(gbar, GT, !fr)) {
                         ok = false;
                         break;
                     }
                 }
                 if (all_run) {
-                    if (gt == 0) {
+                    if (lt == 0) {
                         tc::mbar_expect_tx(&kfull[b], 65536u);
 #pragma unroll 1
                         for (int kb = 0; kb < 8; kb++)
@@ -351,7 +411,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     // two threads per row: body bytes [224 * half, +224) as 14
                     // pieces of 16 codes (each inside one 64-dim scale group),
                     // decoded to bf16; RoPE dims and bf16 window rows by cp.async
-                    const int row = gt >> 1, half = gt & 1;
+                    const int row = lt >> 1, half = lt & 1;
                     const int64_t er = krow[row];
                     uint8_t *rbase = kbuf + row * 128;
                     if (er >= 0) {
@@ -387,7 +447,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             }
                         }
                     } else {
-                        const __nv_bfloat16 *sp = kptr[row];
+                        const __nv_bfloat16 *sp = gptr[row];
 #pragma unroll 1
                         for (int kb = half * 4; kb < half * 4 + 4; kb++)
 #pragma unroll
@@ -397,31 +457,38 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                                sp ? 16u : 0u);
                     }
                 } else {
-                    // this thread's 4 rows, read once (a pointer re-read from
-                    // shared memory before every copy would serialise the issue)
-                    const __nv_bfloat16 *sp[4];
-                    uint8_t *dp[4];
+                    // this thread's KT * 8 / GT rows, read once (a pointer re-read
+                    // from shared memory before every copy would serialise the issue)
+                    // (destinations as 32-bit shared addresses: row r of a slot
+                    // at r * 128, its 16-byte chunk c at (c ^ (r & 7)) * 16)
+                    constexpr int RPT = KT * 8 / GT;           // rows per thread
+                    const __nv_bfloat16 *sp[RPT];
+                    const int c = lt & 7;
+                    const uint32_t d0 = tc::smem_u32(kbuf) + (uint32_t)(lt >> 3) * 128u;
 #pragma unroll
-                    for (int u = 0; u < 4; u++) {
-                        const int row = u * 16 + (gt >> 3), c = gt & 7;
-                        const __nv_bfloat16 *p = kptr[row];
+                    for (int u = 0; u < RPT; u++) {
+                        const int row = u * (GT / 8) + (lt >> 3);
+                        const __nv_bfloat16 *p = gptr[row];
                         sp[u] = p ? p + c * 8 : nullptr;
-                        dp[u] = kbuf + row * 128 + ((c ^ (row & 7)) << 4);
                     }
 #pragma unroll
                     for (int kb = 0; kb < 8; kb++)
 #pragma unroll
-                        for (int u = 0; u < 4; u++)
-                            tc::cp_async16(dp[u] + slot_of(kb) * 8192,
-                                           sp[u] ? (const void *)(sp[u] + kb * 64) : zero_src,
-                                           sp[u] ? 16u : 0u);
+                        for (int u = 0; u < RPT; u++) {
+                            const int row = u * (GT / 8) + (lt >> 3);
+                            tc::cp_async16_s(d0 + (uint32_t)(u * (GT / 8) * 128 + slot_of(kb) * 8192 +
+                                                             ((c ^ (row & 7)) << 4)),
+                                             sp[u] ? (const void *)(sp[u] + kb * 64) : zero_src,
+                                             sp[u] ? 16u : 0u);
+                        }
                 }
                 tc::cp_async_commit();
                 tc::cp_async_wait_all();
                 tc::fence_async_shared();
                 tc::mbar_arrive(&kfull[b]);
-                tc::named_bar_sync(kGatherBar, 128);     // kptr / krow rewritten next tile
+                tc::named_bar_sync(gbar, GT);     // the group's row pointers rewritten next tile
             }
+            t = t_item + (uint32_t)q.ntiles;
         }
         tc::cp_async_wait_all();
         if (!ok) {

@@ -53,10 +53,17 @@ struct Cfg {
     static constexpr int N = NT * HI;          // columns of one accumulator
     static constexpr int TT = NT * NSUB;       // tokens of a block
     static constexpr int QROWS = TT * HI;      // query rows (token, head) of a block
-    // epilogue warps per TMEM lane quarter; each drains NT / SPLIT tokens
+    // epilogue: SPLIT warps per TMEM lane quarter drain NT / SPLIT tokens
+    // each; with one token per group (decode) two such warp sets drain
+    // alternate accumulators (set s takes those in TMEM buffer s). A token's
+    // HI columns are read in chunks of CW columns, the next chunk loading
+    // while one is reduced.
+    static constexpr int NSET = NT == 1 ? 2 : 1;
     static constexpr int SPLIT = NT >= 4 ? 4 : NT;
     static constexpr int TPW = NT / SPLIT;
-    static constexpr int THREADS = 32 * (2 + 4 * SPLIT);
+    static constexpr int CW = HI < 32 ? HI : 32;
+    static constexpr int CPT = HI / CW;
+    static constexpr int THREADS = 32 * (2 + 4 * NSET * SPLIT);
     static constexpr int STAGES = FP8 ? (NSUB > 1 ? 4 : 6) : 4;
     static constexpr int TMEM_COLS = (2 * N) < 32 ? 32 : 2 * N;
     static constexpr uint32_t IDESC = FP8 ? tc::idesc_e4m3(128, N) : tc::idesc_bf16(128, N);
@@ -72,24 +79,19 @@ struct Cfg {
 template <int HI>
 __device__ __forceinline__ float relu_dot(const uint32_t *x, const float *w)
 {
-    uint64_t acc0 = 0, acc1 = 0;           // (+0.f, +0.f)
+    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < HI; j += 4) {
         const float4 wv = *(const float4 *)(w + j);
-        uint64_t xa, xb, wa, wb;
-        asm("mov.b64 %0, {%1, %2};" : "=l"(xa) : "f"(fmaxf(__uint_as_float(x[j]), 0.f)),
-            "f"(fmaxf(__uint_as_float(x[j + 1]), 0.f)));
-        asm("mov.b64 %0, {%1, %2};" : "=l"(xb) : "f"(fmaxf(__uint_as_float(x[j + 2]), 0.f)),
-            "f"(fmaxf(__uint_as_float(x[j + 3]), 0.f)));
-        asm("mov.b64 %0, {%1, %2};" : "=l"(wa) : "f"(wv.x), "f"(wv.y));
-        asm("mov.b64 %0, {%1, %2};" : "=l"(wb) : "f"(wv.z), "f"(wv.w));
-        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc0) : "l"(xa), "l"(wa));
-        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc1) : "l"(xb), "l"(wb));
+        const float2 xa = make_float2(fmaxf(__uint_as_float(x[j]), 0.f),
+                                      fmaxf(__uint_as_float(x[j + 1]), 0.f));
+        const float2 xb = make_float2(fmaxf(__uint_as_float(x[j + 2]), 0.f),
+                                      fmaxf(__uint_as_float(x[j + 3]), 0.f));
+        acc0 = __ffma2_rn(xa, make_float2(wv.x, wv.y), acc0);
+        acc1 = __ffma2_rn(xb, make_float2(wv.z, wv.w), acc1);
     }
-    asm("add.rn.f32x2 %0, %0, %1;" : "+l"(acc0) : "l"(acc1));
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc0));
-    return lo + hi;
+    acc0 = __fadd2_rn(acc0, acc1);
+    return acc0.x + acc0.y;
 }
 
 template <bool FP8, int HI, int NT, int NSUB>
@@ -149,7 +151,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         tc::mbar_init(bfull, 1);
         for (int i = 0; i < 2; i++) {
             tc::mbar_init(&accf[i], 1);
-            tc::mbar_init(&acce[i], 4 * C::SPLIT);
+            tc::mbar_init(&acce[i], 4 * C::SPLIT);     // the warps that drain buffer i
         }
         tc::mbar_init(done, 1);
         tc::fence_mbar_init();
@@ -262,14 +264,19 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             static_cast<void>(tc::mbar_wait(done, 0, &never, 200000000ull));
         }
     } else {
-        // ---------------- epilogue: warps 2.., lane quarter = warp % 4; in each
-        // token group, tokens part * TPW .. part * TPW + TPW - 1
+        // ---------------- epilogue: warps 2..; set = which TMEM buffer (with
+        // two sets), lane quarter = warp % 4; in each token group, tokens
+        // part * TPW .. part * TPW + TPW - 1
+        constexpr int CW = C::CW, CPT = C::CPT, NC = C::TPW * C::CPT;
         const int q4 = warp & 3;
-        const int part = (warp - 2) >> 2;
+        const int set = (warp - 2) / (4 * C::SPLIT);
+        const int part = ((warp - 2) >> 2) % C::SPLIT;
         const int row = q4 * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
         bool ok = true;
         for (int i = 0; i < ntiles && ok; i++) {
+            if (C::NSET == 2 && NSUB == 1 && (i & 1) != set)
+                continue;
             const int64_t s = s_begin + (int64_t)i * 128 + row;
             // the key's scale is requested before the wait for its accumulator
             float ks = 1.f;
@@ -278,6 +285,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 #pragma unroll 1
             for (int j = 0; j < NSUB; j++) {
                 const int g = i * NSUB + j, buf = g & 1;
+                if (C::NSET == 2 && buf != set)
+                    continue;
                 if (!tc::mbar_wait(&accf[buf], (g / 2) & 1, abort_flag)) {
                     *abort_flag = 1;
                     report(a.err, CSA_ERR_TIMEOUT, K_INDEXER_TC, blockIdx.x, 2);
@@ -286,28 +295,33 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 }
                 tc::fence_after();
                 const uint32_t base = lane_addr + (uint32_t)(buf * N);
+                // chunk c: columns (part * TPW + c / CPT) * HI + (c % CPT) * CW
+                uint32_t rb[2][CW];
+                auto load = [&](int c, uint32_t(&r)[CW]) {
+                    const uint32_t col = (uint32_t)((part * C::TPW + c / CPT) * HI + (c % CPT) * CW);
+                    if constexpr (CW == 32)
+                        tc::tmem_ld32(base + col, r);
+                    else
+                        tc::tmem_ld16(base + col, r);
+                };
+                load(0, rb[0]);
+                tc::tmem_ld_wait();
+                float sacc = 0.f;
 #pragma unroll
-                for (int u = 0; u < C::TPW; u++) {
-                    const int tl = part * C::TPW + u;      // token inside the group
-                    const int tt = j * NT + tl;            // token inside the block
-                    float sacc;
-                    if constexpr (HI >= 32) {
-                        uint32_t r[HI];
-#pragma unroll
-                        for (int cc = 0; cc < HI / 32; cc++)
-                            tc::tmem_ld32(base + (uint32_t)(tl * HI + cc * 32),
-                                          *reinterpret_cast<uint32_t(*)[32]>(r + cc * 32));
-                        tc::tmem_ld_wait();
-                        sacc = relu_dot<HI>(r, wsm + tt * HI);
-                    } else {
-                        uint32_t r[16];
-                        tc::tmem_ld16(base + (uint32_t)(tl * HI), r);
-                        tc::tmem_ld_wait();
-                        sacc = relu_dot<16>(r, wsm + tt * HI);
+                for (int c = 0; c < NC; c++) {
+                    if (c + 1 < NC)
+                        load(c + 1, rb[(c + 1) & 1]);
+                    const int tl = part * C::TPW + c / CPT;   // token inside the group
+                    const int tt = j * NT + tl;               // token inside the block
+                    sacc += relu_dot<CW>(rb[c & 1], wsm + tt * HI + (c % CPT) * CW);
+                    if (c % CPT == CPT - 1) {
+                        const int64_t t = t0 + tt;
+                        if (t < a.n_q && s < vt[tt])
+                            a.scores[((int64_t)b * a.n_q + t) * a.ld + s] = sacc * ks;
+                        sacc = 0.f;
                     }
-                    const int64_t t = t0 + tt;
-                    if (t < a.n_q && s < vt[tt])
-                        a.scores[((int64_t)b * a.n_q + t) * a.ld + s] = sacc * ks;
+                    if (c + 1 < NC)
+                        tc::tmem_ld_wait();
                 }
                 tc::fence_before();
                 __syncwarp();
