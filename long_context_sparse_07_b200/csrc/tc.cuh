@@ -314,19 +314,6 @@ __device__ __forceinline__ void cp_async_wait_all()
 namespace csa {
 namespace tc {
 
-// Four rows (row0..row3) of a 2D tensor map, `x` = first column, each row one
-// box of (128 / esize) columns, landing as 4 consecutive 128-byte rows at
-// `dst` with the map's 128-byte swizzle. The map's box height must be 1.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar,
-                                            int x, int r0, int r1, int r2, int r3)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
-}
-
 // Barrier among the `count` threads of named barrier `id` (id 0 is
 // __syncthreads); returns true on every thread if `pred` held on any.
 __device__ __forceinline__ bool named_bar_or(int id, int count, bool pred)

@@ -7,8 +7,11 @@
 // element with key > T and the first `need` elements with key == T, so each
 // row comes out in ascending index order. Three layouts of the work:
 //  * short rows (<= 2048 visible): one warp per row, keys in registers;
-//  * rows up to 64 K: one block per row, keys staged once in shared memory
-//    when they fit (re-read from L2 otherwise), 12 + 12 + 8-bit digits;
+//  * rows up to 64 K: one block per row; for k <= 1024 the row's candidates
+//    (entries at or above a lower bound taken from a sample of the row) are
+//    kept in shared memory and selected exactly with 8-bit digits; for larger
+//    k the keys are staged once in shared memory when they fit (re-read from
+//    L2 otherwise) and selected with 12 + 12 + 8-bit digits;
 //  * longer rows (decode): chunks of the row over many blocks, then one block
 //    per row over the candidates of the threshold bin.
 #include "common.cuh"
@@ -296,6 +299,329 @@ topk_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
     }
     RowScores src{scores + row * ld};
     block_select(src, V, k, out, keys, resident && V <= kResident, sh);
+}
+
+// ---------------------------------------------------------------------------
+// Rows of 2049 .. 65535 entries (prefill), k <= 1024: one block of 16 warps
+// per row, two blocks per SM.
+//  1. A lower bound L from 1024 samples of the row (16 runs of 64 consecutive
+//     entries spread over it): L is the 16-bit key prefix of the sample that
+//     about 1.25 k + 4 sqrt(.) + 8 of the samples reach, when the row's k-th
+//     largest entry is expected at k * 1024 / V of them.
+//  2. Warp w reads its contiguous segment of the row and keeps the entries
+//     with key >= L, in index order, in its own region of shared memory.
+//  3. The exact top-k of the candidates (8-bit radix digits, histograms
+//     updated once per group of equal digits of a warp), written in index
+//     order: warp w's candidates follow those of warps < w.
+// When the candidates are fewer than k or a warp's region overflows, steps 3
+// run over the row itself (re-read from L2) instead: the result is the exact
+// top-k of the row either way.
+
+constexpr int kMidThreads = 512;
+constexpr int kMidWarps = kMidThreads / 32;
+constexpr int kMidCapW = 512;                 // candidates per warp region
+constexpr int kMidMaxK = 1024;
+
+template <typename IdxT>
+struct SelShared {
+    uint32_t ckey[kMidWarps][kMidCapW];
+    IdxT cidx[kMidWarps][kMidCapW];
+    uint32_t skey[1024];
+    unsigned hist[256];
+    unsigned wcnt[kMidWarps], wpre[kMidWarps], wpre2[kMidWarps];
+    unsigned wgt[kMidWarps], weq[kMidWarps];
+    unsigned bin, need, total;
+    int fallback, last;
+};
+using MidShared = SelShared<uint16_t>;     // rows < 65536: 16-bit indices
+
+// Adds 1 to hist[d] for every lane with `on`, one atomic per distinct d.
+__device__ __forceinline__ void hist_add(unsigned *hist, unsigned d, bool on)
+{
+    const unsigned act = __ballot_sync(0xffffffffu, on);
+    if (on) {
+        const unsigned same = __match_any_sync(act, d);
+        if ((threadIdx.x & 31) == __ffs(same) - 1)
+            atomicAdd(&hist[d], (unsigned)__popc(same));
+    }
+}
+
+// Digit of the 256-bin histogram (descending) where the count from the top
+// reaches `need` (warp 0 scans; every thread reads the result after the
+// barrier): sh.bin and sh.need (what is still needed inside that bin).
+template <typename SH>
+__device__ __forceinline__ void mid_find(SH &sh, unsigned need)
+{
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        unsigned local = 0;
+#pragma unroll
+        for (int j = 0; j < 8; j++)
+            local += sh.hist[255 - 8 * lane - j];
+        unsigned incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += y;
+        }
+        const unsigned excl = incl - local;
+        if (excl < need && need <= incl) {
+            unsigned cum = excl;
+            for (int j = 0; j < 8; j++) {
+                const unsigned hb = sh.hist[255 - 8 * lane - j];
+                if (cum + hb >= need) {
+                    sh.bin = 255u - 8u * lane - j;
+                    sh.need = need - cum;
+                    break;
+                }
+                cum += hb;
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// Exclusive prefix over warps of v (the same value on every lane of a warp):
+// returns this warp's prefix.
+__device__ __forceinline__ unsigned mid_warp_prefix(unsigned *slot, unsigned *pre, unsigned v)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (lane == 0)
+        slot[wid] = v;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const unsigned x = lane < kMidWarps ? slot[lane] : 0u;
+        unsigned incl = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += y;
+        }
+        if (lane < kMidWarps)
+            pre[lane] = incl - x;
+    }
+    __syncthreads();
+    return pre[wid];
+}
+
+// Element j of warp w: from its candidate region, or from its row segment.
+template <typename SH>
+struct MidSrc {
+    const float *row;
+    const SH *sh;
+    int seg, V;
+    bool cand;
+    __device__ __forceinline__ int count(int w) const
+    {
+        if (cand)
+            return (int)sh->wcnt[w];
+        const int a = w * seg, b = a + seg < V ? a + seg : V;
+        return b > a ? b - a : 0;
+    }
+    __device__ __forceinline__ uint32_t key(int w, int j) const
+    {
+        return cand ? sh->ckey[w][j] : float_key(__ldg(row + w * seg + j));
+    }
+    __device__ __forceinline__ int32_t index(int w, int j) const
+    {
+        return cand ? (int32_t)sh->cidx[w][j] : (int32_t)(w * seg + j);
+    }
+};
+
+// Exact top-k of the source (more than k elements in total), written to out
+// in index order; ties at the k-th key go to the lower indices.
+template <typename SH>
+__device__ void mid_select(const MidSrc<SH> &src, int k, int32_t *__restrict__ out, SH &sh)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int n = src.count(wid);
+    uint32_t prefix = 0, pmask = 0;
+    unsigned need = (unsigned)k;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        if (threadIdx.x < 256)
+            sh.hist[threadIdx.x] = 0;
+        __syncthreads();
+        for (int j0 = 0; j0 < n; j0 += 32) {
+            const int j = j0 + lane;
+            const uint32_t u = j < n ? src.key(wid, j) : 0u;
+            hist_add(sh.hist, (u >> shift) & 255u, j < n && (u & pmask) == prefix);
+        }
+        __syncthreads();
+        mid_find(sh, need);
+        prefix |= sh.bin << shift;
+        pmask |= 255u << shift;
+        need = sh.need;
+        __syncthreads();                                   // hist, bin, need reused
+    }
+    const uint32_t T = prefix;
+    // every warp: its count of keys above T and equal to T, then the prefix
+    // over warps decides where it writes and how many of the ties it takes
+    unsigned ngt = 0, neq = 0;
+    for (int j = lane; j < n; j += 32) {
+        const uint32_t u = src.key(wid, j);
+        ngt += u > T;
+        neq += u == T;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ngt += __shfl_xor_sync(0xffffffffu, ngt, o);
+        neq += __shfl_xor_sync(0xffffffffu, neq, o);
+    }
+    const unsigned gt_before = mid_warp_prefix(sh.wgt, sh.wpre, ngt);
+    const unsigned eq_before = mid_warp_prefix(sh.weq, sh.wpre2, neq);
+    unsigned base = gt_before + (eq_before < need ? eq_before : need);
+    unsigned eq_seen = eq_before;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t u = j < n ? src.key(wid, j) : 0u;
+        const bool gt = j < n && u > T;
+        const bool eq = j < n && u == T;
+        const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+        const bool take = gt || (eq && eq_seen + __popc(eqb & lt) < need);
+        const unsigned tb = __ballot_sync(0xffffffffu, take);
+        const unsigned pos = base + __popc(tb & lt);
+        if (take && pos < (unsigned)k)
+            out[pos] = src.index(wid, j);
+        base += __popc(tb);
+        eq_seen += __popc(eqb);
+    }
+}
+
+__global__ void __launch_bounds__(kMidThreads, 2)
+topk_mid_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
+                const int64_t *__restrict__ q_pos, int m, int k, int32_t *__restrict__ idx)
+{
+    extern __shared__ uint8_t dyn[];
+    MidShared &sh = *reinterpret_cast<MidShared *>(dyn);
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int64_t row = blockIdx.x;
+    const int V = (int)visible(q_pos[row], m, E);
+    int32_t *out = idx + row * k;
+    if (V <= k) {
+        for (int j = tid; j < k; j += kMidThreads)
+            out[j] = j < V ? j : -1;
+        return;
+    }
+    const float *src = scores + row * ld;
+    if (tid == 0)
+        sh.fallback = 0;
+    __syncthreads();
+    // segments of the row: a multiple of 4 entries per warp
+    const int seg = ((V + kMidWarps - 1) / kMidWarps + 3) & ~3;
+    // 1. lower bound from the samples: warp w reads runs at two places
+    uint32_t L = 0;
+    if (V > 4 * k) {
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const int r = wid * 2 + h;                          // run 0..31
+            const int s0 = (int)(((int64_t)r * V) / 32);
+            const int si = s0 + lane < V ? s0 + lane : V - 1;
+            sh.skey[r * 32 + lane] = float_key(__ldg(src + si));
+        }
+        const float mu = (float)k * 1024.f / (float)V;
+        unsigned ks = (unsigned)(1.25f * mu + 4.f * sqrtf(mu) + 8.f);
+        ks = ks > 1024u ? 1024u : ks;
+        uint32_t pre = 0, msk = 0;
+        unsigned nd = ks;
+#pragma unroll 1
+        for (int shift = 24; shift >= 16; shift -= 8) {
+            if (tid < 256)
+                sh.hist[tid] = 0;
+            __syncthreads();
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const uint32_t u = sh.skey[tid * 2 + h];
+                hist_add(sh.hist, (u >> shift) & 255u, (u & msk) == pre);
+            }
+            __syncthreads();
+            mid_find(sh, nd);
+            pre |= sh.bin << shift;
+            msk |= 255u << shift;
+            nd = sh.need;
+            __syncthreads();
+        }
+        L = pre;
+    }
+    // 2. candidates: warp w's segment, 128 entries per step (4 per lane),
+    // kept in index order in the warp's region; the loads of four steps are
+    // issued before any of them is used
+    {
+        const int a0 = wid * seg, a1 = a0 + seg < V ? a0 + seg : V;
+        const bool vec = (((uintptr_t)(src + a0)) & 15u) == 0;
+        unsigned cnt = 0;
+        bool over = false;
+        for (int b0 = a0; b0 < a1; b0 += 4 * 128) {
+            uint32_t u[4][4];
+#pragma unroll
+            for (int st = 0; st < 4; st++) {
+                const int p = b0 + st * 128 + 4 * lane;
+                if (vec && p + 3 < a1) {
+                    const float4 f = __ldg((const float4 *)(src + p));
+                    u[st][0] = float_key(f.x);
+                    u[st][1] = float_key(f.y);
+                    u[st][2] = float_key(f.z);
+                    u[st][3] = float_key(f.w);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; j++)
+                        u[st][j] = p + j < a1 ? float_key(__ldg(src + p + j)) : 0u;
+                }
+            }
+#pragma unroll
+            for (int st = 0; st < 4; st++) {
+                const int p = b0 + st * 128 + 4 * lane;
+                unsigned c = 0;
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    c += (p + j < a1 && u[st][j] >= L) ? 1u : 0u;
+                unsigned incl = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o)
+                        incl += y;
+                }
+                unsigned pos = cnt + incl - c;
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    if (p + j < a1 && u[st][j] >= L) {
+                        if (pos < (unsigned)kMidCapW) {
+                            sh.ckey[wid][pos] = u[st][j];
+                            sh.cidx[wid][pos] = (uint16_t)(p + j);
+                        }
+                        ++pos;
+                    }
+                }
+                cnt += __shfl_sync(0xffffffffu, incl, 31);
+            }
+        }
+        over = cnt > (unsigned)kMidCapW;
+        if (lane == 0) {
+            sh.wcnt[wid] = over ? 0u : cnt;
+            if (over)
+                sh.fallback = 1;
+        }
+    }
+    if (tid == 0)
+        sh.total = 0;
+    __syncthreads();
+    if (tid < 32) {
+        unsigned t = tid < kMidWarps ? sh.wcnt[tid] : 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (tid == 0)
+            sh.total = t;
+    }
+    __syncthreads();
+    const bool fb = sh.fallback || sh.total < (unsigned)k;
+    __syncthreads();
+    MidSrc<MidShared> ms{src, &sh, seg, V, !fb};
+    mid_select(ms, k, out, sh);
 }
 
 // ---------------------------------------------------------------------------
@@ -693,6 +1019,13 @@ cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s)
                              kResident * (int)sizeof(uint32_t));
         topk_final_kernel<<<(unsigned)a.rows, kThreads, kResident * sizeof(uint32_t), s>>>(
             a.q_pos, a.E, a.m, a.k, nchunks, w, a.idx);
+        return cudaGetLastError();
+    }
+    if (a.k <= kMidMaxK) {
+        cudaFuncSetAttribute(topk_mid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(MidShared));
+        topk_mid_kernel<<<(unsigned)a.rows, kMidThreads, sizeof(MidShared), s>>>(
+            a.scores, a.E, a.ld, a.q_pos, a.m, a.k, a.idx);
         return cudaGetLastError();
     }
     const int resident = a.E > a.k;

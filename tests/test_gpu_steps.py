@@ -203,6 +203,26 @@ def test_topk_block_rows_streamed_and_ties():
     np.testing.assert_array_equal(idx.cpu().numpy(), ref)
 
 
+def test_topk_mid_rows_clustered_sorted_and_sparse():
+    # rows of 2K..64K entries take a sampled lower bound and per-warp candidate
+    # regions; rows whose top entries crowd one part of the row (sorted rows,
+    # one hot cluster) overflow a region and are selected from the row itself
+    rows, E, k = 6, 40000, 1024
+    rng = np.random.default_rng(27)
+    sc = rng.standard_normal((rows, E)).astype(np.float32)
+    sc[0] = np.arange(E, dtype=np.float32)                 # ascending: top-k at the end
+    sc[1] = -np.arange(E, dtype=np.float32)                # descending: top-k at the start
+    sc[2, 20000:22000] += 50.0                             # one hot cluster of 2000
+    sc[3] = np.where(rng.random(E) < 0.03, 10.0, -10.0)    # 3 % hot entries, all tied
+    sc[4, ::7] = 3.0                                       # a tied grid near the bound
+    q_pos = torch.tensor([E - 1, E - 1, E - 1, E - 1, E - 1, 30000], dtype=torch.int64)
+    idx = torch.empty(rows, k, device=DEV, dtype=torch.int32)
+    abi.csa_topk(torch.as_tensor(sc).to(DEV), q_pos.to(DEV), 1, k, idx, E)
+    abi.csa_get_error()
+    ref = oracle.topk(sc.astype(np.float64), q_pos.numpy(), 1, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+
+
 def test_topk_long_rows_split_over_blocks():
     # rows past 65536 entries go through the four-launch chunked path with a
     # caller workspace: candidates of the threshold bin across chunk borders,
