@@ -367,6 +367,70 @@ def workload_summary(w, p, step_ms, kavg, use_graph, pk, steps):
     return out
 
 
+def time_norm_rope(p, w, pk, stream, steps=5):
+    """Device time of the RMSNorm + partial RoPE calls on a CSA step's own
+    tensors (entries and window rows; queries; the output turned back), each
+    read and written once: bytes = 2 x the tensor's bytes."""
+    from long_context_sparse_07_b200 import abi
+    kwin = torch.empty_like(p.d["Ca"])
+    calls = {
+        "rope_entries": (lambda: abi.csa_norm_rope(p.entries.body, 64, pos=None, pos_mul=w.m,
+                                                   pos_add=w.m - 1), p.entries.body),
+        "rope_window": (lambda: abi.csa_norm_rope(kwin, 64, pos=None), kwin),
+        "rope_q": (lambda: abi.csa_norm_rope(p.d["q"], 64, pos=p.q_pos), p.d["q"]),
+        "rotate_back": (lambda: abi.csa_norm_rope(p.out[0], 64, pos=p.q_pos, pos_mul=-1,
+                                                  normalise=False), p.out),
+    }
+    res = {}
+    for name, (f, t) in calls.items():
+        f()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            f()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+        by = 2 * t.numel() * t.element_size()
+        res[name] = {"ms": ms, "bytes": by, "achieved": by / (ms * 1e-3) / 1e9,
+                     "peak": pk["hbm"], "unit": "GB/s", "frac": by / (ms * 1e-3) / 1e9 / pk["hbm"]}
+    abi.csa_get_error()
+    del kwin
+    return res
+
+
+def time_out_proj(p, w, pk, stream, steps=3, g=8, dg=1024, d=4096):
+    """Device time of the grouped output projection (g groups of d_g, then
+    d; the Flash configuration) on the step's own attention output; random
+    N(0, 0.02^2) weights. Work: 2 n (h c d_g + g d_g d) FLOPs."""
+    from long_context_sparse_07_b200 import abi
+    n = w.n
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    Wg = (torch.randn(g * dg, w.h * w.c // g, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
+    Wo = (torch.randn(d, g * dg, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
+    u = torch.empty(n, g * dg, device="cuda", dtype=torch.bfloat16)
+    out = torch.empty(n, d, device="cuda", dtype=torch.bfloat16)
+    o = p.out[0]
+    abi.csa_grouped_out_proj(o, Wg, Wo, g, u, out)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        abi.csa_grouped_out_proj(o, Wg, Wo, g, u, out)
+    b.record(stream)
+    torch.cuda.synchronize()
+    abi.csa_get_error()
+    ms = a.elapsed_time(b) / steps
+    fl = 2.0 * n * (w.h * w.c * dg + g * dg * d)
+    del Wg, Wo, u, out
+    return {"ms": ms, "flops": fl, "achieved": fl / (ms * 1e-3) / 1e12, "peak": pk["bf16"],
+            "unit": "TFLOP/s", "frac": fl / (ms * 1e-3) / 1e12 / pk["bf16"],
+            "shape": {"n": n, "h": w.h, "c": w.c, "g": g, "dg": dg, "d": d}}
+
+
 # --------------------------------------------------------------------------- CPU oracle
 
 
@@ -544,6 +608,14 @@ def run_ours(args, w):
     e_ms, h2d, d2h = time_e2e(p, e2e_steps, stream)
     e2e_value, _ = job_rate(sum(e_ms) / len(e_ms), units_per_step(w), world, dist, "cuda")
 
+    # the Module D normalisation and partial RoPE (outside the configs' step):
+    # timed on this workload's own buffers, after the step measurements
+    extras = {}
+    if w.kind == "csa" and w.c >= 64 and not args.no_per_workload:
+        extras["norm_rope"] = time_norm_rope(p, w, pk, stream)
+        if w.dtype == "bf16" and w.h % 8 == 0:
+            extras["grouped_out_proj"] = time_out_proj(p, w, pk, stream)
+
     dom = summ["dominant"]
     roof = dict(summ["kernels"][dom])
     roof.pop("ideal_ms", None)
@@ -592,6 +664,8 @@ def run_ours(args, w):
         }
         if per:
             line["per_workload"] = per
+        if extras:
+            line["extras"] = extras
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, host_ops)
         print(json.dumps(line), flush=True)

@@ -246,6 +246,54 @@ csa_status csa_sparse_mqa_noalloc(const void *q, csa_dtype q_dt, csa_entries kv,
 size_t csa_noalloc_scratch_bytes(void);
 
 /*
+ * csa_norm_rope -- Q/KV RMSNorm and partial RoPE before the core attention,
+ * and the rotation of its output back by the query position (Module D: "Q/KV
+ * normalisation", "partial RoPE": RoPE only on the last 64 dims of queries
+ * and KV entries; since an entry is key and value, the output o_t then
+ * carries the entries' absolute positions, and turning its last 64 dims by
+ * the position -t leaves relative positions). In place on x, [rows, heads, c]
+ * of dt (F32 or BF16), per head vector:
+ *   when normalise: x <- x / sqrt(mean_j x_j^2 + eps) * gamma[j]
+ *                   (gamma [c] float32, or NULL for a gain of 1);
+ *   then the last rope_dims dims turn in adjacent pairs (c - R + 2p,
+ *   c - R + 2p + 1), p < R / 2, by phi_p = P * base^(-2p / R):
+ *   (a, b) <- (a cos phi - b sin phi, a sin phi + b cos phi), with the
+ *   position P = pos_mul * (pos ? pos[row] : row) + pos_add (pos [rows]
+ *   int64 or NULL). Queries: pos = q_pos, pos_mul = 1; compressed entry i:
+ *   pos = NULL, pos_mul = m, pos_add = m - 1 (the position of its last
+ *   token); window rows: pos = NULL, pos_mul = 1, pos_add = the position of
+ *   row 0; the attention output: pos = q_pos, pos_mul = -1, normalise = 0.
+ *   The method's pages fix neither the pairing, the base, the entry
+ *   positions nor eps; these are this library's readings.
+ * Requirements: c in {64, 128, 256, 512, 1024}; rope_dims even, <= c;
+ *   eps > 0 when normalising; base > 1 when rope_dims > 0; x 16-byte aligned.
+ */
+csa_status csa_norm_rope(void *x, csa_dtype dt, const float *gamma, int64_t rows, int heads, int c,
+                         int rope_dims, const int64_t *pos, int64_t pos_mul, int64_t pos_add,
+                         int normalise, float eps, float base, void *stream);
+
+/*
+ * csa_grouped_out_proj -- grouped output projection (Module B step 4: the
+ * n_h head outputs are cut into g groups, each group is projected to an
+ * intermediate d_g, and the concatenation is projected to d), bf16 operands
+ * with float32 accumulation:
+ *   u[t, j d_g + e] = sum_x o[t, j K_g + x] * Wg[j d_g + e, x]   (j < g,
+ *                     K_g = h c / g; group j holds heads j h/g .. (j+1) h/g - 1)
+ *   out[t, f]       = sum_y u[t, y] * Wo[f, y]
+ * Arguments (all bf16, row-major, 16-byte aligned, owned by the caller):
+ *   o   [n, h, c]      attention outputs;
+ *   Wg  [g * dg, K_g]  the g group weights, output features by input features;
+ *   Wo  [d, g * dg]    the final weight;
+ *   u   [n, g * dg]    written: the grouped projections, stored as bf16;
+ *   out [n, d]         written.
+ * Requirements: g divides h; K_g a multiple of 64; dg and d multiples of
+ *   256. The pages fix g = 8, d_g = 1024 (Flash) but no weight layout or
+ *   intermediate precision; the layout above and bf16 u are this library's.
+ */
+csa_status csa_grouped_out_proj(const void *o, const void *Wg, const void *Wo, int64_t n, int h,
+                                int c, int g, int dg, int d, void *u, void *out, void *stream);
+
+/*
  * csa_debug_wait_probe -- checks the device-side failure path. Launches one
  * thread that waits, through the same bounded mbarrier wait every pipeline
  * kernel uses, on a barrier that nothing completes; after limit_ns

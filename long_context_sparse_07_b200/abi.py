@@ -28,7 +28,8 @@ STATUS = {0: "CSA_OK", -1: "CSA_ERR_INVALID_ARG", -2: "CSA_ERR_UNSUPPORTED",
 EXPORTS = ("csa_abi_version", "csa_status_string", "csa_last_message", "csa_compress_kv",
            "csa_indexer_scores", "csa_topk", "csa_topk_workspace_size", "csa_sparse_mqa",
            "hca_dense_mqa", "csa_mqa_workspace_size", "csa_sparse_mqa_noalloc",
-           "csa_noalloc_scratch_bytes", "csa_debug_wait_probe", "csa_get_error")
+           "csa_noalloc_scratch_bytes", "csa_norm_rope", "csa_grouped_out_proj",
+           "csa_debug_wait_probe", "csa_get_error")
 
 
 class CsaError(RuntimeError):
@@ -85,6 +86,10 @@ def load(path: str = LIB_PATH):
                                          _P, _I, _I64, _I, _F, _P, _P, _P]
     L.csa_noalloc_scratch_bytes.restype = _S
     L.csa_noalloc_scratch_bytes.argtypes = []
+    L.csa_norm_rope.restype = _I
+    L.csa_norm_rope.argtypes = [_P, _I, _P, _I64, _I, _I, _I, _P, _I64, _I64, _I, _F, _F, _P]
+    L.csa_grouped_out_proj.restype = _I
+    L.csa_grouped_out_proj.argtypes = [_P, _P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P]
     L.csa_debug_wait_probe.restype = _I
     L.csa_debug_wait_probe.argtypes = [ctypes.c_uint64, _P]
     L.csa_get_error.restype = _I
@@ -213,6 +218,26 @@ def hca_dense_mqa(q, kv: Entries, E: int, m: int, kwin, win_pos0, n_win: int, q_
                                 win_rows, _ptr(win_pos0), n_win, _ptr(q_pos), _ptr(sink), B,
                                 n_q, h, scale, _ptr(out), _ptr(lse), _ptr(workspace), ws,
                                 _stream(stream)))
+
+
+def csa_norm_rope(x, rope_dims: int, pos=None, pos_mul: int = 1, pos_add: int = 0, gamma=None,
+                  normalise: bool = True, eps: float = 1e-6, base: float = 10000.0, stream=None):
+    """In-place RMSNorm and partial RoPE of x [rows, heads, c] or [rows, c]."""
+    c = x.shape[-1]
+    rows = x.shape[0]
+    heads = x.numel() // (rows * c) if rows else 1
+    _check(load().csa_norm_rope(_ptr(x), dtype_code(x), _ptr(gamma), rows, heads, c, rope_dims,
+                                _ptr(pos), pos_mul, pos_add, int(bool(normalise)), eps, base,
+                                _stream(stream)))
+
+
+def csa_grouped_out_proj(o, Wg, Wo, g: int, u, out, stream=None):
+    """Grouped output projection: o [n, h, c] -> u [n, g dg] -> out [n, d]."""
+    n, h, c = o.shape
+    dg = Wg.shape[0] // g
+    d = Wo.shape[0]
+    _check(load().csa_grouped_out_proj(_ptr(o), _ptr(Wg), _ptr(Wo), n, h, c, g, dg, d, _ptr(u),
+                                       _ptr(out), _stream(stream)))
 
 
 def csa_debug_wait_probe(limit_ns: int, stream=None):

@@ -301,6 +301,57 @@ csa_status hca_dense_mqa(const void *q, csa_dtype q_dt, csa_entries kv, int64_t 
                          ws_bytes, stream);
 }
 
+csa_status csa_norm_rope(void *x, csa_dtype dt, const float *gamma, int64_t rows, int heads, int c,
+                         int rope_dims, const int64_t *pos, int64_t pos_mul, int64_t pos_add,
+                         int normalise, float eps, float base, void *stream)
+{
+    const char *w = "csa_norm_rope";
+    REQUIRE(x, CSA_ERR_INVALID_ARG, "%s: x is NULL", w);
+    REQUIRE(dt == CSA_F32 || dt == CSA_BF16, CSA_ERR_UNSUPPORTED, "%s: dtype must be F32 or BF16",
+            w);
+    REQUIRE(rows >= 0 && heads >= 1, CSA_ERR_INVALID_ARG, "%s: bad rows / heads", w);
+    REQUIRE(c == 64 || c == 128 || c == 256 || c == 512 || c == 1024, CSA_ERR_UNSUPPORTED,
+            "%s: c = %d unsupported (64 .. 1024, a power of two)", w, c);
+    REQUIRE(rope_dims >= 0 && rope_dims <= c && rope_dims % 2 == 0, CSA_ERR_INVALID_ARG,
+            "%s: rope_dims = %d must be even and at most c", w, rope_dims);
+    REQUIRE(!normalise || eps > 0.f, CSA_ERR_INVALID_ARG, "%s: eps must be positive", w);
+    REQUIRE(rope_dims == 0 || base > 1.f, CSA_ERR_INVALID_ARG, "%s: base must exceed 1", w);
+    REQUIRE(aligned16(x), CSA_ERR_INVALID_ARG, "%s: x must be 16-byte aligned", w);
+    csa::NormRopeArgs a{x, dt, gamma, rows, heads, c, rope_dims, pos, pos_mul, pos_add,
+                        normalise ? 1 : 0, eps, base};
+    return launched(csa::launch_norm_rope(a, (cudaStream_t)stream), w);
+}
+
+csa_status csa_grouped_out_proj(const void *o, const void *Wg, const void *Wo, int64_t n, int h,
+                                int c, int g, int dg, int d, void *u, void *out, void *stream)
+{
+    const char *w = "csa_grouped_out_proj";
+    REQUIRE(o && Wg && Wo && u && out, CSA_ERR_INVALID_ARG, "%s: every buffer is required", w);
+    REQUIRE(n >= 0 && n <= INT32_MAX && h >= 1 && c >= 1 && g >= 1 && h % g == 0,
+            CSA_ERR_INVALID_ARG, "%s: bad n / h / c / g (g must divide h)", w);
+    const int64_t Kg = (int64_t)h * c / g;
+    REQUIRE(Kg % 64 == 0 && Kg <= INT32_MAX, CSA_ERR_UNSUPPORTED,
+            "%s: h c / g = %lld must be a multiple of 64", w, (long long)Kg);
+    REQUIRE(dg >= 256 && dg % 256 == 0 && d >= 256 && d % 256 == 0, CSA_ERR_UNSUPPORTED,
+            "%s: d_g and d must be multiples of 256", w);
+    REQUIRE((int64_t)g * dg % 64 == 0, CSA_ERR_UNSUPPORTED, "%s: g d_g must be a multiple of 64",
+            w);
+    REQUIRE(aligned16(o) && aligned16(Wg) && aligned16(Wo) && aligned16(u) && aligned16(out),
+            CSA_ERR_INVALID_ARG, "%s: buffers must be 16-byte aligned", w);
+    unsigned *err = err_word();
+    REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
+    if (n == 0)
+        return CSA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    csa::GemmArgs a1{o, Wg, u, n, dg, (int)Kg, g, (int64_t)h * c, (int64_t)g * dg,
+                     (int64_t)g * dg, Kg, dg, dg};
+    cudaError_t e = csa::launch_gemm_nt(a1, err, s);
+    if (e != cudaSuccess)
+        return launched(e, w);
+    csa::GemmArgs a2{u, Wo, out, n, d, g * dg, 1, (int64_t)g * dg, d, d, 0, 0, 0};
+    return launched(csa::launch_gemm_nt(a2, err, s), w);
+}
+
 csa_status csa_debug_wait_probe(uint64_t limit_ns, void *stream)
 {
     const char *w = "csa_debug_wait_probe";

@@ -14,7 +14,7 @@ namespace csa {
 // [1] = kernel id, [2], [3] = kernel-specific detail (row, index).
 enum KernelId : unsigned {
     K_COMPRESS = 1, K_INDEXER = 2, K_TOPK = 3, K_ATTEND = 4, K_ATTEND_TC = 5,
-    K_INDEXER_TC = 6, K_COMBINE = 7, K_PROBE = 8
+    K_INDEXER_TC = 6, K_COMBINE = 7, K_PROBE = 8, K_GEMM = 9
 };
 
 __device__ __forceinline__ void report(unsigned *err, csa_status code, unsigned kernel,

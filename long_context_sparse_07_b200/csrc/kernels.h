@@ -75,6 +75,32 @@ csa_status check_attend(const char *what, const void *q, csa_dtype q_dt, const c
                         int64_t win_rows, int n_win, const int64_t *q_pos, const float *sink,
                         int B, int64_t n_q, int h, void *out);
 
+struct NormRopeArgs {
+    void *x;
+    csa_dtype dt;
+    const float *gamma;
+    int64_t rows;
+    int heads, c, rope_dims;
+    const int64_t *pos;
+    int64_t pos_mul, pos_add;
+    int normalise;
+    float eps, base;
+};
+cudaError_t launch_norm_rope(const NormRopeArgs &a, cudaStream_t s);
+
+// C[M, N] (+ group offsets) = A[M, K] . B[N, K]^T, bf16, for `groups`
+// independent groups: group j reads A columns j * a_col_off .., B rows
+// j * b_row_off .., writes C columns j * c_col_off ..
+struct GemmArgs {
+    const void *A, *B;
+    void *C;
+    int64_t M;
+    int N, K, groups;
+    int64_t lda, b_rows, ldc;
+    int64_t a_col_off, b_row_off, c_col_off;
+};
+cudaError_t launch_gemm_nt(const GemmArgs &g, unsigned *err, cudaStream_t s);
+
 // One bounded wait that nothing completes (csa_debug_wait_probe).
 cudaError_t launch_wait_probe(uint64_t limit_ns, unsigned *err, cudaStream_t s);
 

@@ -37,13 +37,19 @@ class CsaPrefill:
 
     @property
     def launches_per_step(self):
-        """Kernels launched by one step (top-k of long rows takes four)."""
-        return 4 + (4 if self.topk_ws is not None else 1)
+        """Kernels launched by one step (top-k of long rows takes four; the
+        normalisation and RoPE add four)."""
+        return 4 + (4 if self.topk_ws is not None else 1) + (4 if self.rope_dims else 0)
 
-    def __init__(self, w, ops: Dict[str, torch.Tensor], device="cuda"):
+    def __init__(self, w, ops: Dict[str, torch.Tensor], device="cuda", rope_dims: int = 0):
         self.w = w
         d = self.d = _dev(ops, device)
         n, c, E = w.n, w.c, w.E
+        # with rope_dims > 0 the step also applies Module D's RMSNorm and
+        # partial RoPE to the entries, the window rows (a copy of C^a) and the
+        # queries, and turns the output back by the query position
+        self.rope_dims = rope_dims
+        self.kwin = torch.empty_like(d["Ca"]) if rope_dims else d["Ca"]
         self.q_pos = torch.arange(n, device=device, dtype=torch.int64)
         self.win_pos0 = torch.zeros(1, device=device, dtype=torch.int64)
         self.entries = Entries(torch.empty(E, c, device=device, dtype=DT[w.dtype]), c)
@@ -85,14 +91,34 @@ class CsaPrefill:
 
     def attend(self, stream=None):
         d, w = self.d, self.w
-        abi.csa_sparse_mqa(d["q"][None], self.entries, w.E, w.m, self.idx, w.k, d["Ca"][None],
+        abi.csa_sparse_mqa(d["q"][None], self.entries, w.E, w.m, self.idx, w.k, self.kwin[None],
                            self.win_pos0, w.n_win, self.q_pos[None], d["sink"], self.scale,
                            self.out, self.lse, stream=stream)
 
+    def rope_kv(self, stream=None):
+        """RMSNorm + RoPE of the entries (at their blocks' last tokens) and of
+        the window rows (a copy of C^a, at their own positions)."""
+        w = self.w
+        abi.csa_norm_rope(self.entries.body, self.rope_dims, pos=None, pos_mul=w.m,
+                          pos_add=w.m - 1, stream=stream)
+        self.kwin.copy_(self.d["Ca"])
+        abi.csa_norm_rope(self.kwin, self.rope_dims, pos=None, stream=stream)
+
+    def rope_q(self, stream=None):
+        abi.csa_norm_rope(self.d["q"], self.rope_dims, pos=self.q_pos, stream=stream)
+
+    def rotate_back(self, stream=None):
+        abi.csa_norm_rope(self.out[0], self.rope_dims, pos=self.q_pos, pos_mul=-1,
+                          normalise=False, stream=stream)
+
     def phases(self):
         """The kernels of one step, in order: (name, launch)."""
-        return [("compress_kv", self.compress_kv), ("compress_index", self.compress_index),
-                ("indexer", self.index), ("topk", self.select), ("attend", self.attend)]
+        ph = [("compress_kv", self.compress_kv), ("compress_index", self.compress_index),
+              ("indexer", self.index), ("topk", self.select), ("attend", self.attend)]
+        if self.rope_dims:
+            ph = ph[:1] + [("rope_kv", self.rope_kv)] + ph[1:4] + [("rope_q", self.rope_q)] + \
+                ph[4:] + [("rotate_back", self.rotate_back)]
+        return ph
 
     def inputs(self):
         """Device operands a step reads (copied from the host in end-to-end runs)."""

@@ -63,6 +63,8 @@ def lib():
             L.oracle_compress.argtypes = [_d, _d, _d, _d, _d, _d, _I64, _I, _I, _I, _d]
             L.oracle_indexer.argtypes = [_d, _d, _d, _i64, _I, _I64, _I64, _I, _I, _I, _d]
             L.oracle_topk.argtypes = [_d, _I64, _I64, _I64, _i64, _I, _I, _i32]
+            L.oracle_norm_rope.argtypes = [_d, _I64, _I, _I, _I, _i64, _d, _I, ctypes.c_double,
+                                           ctypes.c_double]
             L.oracle_attend.restype = _I
             L.oracle_attend.argtypes = [_d, _d, _I64, _i32, _I, _I, _d, _I64, _i64, _I,
                                         _i64, _d, _I, _I64, _I, _I, ctypes.c_double, _d, _d]
@@ -194,3 +196,21 @@ def attend(q, entries, idx, k: int, m: int, kwin, win_pos0, n_win: int, q_pos, s
     if rc != 0:
         raise ValueError("oracle_attend: selection index or window position out of range")
     return out, lse
+
+
+def norm_rope(x, pos, rope_dims: int, gamma=None, normalise: bool = True, eps: float = 1e-6,
+              base: float = 10000.0) -> np.ndarray:
+    """RMSNorm of each head vector (x [rows, heads, c] or [rows, c]) and RoPE
+    on its last rope_dims dims at position pos[row] (Module D); float64 copy."""
+    a = np.array(f64(x), dtype=np.float64, copy=True)
+    shp = a.shape
+    if a.ndim == 2:
+        a = a[:, None, :]
+    rows, heads, c = a.shape
+    a = np.ascontiguousarray(a)
+    p = np.ascontiguousarray(np.asarray(pos, dtype=np.int64).reshape(rows))
+    g = None if gamma is None else np.ascontiguousarray(f64(gamma).reshape(c))
+    lib().oracle_norm_rope(_p(a, _d), rows, heads, c, int(rope_dims), _p(p, _i64),
+                           _p(g, _d) if g is not None else None, int(bool(normalise)),
+                           float(eps), float(base))
+    return a.reshape(shp)

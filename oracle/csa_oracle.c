@@ -327,3 +327,40 @@ int oracle_attend(const double *q, const double *entries, int64_t E,
     }
     return bad ? -1 : 0;
 }
+
+/* RMSNorm of one head vector, then partial RoPE on its last R dims (Module D:
+ * "Q/KV normalisation" and "partial RoPE"). In place on rows x heads vectors
+ * of c values:
+ *   x <- x / sqrt(mean_j x_j^2 + eps) * gamma          (gamma [c], or NULL: 1)
+ *   for pair p = 0 .. R/2-1 of the last R dims, at position pos[row]:
+ *     phi = pos * base^(-2p/R),
+ *     (a, b) <- (a cos phi - b sin phi, a sin phi + b cos phi)
+ * Readings (the pages are silent): the RoFormer pairing of adjacent dims
+ * (c-R+2p, c-R+2p+1); frequencies base^(-2p/R) over the rotated dims only;
+ * normalise = 0 skips the RMSNorm (rotation alone). */
+void oracle_norm_rope(double *x, int64_t rows, int heads, int c, int R, const int64_t *pos,
+                      const double *gamma, int normalise, double eps, double base)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        for (int h = 0; h < heads; h++) {
+            double *v = x + (r * heads + h) * (int64_t)c;
+            if (normalise) {
+                double ss = 0.0;
+                for (int j = 0; j < c; j++)
+                    ss += v[j] * v[j];
+                const double inv = 1.0 / sqrt(ss / c + eps);
+                for (int j = 0; j < c; j++)
+                    v[j] = v[j] * inv * (gamma ? gamma[j] : 1.0);
+            }
+            for (int p = 0; p < R / 2; p++) {
+                const double phi = (double)pos[r] * pow(base, -2.0 * p / R);
+                const double cs = cos(phi), sn = sin(phi);
+                double *a = v + (c - R) + 2 * p;
+                const double a0 = a[0], a1 = a[1];
+                a[0] = a0 * cs - a1 * sn;
+                a[1] = a0 * sn + a1 * cs;
+            }
+        }
+    }
+}

@@ -25,7 +25,7 @@ from typing import Dict, Optional, Sequence
 import numpy as np
 import torch
 
-from . import attend, compress, dequantize, f64, indexer, quantize_e4m3, topk
+from . import attend, compress, dequantize, f64, indexer, norm_rope, quantize_e4m3, topk
 
 
 def store(x: np.ndarray, dtype: str) -> np.ndarray:
@@ -114,3 +114,30 @@ def decode(ops: Dict[str, torch.Tensor], w) -> dict:
                         w.n_win, pos, ops["sink"], scale)
     return {"scores": sc32, "idx": sel, "out": out, "lse": lse, "hca_out": hout,
             "hca_lse": hlse}
+
+
+def csa_prefill_rope(ops: Dict[str, torch.Tensor], w, rows: Optional[Sequence[int]] = None,
+                     rope_dims: int = 64, gamma_q=None, gamma_kv=None, eps: float = 1e-6,
+                     base: float = 10000.0, shift: int = 0) -> dict:
+    """CSA prefill with the Q/KV RMSNorm and partial RoPE of Module D before
+    the core attention, and its output rotated back by the query position:
+    queries at their positions t, compressed entry i at the position of its
+    last token m i + m - 1, window rows at their own positions; every
+    normalised and rotated tensor is stored in the path's dtype. ``shift``
+    adds a constant to every RoPE position (a test of relative positions)."""
+    n = w.n
+    rows = np.arange(n) if rows is None else np.asarray(rows, dtype=np.int64)
+    base_res = csa_prefill(ops, w, rows)                 # compression, indexer, top-k
+    E = base_res["entries"].shape[0]
+    ent = store(norm_rope(base_res["entries"], np.arange(E) * w.m + w.m - 1 + shift,
+                          rope_dims, gamma_kv, True, eps, base), w.dtype)
+    win = store(norm_rope(f64(ops["Ca"]), np.arange(n) + shift, rope_dims, gamma_kv, True,
+                          eps, base), w.dtype)
+    q = store(norm_rope(f64(ops["q"][rows]), rows + shift, rope_dims, gamma_q, True, eps,
+                        base).reshape(len(rows), w.h, w.c), w.dtype)
+    pos = rows.reshape(1, -1)
+    out, lse = attend(q[None], ent[None], base_res["idx"], w.k, w.m, win[None], [0], w.n_win,
+                      pos, ops["sink"], 1.0 / math.sqrt(w.c))
+    o = norm_rope(out[0], -(rows + shift), rope_dims, None, False, eps, base)
+    return {"entries": ent, "idx": base_res["idx"], "out": o, "lse": lse[0], "rows": rows,
+            "q": q, "win": win}
