@@ -2,7 +2,8 @@
 """Throughput of the CSA / HCA hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--no-per-workload] [--no-cpu-baseline]
+                    [--impl ours|reference] [--no-per-workload] [--no-extras]
+                    [--no-cpu-baseline] [--n N] [--graph auto|on|off]
 
 One step = one pass of the whole path over one synthetic sequence (CSA:
 compress KV, compress indexer keys, indexer scores, top-k, sparse attention;
@@ -611,7 +612,7 @@ def run_ours(args, w):
     # the Module D normalisation and partial RoPE (outside the configs' step):
     # timed on this workload's own buffers, after the step measurements
     extras = {}
-    if w.kind == "csa" and w.c >= 64 and not args.no_per_workload:
+    if w.kind == "csa" and w.c >= 64 and not args.no_extras:
         extras["norm_rope"] = time_norm_rope(p, w, pk, stream)
         if w.dtype == "bf16" and w.h % 8 == 0:
             extras["grouped_out_proj"] = time_out_proj(p, w, pk, stream)
@@ -721,6 +722,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="time only the selected workload")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the RMSNorm/RoPE and grouped-projection timings")
     ap.add_argument("--n", type=int, default=None,
                     help="run the workload on a shorter sequence of n tokens (small profiling cases)")
     ap.add_argument("--graph", default="auto", choices=["auto", "on", "off"],
