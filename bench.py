@@ -228,7 +228,12 @@ def kernel_roofline(w, name, a, ms, pk):
 # (summarised under profiles/), keyed by workload and kernel; each entry holds the
 # SHA-1 of the kernel source it was taken on and the number of launches it covers
 # scaled to a full launch, and counts only while that source is unchanged.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    # attention at n = 16384 (1.16 GB read + 1.04 GB write, q / out dominated),
+    # scaled by 131072 / 16384 = 8 queries per captured query
+    ("csa_fp8idx_n131072", "attend"): ("attend_tc.cu", "99901d1152b0dc2bdd984b72efca53cb4622615e",
+                                       8 * (1.163732e9 + 1.040877e9)),
+}
 
 
 def measured_traffic(workload, kernel):
