@@ -179,7 +179,7 @@ def build_path(w, rank, keep_ops=False):
     wr = rank_workload(w, rank)
     if w.kind == "csa":
         ops = W.csa_operands(wr)
-        p = path.CsaPrefill(wr, ops)
+        p = path.CsaPrefill(wr, ops, fused=True)
     elif w.kind == "hca":
         ops = W.hca_operands(wr)
         p = path.HcaPrefill(wr, ops)
@@ -206,7 +206,7 @@ def kernel_roofline(w, name, a, ms, pk):
         # CUDA-core float32 path of the parity-sized workload: no tensor peak
         # applies; report against HBM only
         tensor_peak, pdt = None, None
-    elif name == "indexer" and w.idx_dtype == "e4m3":
+    elif name in ("indexer", "indexer_topk") and w.idx_dtype == "e4m3":
         tensor_peak, pdt = pk["fp8"], "e4m3"
     else:
         tensor_peak, pdt = pk["bf16"], "bf16"

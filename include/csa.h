@@ -162,6 +162,46 @@ csa_status csa_topk(const float *scores, int64_t rows, int64_t E, int64_t ld,
 size_t csa_topk_workspace_size(int64_t rows, int64_t E, int k);
 
 /*
+ * csa_indexer_topk -- the indexer scores (Eq. 16) and the top-k selection
+ * (Eq. 17) of Module B step 2 in one call: idx gets exactly what
+ * csa_indexer_scores followed by csa_topk would write (the same entries, in
+ * ascending order, ties to the lower index, -1 padding), but the full score
+ * rows are not written when the rows are much longer than k. For e4m3 or
+ * bf16 indexers that the tensor-core kernel takes (hI in {16, 32, 64}, cI
+ * bytes 128 or 256), E >= 16 k, E a multiple of the sample spacing (32,
+ * doubled until a row has at most 1024 samples) and enough queries that
+ * every indexer block owns whole rows (prefill), the call
+ *   1. scores every query against that sample of the keys,
+ *   2. runs the indexer keeping, per query, only the scores at or above a
+ *      lower bound taken from its sample scores (a rank of the sample that
+ *      the k-th largest score of the row exceeds with a wide margin),
+ *   3. selects the top-k exactly from those candidates,
+ *   4. recomputes in full the rows whose candidates cannot decide it (fewer
+ *      than k, or more than the workspace holds): rare for scores that are
+ *      not massively tied; correct in every case.
+ * Other calls (decode among them: a few rows, cheap to write and read back)
+ * run the two plain calls through the workspace.
+ * Arguments: as csa_indexer_scores (without scores / ld), plus
+ *   k         1 <= k <= 4096.
+ *   idx       [B * n_q, k] int32 output.
+ *   workspace csa_indexer_topk_workspace_size(B, n_q, E, hI, cI, k, dt)
+ *             bytes of device scratch, 256-byte aligned, owned by the caller;
+ *             nothing in it must be initialised. It holds a [B * n_q, E]
+ *             float32 area (score rows or candidate pairs) and small tables.
+ */
+csa_status csa_indexer_topk(const void *qI, const float *qI_scale, const float *wI,
+                            csa_entries kI, const int64_t *q_pos, int B, int64_t n_q, int64_t E,
+                            int hI, int cI, int m, csa_dtype dt, int k, int32_t *idx,
+                            void *workspace, size_t ws_bytes, void *stream);
+size_t csa_indexer_topk_workspace_size(int B, int64_t n_q, int64_t E, int hI, int cI, int k,
+                                       csa_dtype dt);
+/* Kernel launches csa_indexer_topk makes for these shapes (6 on the
+ * candidate path, 2 to 5 for the two plain calls) on the current device,
+ * for 16-byte aligned qI and kI; -1 for arguments out of range. */
+int csa_indexer_topk_launches(int B, int64_t n_q, int64_t E, int hI, int cI, int k,
+                              csa_dtype dt);
+
+/*
  * csa_sparse_mqa -- shared-KV multi-query attention over the selected
  * compressed entries, Eq. 18-19 (Module B step 3), joined by the sliding-window
  * branch and the attention sink (Module D). Every key is also its own value.

@@ -26,7 +26,8 @@ STATUS = {0: "CSA_OK", -1: "CSA_ERR_INVALID_ARG", -2: "CSA_ERR_UNSUPPORTED",
 
 # every symbol that include/csa.h declares
 EXPORTS = ("csa_abi_version", "csa_status_string", "csa_last_message", "csa_compress_kv",
-           "csa_indexer_scores", "csa_topk", "csa_topk_workspace_size", "csa_sparse_mqa",
+           "csa_indexer_scores", "csa_topk", "csa_topk_workspace_size", "csa_indexer_topk",
+           "csa_indexer_topk_workspace_size", "csa_indexer_topk_launches", "csa_sparse_mqa",
            "hca_dense_mqa", "csa_mqa_workspace_size", "csa_sparse_mqa_noalloc",
            "csa_noalloc_scratch_bytes", "csa_norm_rope", "csa_grouped_out_proj",
            "csa_debug_wait_probe", "csa_get_error")
@@ -73,6 +74,13 @@ def load(path: str = LIB_PATH):
     L.csa_topk.argtypes = [_P, _I64, _I64, _I64, _P, _I, _I, _P, _P, _S, _P]
     L.csa_topk_workspace_size.restype = _S
     L.csa_topk_workspace_size.argtypes = [_I64, _I64, _I]
+    L.csa_indexer_topk.restype = _I
+    L.csa_indexer_topk.argtypes = [_P, _P, _P, _Entries, _P, _I, _I64, _I64, _I, _I, _I, _I, _I,
+                                   _P, _P, _S, _P]
+    L.csa_indexer_topk_workspace_size.restype = _S
+    L.csa_indexer_topk_workspace_size.argtypes = [_I, _I64, _I64, _I, _I, _I, _I]
+    L.csa_indexer_topk_launches.restype = _I
+    L.csa_indexer_topk_launches.argtypes = [_I, _I64, _I64, _I, _I, _I, _I]
     L.csa_sparse_mqa.restype = _I
     L.csa_sparse_mqa.argtypes = [_P, _I, _Entries, _I64, _I, _P, _I, _P, _I64, _P, _I, _P, _P,
                                  _I, _I64, _I, _F, _P, _P, _P, _S, _P]
@@ -176,6 +184,29 @@ def csa_topk(scores, q_pos, m: int, k: int, idx, E: Optional[int] = None, worksp
     ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(load().csa_topk(_ptr(scores), rows, E, ld, _ptr(q_pos), m, k, _ptr(idx),
                            _ptr(workspace), ws, _stream(stream)))
+
+
+def csa_indexer_topk_workspace_size(B: int, n_q: int, E: int, hI: int, cI: int, k: int,
+                                    dt) -> int:
+    code = dt if isinstance(dt, int) else dtype_code(dt)
+    return int(load().csa_indexer_topk_workspace_size(B, n_q, E, hI, cI, k, code))
+
+
+def csa_indexer_topk_launches(B: int, n_q: int, E: int, hI: int, cI: int, k: int, dt) -> int:
+    """Kernel launches of csa_indexer_topk for these shapes (6: candidate path)."""
+    code = dt if isinstance(dt, int) else dtype_code(dt)
+    return int(load().csa_indexer_topk_launches(B, n_q, E, hI, cI, k, code))
+
+
+def csa_indexer_topk(qI, qI_scale, wI, kI: Entries, q_pos, m: int, k: int, idx, E: int,
+                     workspace=None, stream=None):
+    """Indexer scores and top-k in one call: idx [B * n_q, k] as
+    csa_indexer_scores followed by csa_topk would give."""
+    B, n_q, hI, cI = qI.shape
+    ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load().csa_indexer_topk(_ptr(qI), _ptr(qI_scale), _ptr(wI), kI.struct(), _ptr(q_pos),
+                                   B, n_q, E, hI, cI, m, dtype_code(qI), k, _ptr(idx),
+                                   _ptr(workspace), ws, _stream(stream)))
 
 
 def csa_mqa_workspace_size(B: int, n_q: int, h: int, c: int, max_keys: int) -> int:

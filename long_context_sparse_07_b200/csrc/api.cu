@@ -147,25 +147,28 @@ csa_status csa_compress_kv(const void *Ca, const void *Cb, const void *Za, const
     return launched(csa::launch_compress(a, err, (cudaStream_t)stream), w);
 }
 
-csa_status csa_indexer_scores(const void *qI, const float *qI_scale, const float *wI,
-                              csa_entries kI, const int64_t *q_pos, int B, int64_t n_q,
-                              int64_t E, int hI, int cI, int m, csa_dtype dt, float *scores,
-                              int64_t ld, void *stream)
+}  // extern "C"
+
+namespace {
+
+// Host-side checks shared by the indexer calls (scores and outputs aside).
+csa_status check_indexer(const char *w, const void *qI, const float *qI_scale, const float *wI,
+                         const csa_entries &kI, const int64_t *q_pos, int B, int64_t n_q,
+                         int64_t E, int hI, int cI, int m, csa_dtype dt)
 {
-    const char *w = "csa_indexer_scores";
-    REQUIRE(qI && wI && q_pos && scores, CSA_ERR_INVALID_ARG,
-            "%s: qI, wI, q_pos and scores are required", w);
+    REQUIRE(qI && wI && q_pos, CSA_ERR_INVALID_ARG, "%s: qI, wI and q_pos are required", w);
     REQUIRE(B >= 0 && n_q >= 0 && E >= 0 && E <= INT32_MAX, CSA_ERR_INVALID_ARG,
             "%s: bad B / n_q / E", w);
     REQUIRE(hI >= 1 && hI <= 128, CSA_ERR_UNSUPPORTED, "%s: hI = %d out of [1, 128]", w, hI);
     REQUIRE(cI >= 16 && cI <= 256 && cI % 16 == 0, CSA_ERR_UNSUPPORTED,
             "%s: cI = %d unsupported", w, cI);
     REQUIRE(m >= 1, CSA_ERR_INVALID_ARG, "%s: m must be >= 1", w);
-    REQUIRE(ld >= E, CSA_ERR_INVALID_ARG, "%s: ld < E", w);
     REQUIRE(dt == CSA_F32 || dt == CSA_BF16 || dt == CSA_E4M3, CSA_ERR_INVALID_ARG,
             "%s: unknown dtype", w);
     REQUIRE(kI.dt == dt, CSA_ERR_INVALID_ARG, "%s: kI dtype differs from qI dtype", w);
-    csa_status st = check_entries(kI, cI, true, "csa_indexer_scores(kI)");
+    char what[64];
+    snprintf(what, sizeof what, "%s(kI)", w);
+    csa_status st = check_entries(kI, cI, true, what);
     if (st != CSA_OK)
         return st;
     if (dt == CSA_E4M3) {
@@ -174,6 +177,24 @@ csa_status csa_indexer_scores(const void *qI, const float *qI_scale, const float
                 "%s: e4m3 keys need one scale per key and no rope part", w);
     }
     REQUIRE(aligned16(qI), CSA_ERR_INVALID_ARG, "%s: qI not 16-byte aligned", w);
+    return CSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+csa_status csa_indexer_scores(const void *qI, const float *qI_scale, const float *wI,
+                              csa_entries kI, const int64_t *q_pos, int B, int64_t n_q,
+                              int64_t E, int hI, int cI, int m, csa_dtype dt, float *scores,
+                              int64_t ld, void *stream)
+{
+    const char *w = "csa_indexer_scores";
+    REQUIRE(scores, CSA_ERR_INVALID_ARG, "%s: scores is required", w);
+    csa_status st = check_indexer(w, qI, qI_scale, wI, kI, q_pos, B, n_q, E, hI, cI, m, dt);
+    if (st != CSA_OK)
+        return st;
+    REQUIRE(ld >= E, CSA_ERR_INVALID_ARG, "%s: ld < E", w);
     unsigned *err = err_word();
     REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
     csa::IndexerArgs a{qI, qI_scale, wI, kI, q_pos, B, n_q, E, hI, cI, m, dt, scores, ld};
@@ -185,6 +206,55 @@ csa_status csa_indexer_scores(const void *qI, const float *qI_scale, const float
 size_t csa_topk_workspace_size(int64_t rows, int64_t E, int k)
 {
     return csa::topk_workspace_size(rows, E, k);
+}
+
+size_t csa_indexer_topk_workspace_size(int B, int64_t n_q, int64_t E, int hI, int cI, int k,
+                                       csa_dtype dt)
+{
+    if (B < 0 || n_q < 0 || E < 0 || E > INT32_MAX || k < 1 || k > 4096)
+        return 0;
+    return csa::indexer_topk_workspace_size(B, n_q, E, hI, cI, k, dt);
+}
+
+int csa_indexer_topk_launches(int B, int64_t n_q, int64_t E, int hI, int cI, int k,
+                              csa_dtype dt)
+{
+    if (B < 0 || n_q < 0 || E < 0 || E > INT32_MAX || k < 1 || k > 4096 ||
+        (dt != CSA_F32 && dt != CSA_BF16 && dt != CSA_E4M3))
+        return -1;
+    // 16-byte aligned stand-ins: only the shapes decide
+    static const uint8_t dummy[16] __attribute__((aligned(256))) = {0};
+    csa_entries kI{};
+    kI.body = const_cast<uint8_t *>(dummy);
+    kI.c = cI;
+    kI.dt = dt;
+    csa::IndexerArgs ix{dummy, nullptr, nullptr, kI, nullptr, B, n_q, E, hI, cI, 1, dt,
+                        nullptr, E};
+    return csa::indexer_topk_launches(ix, k);
+}
+
+csa_status csa_indexer_topk(const void *qI, const float *qI_scale, const float *wI,
+                            csa_entries kI, const int64_t *q_pos, int B, int64_t n_q, int64_t E,
+                            int hI, int cI, int m, csa_dtype dt, int k, int32_t *idx,
+                            void *workspace, size_t ws_bytes, void *stream)
+{
+    const char *w = "csa_indexer_topk";
+    REQUIRE(idx, CSA_ERR_INVALID_ARG, "%s: idx is required", w);
+    csa_status st = check_indexer(w, qI, qI_scale, wI, kI, q_pos, B, n_q, E, hI, cI, m, dt);
+    if (st != CSA_OK)
+        return st;
+    REQUIRE(k >= 1 && k <= 4096, CSA_ERR_UNSUPPORTED, "%s: k = %d out of [1, 4096]", w, k);
+    REQUIRE((int64_t)B * n_q <= INT32_MAX, CSA_ERR_INVALID_ARG, "%s: too many rows", w);
+    const size_t need = csa::indexer_topk_workspace_size(B, n_q, E, hI, cI, k, dt);
+    REQUIRE(ws_bytes >= need && (need == 0 || workspace), CSA_ERR_INVALID_ARG,
+            "%s: workspace of %zu bytes required", w, need);
+    REQUIRE(((uintptr_t)workspace & 255u) == 0, CSA_ERR_INVALID_ARG,
+            "%s: workspace must be 256-byte aligned", w);
+    unsigned *err = err_word();
+    REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
+    csa::IndexerArgs ix{qI, qI_scale, wI, kI, q_pos, B, n_q, E, hI, cI, m, dt, nullptr, E};
+    csa::IndexerTopkArgs a{ix, k, idx, workspace, ws_bytes};
+    return launched(csa::launch_indexer_topk(a, err, (cudaStream_t)stream), w);
 }
 
 csa_status csa_topk(const float *scores, int64_t rows, int64_t E, int64_t ld,

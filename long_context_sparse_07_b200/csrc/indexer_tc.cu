@@ -45,6 +45,17 @@ struct TcArgs {
     int64_t key_chunk;
     float *scores;
     int64_t ld;
+    int64_t ks_stride;    // key s has its scale at kI_scale[s * ks_stride]
+    const int *row_flag;  // when set: blocks none of whose tokens is flagged exit
+    // candidate mode (FUSE): every visible key of row r scoring at or above
+    // bound[r] is kept as a (score bits, index) pair in cand; rows of at most
+    // k visible keys keep nothing
+    const float *bound;
+    int k;
+    uint2 *cand;          // row r, chunk c, list l: cand[r * cand_ld + c * key_chunk / 2
+                          //                             + l * room of a list ..]
+    int64_t cand_ld;
+    uint32_t *cnt;        // [rows][nchunks][lists] pairs found (may exceed the room)
     unsigned *err;
 };
 
@@ -70,7 +81,7 @@ struct Cfg {
     static size_t smem_bytes(int kb)
     {
         return 1024 + (size_t)kb * QROWS * 128 + (size_t)STAGES * kb * 16384 + 256 + QROWS * 4 +
-               TT * 8;
+               TT * 16;
     }
 };
 
@@ -94,7 +105,7 @@ __device__ __forceinline__ float relu_dot(const uint32_t *x, const float *w)
     return acc0.x + acc0.y;
 }
 
-template <bool FP8, int HI, int NT, int NSUB>
+template <bool FP8, int HI, int NT, int NSUB, bool FUSE>
 __global__ void __launch_bounds__(Cfg<FP8, HI, NT, NSUB>::THREADS, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmq,
                   const TcArgs a)
@@ -115,6 +126,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     int *abort_flag = (int *)(tmem_slot + 1);
     float *wsm = (float *)(bars + 32);
     int64_t *vt = (int64_t *)(wsm + C::QROWS);
+    float *lbound = (float *)(vt + TT);            // FUSE: per token
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.y;
@@ -126,7 +138,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 
     if (threadIdx.x < TT) {
         const int64_t t = t0 + threadIdx.x;
-        vt[threadIdx.x] = t < a.n_q ? visible(a.q_pos[(int64_t)b * a.n_q + t], a.m, a.E) : 0;
+        int64_t v = t < a.n_q ? visible(a.q_pos[(int64_t)b * a.n_q + t], a.m, a.E) : 0;
+        if (a.row_flag && v > 0 && a.row_flag[(int64_t)b * a.n_q + t] == 0)
+            v = 0;                                 // a row that needs no scores
+        vt[threadIdx.x] = v;
     }
     if (threadIdx.x == 0)
         *abort_flag = 0;
@@ -174,6 +189,15 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     wv *= a.qI_scale[r];
             }
             wsm[col] = wv;
+        }
+        if constexpr (FUSE) {
+            // each token's bound (NaN: the row keeps nothing here, all of its
+            // visible keys being the selection)
+            for (int tt = threadIdx.x - 64; tt < TT; tt += C::THREADS - 64) {
+                const int64_t t = t0 + tt;
+                lbound[tt] = t < a.n_q && vt[tt] > a.k ? a.bound[(int64_t)b * a.n_q + t]
+                                                        : __int_as_float(0x7fc00000);
+            }
         }
     }
     tc::fence_before();
@@ -273,6 +297,32 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         const int part = ((warp - 2) >> 2) % C::SPLIT;
         const int row = q4 * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+        // FUSE: a token's pairs from this key chunk go to one list per
+        // epilogue warp that reduces it ((set, lane quarter): 4 NSET lists),
+        // each with an equal share of the chunk's room; the warp counts its
+        // lists in registers (the same count on every lane)
+        constexpr int LISTS = 4 * C::NSET;
+        const unsigned room_l =
+            (unsigned)(((s_begin + a.key_chunk < a.E ? s_begin + a.key_chunk : a.E) - s_begin) / 2 /
+                       LISTS);
+        const int list = set * 4 + q4;
+        const unsigned lt = (1u << lane) - 1u;
+        // per token of this warp (slot j * TPW + x): its list, bound and
+        // visible length, kept in registers across the key tiles
+        // (the candidate area of a row is at most a few MB: offsets within a
+        // block's rows fit in 32 bits)
+        constexpr int SLOTS = FUSE ? NSUB * C::TPW : 1;
+        uint2 *const dbase =
+            a.cand + ((int64_t)b * a.n_q + t0) * a.cand_ld + s_begin / 2 + (int64_t)list * room_l;
+        const unsigned cld = (unsigned)a.cand_ld;
+        unsigned wc[SLOTS];
+        float lbv[SLOTS];
+#pragma unroll
+        for (int j = 0; j < SLOTS; j++) {
+            const int tt = (j / C::TPW) * NT + part * C::TPW + j % C::TPW;
+            wc[j] = 0u;
+            lbv[j] = FUSE ? lbound[tt] : 0.f;
+        }
         bool ok = true;
         for (int i = 0; i < ntiles && ok; i++) {
             if (C::NSET == 2 && NSUB == 1 && (i & 1) != set)
@@ -281,17 +331,16 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             // the key's scale is requested before the wait for its accumulator
             float ks = 1.f;
             if (FP8)
-                ks = s < a.E ? __ldg(a.kI_scale + (int64_t)b * a.E + s) : 0.f;
-#pragma unroll 1
-            for (int j = 0; j < NSUB; j++) {
+                ks = s < a.E ? __ldg(a.kI_scale + ((int64_t)b * a.E + s) * a.ks_stride) : 0.f;
+            auto group = [&](const int j) {
                 const int g = i * NSUB + j, buf = g & 1;
                 if (C::NSET == 2 && buf != set)
-                    continue;
+                    return;
                 if (!tc::mbar_wait(&accf[buf], (g / 2) & 1, abort_flag)) {
                     *abort_flag = 1;
                     report(a.err, CSA_ERR_TIMEOUT, K_INDEXER_TC, blockIdx.x, 2);
                     ok = false;
-                    break;
+                    return;
                 }
                 tc::fence_after();
                 const uint32_t base = lane_addr + (uint32_t)(buf * N);
@@ -316,8 +365,22 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     sacc += relu_dot<CW>(rb[c & 1], wsm + tt * HI + (c % CPT) * CW);
                     if (c % CPT == CPT - 1) {
                         const int64_t t = t0 + tt;
-                        if (t < a.n_q && s < vt[tt])
-                            a.scores[((int64_t)b * a.n_q + t) * a.ld + s] = sacc * ks;
+                        if constexpr (FUSE) {
+                            // candidates of token tt: the lanes at or above
+                            // its bound, in lane order after this list's count
+                            const int sl = j * C::TPW + c / CPT;
+                            const float v = sacc * ks;
+                            const bool on = s < vt[tt] && v >= lbv[sl];
+                            const unsigned bal = __ballot_sync(0xffffffffu, on);
+                            const unsigned at = wc[sl] + (unsigned)__popc(bal & lt);
+                            if (on && at < room_l)
+                                dbase[(unsigned)tt * cld + at] =
+                                    make_uint2(__float_as_uint(v), (uint32_t)s);
+                            wc[sl] += (unsigned)__popc(bal);
+                        } else {
+                            if (t < a.n_q && s < vt[tt])
+                                a.scores[((int64_t)b * a.n_q + t) * a.ld + s] = sacc * ks;
+                        }
                         sacc = 0.f;
                     }
                     if (c + 1 < NC)
@@ -327,6 +390,30 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 __syncwarp();
                 if (lane == 0)
                     tc::mbar_arrive(&acce[buf]);
+            };
+            if constexpr (FUSE) {
+                // unrolled, so that every list count stays in a register
+#pragma unroll
+                for (int j = 0; j < NSUB; j++)
+                    if (ok)
+                        group(j);
+            } else {
+#pragma unroll 1
+                for (int j = 0; j < NSUB && ok; j++)
+                    group(j);
+            }
+        }
+        if constexpr (FUSE) {
+            if (lane == 0) {
+#pragma unroll
+                for (int j = 0; j < NSUB; j++)
+#pragma unroll
+                    for (int x = 0; x < C::TPW; x++) {
+                        const int64_t t = t0 + j * NT + part * C::TPW + x;
+                        if (t < a.n_q)
+                            a.cnt[(((int64_t)b * a.n_q + t) * a.nchunks + chunk) * LISTS +
+                                  list] = wc[j * C::TPW + x];
+                    }
             }
         }
     }
@@ -338,18 +425,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     }
 }
 
-template <bool FP8, int HI, int NT, int NSUB>
-cudaError_t launch_one(const IndexerArgs &a, unsigned *err, cudaStream_t s)
+template <bool FP8, int HI, int NT, int NSUB, bool FUSE>
+cudaError_t launch_one(const IndexerArgs &a, const IndexerTcExtra &x, unsigned *err, cudaStream_t s)
 {
     using C = Cfg<FP8, HI, NT, NSUB>;
     const int esize = FP8 ? 1 : 2;
-    CUtensorMap tmk, tmq;
-    const CUtensorMapDataType dt =
-        FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if (!make_tmap_2d(&tmk, a.kI.body, dt, esize, (uint64_t)a.B * a.E, a.cI, 128) ||
-        !make_tmap_2d(&tmq, a.qI, dt, esize, (uint64_t)a.B * a.n_q * HI, a.cI,
-                      C::QROWS < 256 ? C::QROWS : 256))
-        return cudaErrorInvalidValue;
     TcArgs t;
     t.wI = a.wI;
     t.qI_scale = a.qI_scale;
@@ -362,9 +442,10 @@ cudaError_t launch_one(const IndexerArgs &a, unsigned *err, cudaStream_t s)
     const int64_t ttiles = (a.n_q + C::TT - 1) / C::TT;
     // few token tiles: split the keys of each tile over several blocks, sized
     // so that all blocks run in one wave (two resident blocks per SM)
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int dev = 0, sms = 148, nsm = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && nsm > 0)
+        sms = nsm;
     const int64_t target = 2 * (int64_t)sms;
     t.key_chunk = a.E;
     t.nchunks = 1;
@@ -376,61 +457,105 @@ cudaError_t launch_one(const IndexerArgs &a, unsigned *err, cudaStream_t s)
     }
     t.scores = a.scores;
     t.ld = a.ld;
+    t.ks_stride = x.key_step;
+    t.row_flag = x.row_flag;
+    t.bound = x.bound;
+    t.k = x.k;
+    t.cand = (uint2 *)a.scores;
+    t.cand_ld = a.ld / 2;
+    t.cnt = x.cnt;
     t.err = err;
+    if (x.nchunks_out)
+        *x.nchunks_out = t.nchunks;
+    if (x.lists_out)
+        *x.lists_out = 4 * C::NSET;
+    if (x.key_chunk_out)
+        *x.key_chunk_out = t.key_chunk;
+    if (x.plan_only)
+        return cudaSuccess;
+    CUtensorMap tmk, tmq;
+    const CUtensorMapDataType dt =
+        FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    // key s of the table is row s * key_step of kI.body
+    if (!make_tmap_2d(&tmk, a.kI.body, dt, esize, (uint64_t)a.B * a.E, a.cI, 128,
+                      (uint64_t)x.key_step * a.cI * esize) ||
+        !make_tmap_2d(&tmq, a.qI, dt, esize, (uint64_t)a.B * a.n_q * HI, a.cI,
+                      C::QROWS < 256 ? C::QROWS : 256))
+        return cudaErrorInvalidValue;
     const size_t smem = C::smem_bytes(t.kb);
-    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<FP8, HI, NT, NSUB>,
+    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<FP8, HI, NT, NSUB, FUSE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
     dim3 grid((unsigned)(ttiles * t.nchunks), (unsigned)a.B);
-    indexer_tc_kernel<FP8, HI, NT, NSUB><<<grid, C::THREADS, smem, s>>>(tmk, tmq, t);
+    indexer_tc_kernel<FP8, HI, NT, NSUB, FUSE><<<grid, C::THREADS, smem, s>>>(tmk, tmq, t);
     return cudaGetLastError();
 }
 
+template <bool FP8, int HI, int NT, int NSUB>
+cudaError_t launch_mode(const IndexerArgs &a, const IndexerTcExtra &x, unsigned *err,
+                        cudaStream_t s)
+{
+    return x.fuse ? launch_one<FP8, HI, NT, NSUB, true>(a, x, err, s)
+                  : launch_one<FP8, HI, NT, NSUB, false>(a, x, err, s);
+}
+
 template <bool FP8>
-cudaError_t dispatch_heads(const IndexerArgs &a, unsigned *err, cudaStream_t s, bool few)
+cudaError_t dispatch_heads(const IndexerArgs &a, const IndexerTcExtra &x, unsigned *err,
+                           cudaStream_t s, bool few)
 {
     // prefill: a block takes 16 tokens (e4m3) or one group of N = 256 (bf16,
     // whose key tiles are twice the size); decode: one token per block
     switch (a.hI) {
     case 16:
-        return few ? launch_one<FP8, 16, 1, 1>(a, err, s) : launch_one<FP8, 16, 16, 1>(a, err, s);
+        return few ? launch_mode<FP8, 16, 1, 1>(a, x, err, s)
+                   : launch_mode<FP8, 16, 16, 1>(a, x, err, s);
     case 32:
         if (few)
-            return launch_one<FP8, 32, 1, 1>(a, err, s);
+            return launch_mode<FP8, 32, 1, 1>(a, x, err, s);
         if constexpr (FP8)
-            return launch_one<FP8, 32, 8, 2>(a, err, s);
+            return launch_mode<FP8, 32, 8, 2>(a, x, err, s);
         else
-            return launch_one<FP8, 32, 8, 1>(a, err, s);
+            return launch_mode<FP8, 32, 8, 1>(a, x, err, s);
     case 64:
         if (few)
-            return launch_one<FP8, 64, 1, 1>(a, err, s);
+            return launch_mode<FP8, 64, 1, 1>(a, x, err, s);
         if constexpr (FP8)
-            return launch_one<FP8, 64, 4, 4>(a, err, s);
+            return launch_mode<FP8, 64, 4, 4>(a, x, err, s);
         else
-            return launch_one<FP8, 64, 4, 1>(a, err, s);
+            return launch_mode<FP8, 64, 4, 1>(a, x, err, s);
     }
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_indexer_tc(const IndexerArgs &a, unsigned *err, cudaStream_t s, bool *taken)
+bool indexer_tc_takes(const IndexerArgs &a)
 {
-    *taken = false;
     if (a.dt == CSA_F32)
-        return cudaSuccess;
+        return false;
     if (a.hI != 16 && a.hI != 32 && a.hI != 64)
-        return cudaSuccess;
+        return false;
     const int esize = a.dt == CSA_E4M3 ? 1 : 2;
     if ((a.cI * esize) % 128 != 0 || a.cI * esize > 256)
-        return cudaSuccess;
-    if (((uintptr_t)a.qI & 15) || ((uintptr_t)a.kI.body & 15))
-        return cudaSuccess;
-    *taken = true;
+        return false;
+    return ((uintptr_t)a.qI & 15) == 0 && ((uintptr_t)a.kI.body & 15) == 0;
+}
+
+cudaError_t launch_indexer_tc_ex(const IndexerArgs &a, const IndexerTcExtra &x, unsigned *err,
+                                 cudaStream_t s)
+{
     const bool few = a.n_q <= 8;
-    return a.dt == CSA_E4M3 ? dispatch_heads<true>(a, err, s, few)
-                            : dispatch_heads<false>(a, err, s, few);
+    return a.dt == CSA_E4M3 ? dispatch_heads<true>(a, x, err, s, few)
+                            : dispatch_heads<false>(a, x, err, s, few);
+}
+
+cudaError_t launch_indexer_tc(const IndexerArgs &a, unsigned *err, cudaStream_t s, bool *taken)
+{
+    *taken = indexer_tc_takes(a);
+    if (!*taken)
+        return cudaSuccess;
+    return launch_indexer_tc_ex(a, IndexerTcExtra{}, err, s);
 }
 
 }  // namespace csa

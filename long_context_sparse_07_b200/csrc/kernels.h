@@ -43,6 +43,67 @@ struct TopkArgs {
 cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s);
 size_t topk_workspace_size(int64_t rows, int64_t E, int k);
 
+// Options of the tensor-core indexer beyond the plain call.
+struct IndexerTcExtra {
+    int key_step = 1;                // key s of the table is row s * key_step of kI
+    const int *row_flag = nullptr;   // score only rows whose flag is nonzero
+    bool fuse = false;               // candidate mode (see indexer_tc.cu)
+    const float *bound = nullptr;    // candidate mode: per-row lower bounds
+    int k = 0;
+    uint32_t *cnt = nullptr;         // [rows][nchunks][lists] pair counts
+    bool plan_only = false;          // only report the key chunking
+    int *nchunks_out = nullptr;
+    int64_t *key_chunk_out = nullptr;
+    int *lists_out = nullptr;
+};
+bool indexer_tc_takes(const IndexerArgs &a);
+cudaError_t launch_indexer_tc_ex(const IndexerArgs &a, const IndexerTcExtra &x, unsigned *err,
+                                 cudaStream_t s);
+
+// Selection from the candidate pairs of the indexer's candidate mode: writes
+// idx rows (or flags the row when its pairs do not decide the top-k).
+struct TopkCandArgs {
+    const uint2 *cand;               // (float bits of the score, index)
+    int64_t cand_ld;
+    const uint32_t *cnt;
+    int nchunks, lists;
+    int64_t key_chunk;
+    const int64_t *q_pos;
+    int m;
+    int64_t E, rows;
+    int k;
+    int32_t *idx;
+    int *flag;
+};
+cudaError_t launch_topk_cand(const TopkCandArgs &a, cudaStream_t s);
+bool topk_cand_fits(int64_t E, int nchunks, int lists, int64_t rows);
+// Per-row lower bound for the candidate mode from sample scores.
+struct TopkBoundArgs {
+    const float *samp;               // [rows, samp_ld]: scores of keys 0, S, 2S, ..
+    int64_t samp_ld;
+    const int64_t *q_pos;
+    int m, S, k;
+    int64_t E, rows;
+    float *bound;
+};
+cudaError_t launch_topk_bound(const TopkBoundArgs &a, cudaStream_t s);
+// Top-k of the flagged rows only (rows whose flag is zero are left alone).
+cudaError_t launch_topk_flagged(const TopkArgs &a, const int *flag, cudaStream_t s);
+
+// The indexer and the top-k in one call (csa_indexer_topk).
+struct IndexerTopkArgs {
+    IndexerArgs ix;
+    int k;
+    int32_t *idx;
+    void *ws;
+    size_t ws_bytes;
+};
+cudaError_t launch_indexer_topk(const IndexerTopkArgs &a, unsigned *err, cudaStream_t s);
+int indexer_topk_launches(const IndexerArgs &ix, int k);
+size_t indexer_topk_workspace_size(int B, int64_t n_q, int64_t E, int hI, int cI, int k,
+                                   csa_dtype dt);
+
+
 struct AttendArgs {
     const void *q;
     csa_dtype q_dt;

@@ -25,15 +25,16 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 
 // Row-major [rows, cols] matrix of `esize`-byte elements, read in boxes of
 // box_rows x (128 / esize) elements with the 128-byte swizzle; out-of-range
-// rows read as zero. Returns false when the map cannot be encoded.
+// rows read as zero. Rows lie `row_bytes` apart (0: cols * esize, packed).
+// Returns false when the map cannot be encoded.
 inline bool make_tmap_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize,
-                         uint64_t rows, uint64_t cols, uint32_t box_rows)
+                         uint64_t rows, uint64_t cols, uint32_t box_rows, uint64_t row_bytes = 0)
 {
     auto enc = tensor_map_encoder();
     if (!enc)
         return false;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)(cols * esize)};
+    cuuint64_t strides[1] = {(cuuint64_t)(row_bytes ? row_bytes : cols * esize)};
     cuuint32_t box[2] = {(cuuint32_t)(128 / esize), (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,

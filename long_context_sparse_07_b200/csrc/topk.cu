@@ -283,22 +283,44 @@ __device__ void block_select(const Src &src, int64_t V, int k, int32_t *__restri
 }
 
 __global__ void __launch_bounds__(kThreads)
-topk_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
+topk_kernel(const float *__restrict__ scores, int64_t rows, int64_t E, int64_t ld,
             const int64_t *__restrict__ q_pos, int m, int k, int32_t *__restrict__ idx,
-            int resident)
+            int resident, const int *__restrict__ row_flag)
 {
     extern __shared__ uint32_t keys[];
     __shared__ Shared sh;
-    const int64_t row = blockIdx.x;
-    const int64_t V = visible(q_pos[row], m, E);
-    int32_t *out = idx + row * k;
-    if (V <= k) {
-        for (int j = threadIdx.x; j < k; j += kThreads)
-            out[j] = j < V ? j : -1;
+    __shared__ int fl[kThreads];
+    auto one = [&](int64_t row) {
+        const int64_t V = visible(q_pos[row], m, E);
+        int32_t *out = idx + row * k;
+        if (V <= k) {
+            for (int j = threadIdx.x; j < k; j += kThreads)
+                out[j] = j < V ? j : -1;
+            return;
+        }
+        RowScores src{scores + row * ld};
+        block_select(src, V, k, out, keys, resident && V <= kResident, sh);
+        __syncthreads();                          // shared state reused by the next row
+    };
+    if (!row_flag) {
+        one(blockIdx.x);                          // one row per block
         return;
     }
-    RowScores src{scores + row * ld};
-    block_select(src, V, k, out, keys, resident && V <= kResident, sh);
+    // the flagged rows only: the flags of kThreads rows at a time, then the
+    // flagged ones among them in turn
+    for (int64_t r0 = (int64_t)blockIdx.x * kThreads; r0 < rows;
+         r0 += (int64_t)gridDim.x * kThreads) {
+        const int64_t my = r0 + threadIdx.x;
+        const int f = my < rows ? row_flag[my] : 0;
+        if (!__syncthreads_or(f))
+            continue;
+        fl[threadIdx.x] = f;
+        __syncthreads();
+        for (int j = 0; j < kThreads && r0 + j < rows; j++)
+            if (fl[j])
+                one(r0 + j);
+        __syncthreads();                          // fl reused
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -979,6 +1001,244 @@ topk_warp_kernel(const float *__restrict__ scores, int64_t rows, int64_t E, int6
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Selection from candidate pairs (the indexer's candidate mode, one key
+// chunk per row). Row r holds `lists` lists of pairs (score bits, index):
+// list l has cnt[r][l] pairs at cand[r * cand_ld + l * room ..] (room = the
+// row's E / 2 pairs over the lists), in no particular order: every visible
+// entry whose score is at or above the row's lower bound. When every list fits
+// in its room and there are at least k pairs, the row's top-k is the top-k of
+// its pairs. One warp per row finds the k-th largest key T and how many keys
+// equal to T to take (8-bit radix digits, most significant first, over the
+// lists one after another), marks the chosen indices in a bitmap of the
+// row's visible range (the lowest indices among the keys equal to T through
+// a second bitmap), and writes the set bits in index order. A row whose pairs
+// overflowed or number fewer than k is flagged (flag[r] = 1) for the full
+// computation; the others get 0.
+
+constexpr int kCandRows = 8;           // rows (warps) per block
+constexpr int kCandMaxLists = 8;
+
+struct CandWarp {
+    unsigned hist[256];
+    unsigned bin, need, bcnt, pad;
+};
+
+__host__ __device__ inline size_t cand_warp_bytes(int words)
+{
+    return sizeof(CandWarp) + (size_t)2 * words * 4;
+}
+
+__global__ void __launch_bounds__(32 * kCandRows)
+topk_cand_kernel(const TopkCandArgs a, int words)
+{
+    extern __shared__ __align__(16) uint8_t cdyn[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint8_t *gbase = cdyn + (size_t)wid * cand_warp_bytes(words);
+    CandWarp &g = *reinterpret_cast<CandWarp *>(gbase);
+    uint32_t *bm_gt = (uint32_t *)(gbase + sizeof(CandWarp));
+    uint32_t *bm_eq = bm_gt + words;
+    const int64_t row = (int64_t)blockIdx.x * kCandRows + wid;
+    if (row >= a.rows)
+        return;
+    const int k = a.k;
+    int32_t *out = a.idx + row * k;
+    const int64_t V = visible(a.q_pos[row], a.m, a.E);
+    if (V <= k) {
+        for (int j = lane; j < k; j += 32)
+            out[j] = j < V ? j : -1;
+        if (lane == 0)
+            a.flag[row] = 0;
+        return;
+    }
+    // 1. the lists: counts, prefixes (the same on every lane)
+    const int L = a.lists;
+    const unsigned room = (unsigned)(a.E / 2 / L);
+    const uint32_t *ccnt = a.cnt + row * L;
+    const uint2 *crow = a.cand + row * a.cand_ld;
+    unsigned nx[kCandMaxLists];
+    unsigned total = 0;
+    bool over = false;
+#pragma unroll
+    for (int x = 0; x < kCandMaxLists; x++) {
+        nx[x] = x < L ? ccnt[x] : 0u;
+        over |= nx[x] > room;
+        total += nx[x];
+    }
+    if (over || total < (unsigned)k) {
+        if (lane == 0)
+            a.flag[row] = 1;
+        return;
+    }
+    // f(pair) for every pair of every list, eight loads in flight per lane
+    auto each = [&](auto &&f) {
+#pragma unroll
+        for (int x = 0; x < kCandMaxLists; x++) {
+            const uint2 *lp = crow + (int64_t)x * room;
+            for (unsigned f0 = 0; f0 < nx[x]; f0 += 256) {
+                uint2 p[8];
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const unsigned j = f0 + i * 32 + lane;
+                    p[i] = j < nx[x] ? lp[j] : make_uint2(0u, 0xffffffffu);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; i++)
+                    f(p[i], f0 + i * 32 + lane < nx[x]);
+            }
+        }
+    };
+    // 2. the k-th largest key T, and how many keys equal to T are taken
+    uint32_t prefix = 0, pmask = 0;
+    unsigned need = (unsigned)k, bcnt = 0;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int b = lane; b < 256; b += 32)
+            g.hist[b] = 0;
+        __syncwarp();
+        each([&](const uint2 &p, bool valid) {
+            const uint32_t u = float_key(__uint_as_float(p.x));
+            hist_add(g.hist, (u >> shift) & 255u, valid && (u & pmask) == prefix);
+        });
+        __syncwarp();
+        {
+            // bin where the count from the top reaches `need`
+            unsigned local = 0;
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                local += g.hist[255 - 8 * lane - j];
+            unsigned incl = local;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o)
+                    incl += y;
+            }
+            const unsigned ex = incl - local;
+            if (ex < need && need <= incl) {
+                unsigned cum = ex;
+                for (int j = 0; j < 8; j++) {
+                    const unsigned hb = g.hist[255 - 8 * lane - j];
+                    if (cum + hb >= need) {
+                        g.bin = 255u - 8u * lane - j;
+                        g.need = need - cum;
+                        g.bcnt = hb;
+                        break;
+                    }
+                    cum += hb;
+                }
+            }
+        }
+        __syncwarp();
+        prefix |= g.bin << shift;
+        pmask |= 255u << shift;
+        need = g.need;
+        bcnt = g.bcnt;
+        __syncwarp();                             // hist and the results reused
+    }
+    const uint32_t T = prefix;
+    // 3. bitmaps of the chosen indices: keys above T, and keys equal to T
+    // (straight into the first when all of them are taken)
+    const int W = (int)((V + 31) / 32);
+    for (int w = lane; w < W; w += 32) {
+        bm_gt[w] = 0u;
+        bm_eq[w] = 0u;
+    }
+    __syncwarp();
+    const bool cut = need < bcnt;
+    each([&](const uint2 &p, bool valid) {
+        const uint32_t s = p.y;
+        if (valid && (int64_t)s < V) {
+            const uint32_t u = float_key(__uint_as_float(p.x));
+            const uint32_t bit = 1u << (s & 31u);
+            if (u > T)
+                atomicOr(&bm_gt[s >> 5], bit);
+            else if (u == T)
+                atomicOr(cut ? &bm_eq[s >> 5] : &bm_gt[s >> 5], bit);
+        }
+    });
+    __syncwarp();
+    const int wper = (W + 31) / 32;
+    const int w0 = lane * wper, w1 = w0 + wper < W ? w0 + wper : W;
+    auto warp_excl = [&](unsigned v) -> unsigned {
+        unsigned incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += y;
+        }
+        return incl - v;
+    };
+    if (cut) {
+        // the `need` lowest indices among the keys equal to T
+        unsigned c = 0;
+        for (int w = w0; w < w1; w++)
+            c += (unsigned)__popc(bm_eq[w]);
+        unsigned e = warp_excl(c);
+        for (int w = w0; w < w1 && e < need; w++) {
+            uint32_t x = bm_eq[w];
+            const unsigned pc = (unsigned)__popc(x);
+            if (e + pc > need) {
+                unsigned keep = need - e;
+                uint32_t y = 0u;
+                while (keep--) {
+                    const uint32_t lb = x & (0u - x);
+                    y |= lb;
+                    x ^= lb;
+                }
+                x = y;
+            }
+            bm_gt[w] |= x;
+            e += (unsigned)__popc(x);
+        }
+        __syncwarp();
+    }
+    // 4. the chosen indices in ascending order
+    unsigned c = 0;
+    for (int w = w0; w < w1; w++)
+        c += (unsigned)__popc(bm_gt[w]);
+    unsigned e = warp_excl(c);
+    const unsigned tot = __reduce_add_sync(0xffffffffu, c);
+    for (int w = w0; w < w1; w++) {
+        uint32_t x = bm_gt[w];
+        while (x) {
+            const int b = __ffs(x) - 1;
+            x &= x - 1u;
+            if (e < (unsigned)k)
+                out[e] = w * 32 + b;
+            ++e;
+        }
+    }
+    for (int j = (int)tot + lane; j < k; j += 32)
+        out[j] = -1;
+    if (lane == 0)
+        a.flag[row] = 0;
+}
+
+bool topk_cand_fits(int64_t E, int nchunks, int lists, int64_t rows)
+{
+    (void)rows;
+    const int words = (int)((E + 31) / 32);
+    return nchunks == 1 && lists >= 1 && lists <= kCandMaxLists &&
+           kCandRows * cand_warp_bytes(words) <= 227 * 1024;
+}
+
+cudaError_t launch_topk_cand(const TopkCandArgs &a, cudaStream_t s)
+{
+    if (a.rows == 0)
+        return cudaSuccess;
+    const int words = (int)((a.E + 31) / 32);
+    const size_t smem = kCandRows * cand_warp_bytes(words);
+    cudaError_t e = cudaFuncSetAttribute(topk_cand_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    topk_cand_kernel<<<(unsigned)((a.rows + kCandRows - 1) / kCandRows), 32 * kCandRows, smem,
+                       s>>>(a, words);
+    return cudaGetLastError();
+}
+
 size_t topk_workspace_size(int64_t rows, int64_t E, int k)
 {
     (void)k;
@@ -1031,8 +1291,94 @@ cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s)
     const int resident = a.E > a.k;
     const int64_t cap = a.E < kResident ? a.E : kResident;
     const size_t smem = resident ? (size_t)cap * sizeof(uint32_t) : 0;
-    topk_kernel<<<(unsigned)a.rows, kThreads, smem, s>>>(a.scores, a.E, a.ld, a.q_pos, a.m,
-                                                         a.k, a.idx, resident);
+    topk_kernel<<<(unsigned)a.rows, kThreads, smem, s>>>(a.scores, a.rows, a.E, a.ld, a.q_pos,
+                                                         a.m, a.k, a.idx, resident, nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk_flagged(const TopkArgs &a, const int *flag, cudaStream_t s)
+{
+    if (a.rows == 0)
+        return cudaSuccess;
+    // the rows are re-read from memory at every digit past the staged size
+    const int64_t cap = a.E < kResident ? a.E : kResident;
+    const size_t smem = (size_t)cap * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kResident * (int)sizeof(uint32_t));
+    if (e != cudaSuccess)
+        return e;
+    int dev = 0, sms = 148, nsm = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && nsm > 0)
+        sms = nsm;
+    const int64_t chunks = (a.rows + kThreads - 1) / kThreads;
+    const int64_t grid = chunks < sms ? chunks : sms;
+    topk_kernel<<<(unsigned)grid, kThreads, smem, s>>>(a.scores, a.rows, a.E, a.ld, a.q_pos, a.m,
+                                                       a.k, a.idx, 1, flag);
+    return cudaGetLastError();
+}
+
+// Lower bound of each row for the candidate mode: from the row's visible
+// samples (scores of keys 0, S, 2S, .. below V, ns = floor(V / S) of them),
+// the ks-th largest, ks = 1.25 mu + 4 sqrt(mu) + 8 where mu = k ns / V is
+// the number of samples expected at or above the row's k-th largest score:
+// the row's k-th largest lies below it only when the sample is off by many
+// standard deviations (then the row is recomputed in full). -inf (keep every
+// visible key) when there are too few samples; NaN (keep none) when the row
+// has at most k visible keys. One warp per row: the top 16 bits of that
+// sample's key are found bit by bit, each step counting the samples at or
+// above the candidate; the bound is the float of those bits with the rest
+// zero (never above the sample itself).
+constexpr int kBoundRows = 8;
+
+__global__ void __launch_bounds__(32 * kBoundRows)
+topk_bound_kernel(const TopkBoundArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kBoundRows + (threadIdx.x >> 5);
+    if (row >= a.rows)
+        return;
+    const int64_t V = visible(a.q_pos[row], a.m, a.E);
+    float out = __int_as_float(0x7fc00000);
+    if (V > a.k) {
+        out = -INFINITY;
+        const int64_t ns = V / a.S;
+        const float mu = (float)a.k * (float)ns / (float)V;
+        const float ksf = 1.25f * mu + 4.f * sqrtf(mu) + 8.f;
+        if (ns <= 1024 && ksf <= (float)ns) {
+            const unsigned ks = (unsigned)ksf;
+            const float *srow = a.samp + row * a.samp_ld;
+            uint32_t u[32];
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                const int64_t j = lane + 32 * i;
+                u[i] = j < ns ? float_key(__ldg(srow + j)) : 0u;
+            }
+            uint32_t T = 0u;
+#pragma unroll 1
+            for (int bit = 31; bit >= 16; bit--) {
+                const uint32_t c = T | (1u << bit);
+                unsigned n = 0;
+#pragma unroll
+                for (int i = 0; i < 32; i++)
+                    n += u[i] >= c ? 1u : 0u;
+                if (__reduce_add_sync(0xffffffffu, n) >= ks)
+                    T = c;
+            }
+            // back to a float (the key of +0 and -0 gives +0)
+            out = __uint_as_float((T & 0x80000000u) ? (T & 0x7fffffffu) : ~T);
+        }
+    }
+    if (lane == 0)
+        a.bound[row] = out;
+}
+
+cudaError_t launch_topk_bound(const TopkBoundArgs &a, cudaStream_t s)
+{
+    if (a.rows == 0)
+        return cudaSuccess;
+    topk_bound_kernel<<<(unsigned)((a.rows + kBoundRows - 1) / kBoundRows), 32 * kBoundRows, 0,
+                        s>>>(a);
     return cudaGetLastError();
 }
 

@@ -4,7 +4,9 @@
 outputs in device memory and run one pass of the path per ``step()``:
 
 * CSA prefill: compress KV entries -> compress indexer keys -> indexer scores
-  -> top-k -> sparse shared-KV attention (window + sink);
+  -> top-k -> sparse shared-KV attention (window + sink); with ``fused`` the
+  scores and the top-k are one call (``csa_indexer_topk``) that does not
+  write the score rows;
 * HCA prefill: compress (m' = 128, no overlap) -> dense shared-KV attention;
 * decode: indexer scores -> top-k -> sparse attention, and HCA dense
   attention, for a batch of single-token queries over long caches.
@@ -39,10 +41,17 @@ class CsaPrefill:
     def launches_per_step(self):
         """Kernels launched by one step (top-k of long rows takes four; the
         normalisation and RoPE add four)."""
-        return 4 + (4 if self.topk_ws is not None else 1) + (4 if self.rope_dims else 0)
+        if self.fused:
+            sel = abi.csa_indexer_topk_launches(1, self.w.n, self.w.E, self.w.hI, self.w.cI,
+                                                self.w.k, self.d["qI"])
+        else:
+            sel = 1 + (4 if self.topk_ws is not None else 1)
+        return 3 + sel + (4 if self.rope_dims else 0)
 
-    def __init__(self, w, ops: Dict[str, torch.Tensor], device="cuda", rope_dims: int = 0):
+    def __init__(self, w, ops: Dict[str, torch.Tensor], device="cuda", rope_dims: int = 0,
+                 fused: bool = False):
         self.w = w
+        self.fused = fused
         d = self.d = _dev(ops, device)
         n, c, E = w.n, w.c, w.E
         # with rope_dims > 0 the step also applies Module D's RMSNorm and
@@ -59,10 +68,15 @@ class CsaPrefill:
                               scale_group=w.cI)
         else:
             self.kI = Entries(torch.empty(E, w.cI, device=device, dtype=DT[w.idx_dtype]), w.cI)
-        self.scores = torch.empty(1, n, E, device=device, dtype=torch.float32)
         self.idx = torch.empty(n, w.k, device=device, dtype=torch.int32)
-        nt = abi.csa_topk_workspace_size(n, E, w.k)
-        self.topk_ws = torch.empty(nt, device=device, dtype=torch.uint8) if nt else None
+        if fused:
+            self.scores = self.topk_ws = None
+            nf = abi.csa_indexer_topk_workspace_size(1, n, E, w.hI, w.cI, w.k, d["qI"])
+            self.fused_ws = torch.empty(nf, device=device, dtype=torch.uint8) if nf else None
+        else:
+            self.scores = torch.empty(1, n, E, device=device, dtype=torch.float32)
+            nt = abi.csa_topk_workspace_size(n, E, w.k)
+            self.topk_ws = torch.empty(nt, device=device, dtype=torch.uint8) if nt else None
         self.out = torch.empty(1, n, w.h, c, device=device, dtype=DT[w.dtype])
         self.lse = torch.empty(1, n, w.h, device=device, dtype=torch.float32)
         self.scale = 1.0 / math.sqrt(c)
@@ -89,6 +103,14 @@ class CsaPrefill:
         abi.csa_topk(self.scores[0], self.q_pos, w.m, w.k, self.idx, w.E, workspace=self.topk_ws,
                      stream=stream)
 
+    def index_select(self, stream=None):
+        """Indexer scores and top-k in one call (no score rows written)."""
+        d, w = self.d, self.w
+        qs = d.get("qI_scale")
+        abi.csa_indexer_topk(d["qI"][None], qs[None] if qs is not None else None, d["wI"][None],
+                             self.kI, self.q_pos[None], w.m, w.k, self.idx, w.E,
+                             workspace=self.fused_ws, stream=stream)
+
     def attend(self, stream=None):
         d, w = self.d, self.w
         abi.csa_sparse_mqa(d["q"][None], self.entries, w.E, w.m, self.idx, w.k, self.kwin[None],
@@ -113,11 +135,13 @@ class CsaPrefill:
 
     def phases(self):
         """The kernels of one step, in order: (name, launch)."""
-        ph = [("compress_kv", self.compress_kv), ("compress_index", self.compress_index),
-              ("indexer", self.index), ("topk", self.select), ("attend", self.attend)]
+        sel = [("indexer_topk", self.index_select)] if self.fused else \
+            [("indexer", self.index), ("topk", self.select)]
+        ph = [("compress_kv", self.compress_kv), ("compress_index", self.compress_index)] + sel + \
+            [("attend", self.attend)]
         if self.rope_dims:
-            ph = ph[:1] + [("rope_kv", self.rope_kv)] + ph[1:4] + [("rope_q", self.rope_q)] + \
-                ph[4:] + [("rotate_back", self.rotate_back)]
+            ph = ph[:1] + [("rope_kv", self.rope_kv)] + ph[1:-1] + [("rope_q", self.rope_q)] + \
+                ph[-1:] + [("rotate_back", self.rotate_back)]
         return ph
 
     def inputs(self):

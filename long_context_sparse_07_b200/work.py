@@ -41,6 +41,10 @@ def csa_prefill(w) -> Dict[str, Dict[str, float]]:
                       "bytes": n * w.hI * w.cI * bi + n * w.hI * 4 + E * w.cI * ki_bytes
                       + pairs * 4}
     out["topk"] = {"bytes": pairs * 4 + n * w.k * 4 + n * 8, "flops": 0}
+    # the indexer and the top-k in one call: the score rows are neither
+    # written nor read back
+    out["indexer_topk"] = {"flops": out["indexer"]["flops"],
+                           "bytes": out["indexer"]["bytes"] - pairs * 4 + n * w.k * 4}
     out["attend"] = {"flops": 4 * keys * w.h * c,
                      "bytes": 2 * n * w.h * c * b + E * c * b + n * c * b + n * w.k * 4
                      + n * w.h * 4}

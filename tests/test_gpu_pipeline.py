@@ -110,6 +110,18 @@ def run_csa(w, rows, ops=None, ref=None):
     # selection, first level: the oracle's top-k over the GPU's own float32
     # score rows is the GPU's selection exactly (same values, same tie rule)
     np.testing.assert_array_equal(gidx, oracle.topk(sc, rows, w.m, w.k))
+    # the indexer and the top-k in one call select exactly the same, on
+    # every row (both select on the same float32 scores)
+    qs = p.d.get("qI_scale")
+    nws = abi.csa_indexer_topk_workspace_size(1, w.n, w.E, w.hI, w.cI, w.k, p.d["qI"])
+    fws = torch.empty(nws, device="cuda", dtype=torch.uint8) if nws else None
+    fidx = torch.full_like(p.idx, -7)
+    abi.csa_indexer_topk(p.d["qI"][None], qs[None] if qs is not None else None, p.d["wI"][None],
+                         p.kI, p.q_pos[None], w.m, w.k, fidx, w.E, workspace=fws)
+    abi.csa_get_error()
+    del fws
+    nbad = int((fidx != p.idx).any(1).sum())
+    assert nbad == 0, "%d rows of csa_indexer_topk differ from the two calls" % nbad
     # second level, on the GPU's keys: the oracle's float64 selection over the
     # same keys differs only at the boundary, within the score error
     own_idx = oracle.topk(own.astype(np.float32).astype(np.float64), rows, w.m, w.k)
