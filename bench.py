@@ -6,7 +6,8 @@
                     [--no-cpu-baseline] [--n N] [--graph auto|on|off]
 
 One step = one pass of the whole path over one synthetic sequence (CSA:
-compress KV, compress indexer keys, indexer scores, top-k, sparse attention;
+compress KV, compress indexer keys, indexer scores and top-k in one call
+(csa_indexer_topk, which does not write the score rows), sparse attention;
 HCA: compress, dense attention; decode: indexer, top-k, sparse and HCA
 attention over a batch of long caches). The default workload is the largest
 prefill that fits one GPU: a 131072-token CSA prefill with an e4m3 indexer

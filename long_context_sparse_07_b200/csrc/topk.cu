@@ -1019,14 +1019,79 @@ topk_warp_kernel(const float *__restrict__ scores, int64_t rows, int64_t E, int6
 constexpr int kCandRows = 8;           // rows (warps) per block
 constexpr int kCandMaxLists = 8;
 
-struct CandWarp {
+constexpr int kCandBin = 512;          // keys of the threshold bin kept aside
+
+struct __align__(16) CandWarp {
     unsigned hist[256];
-    unsigned bin, need, bcnt, pad;
+    unsigned bin, need, bcnt, nb;
 };
 
+// Shared memory of one row: the digit histogram, the bitmap of chosen
+// indices, and an area that holds the threshold bin's pairs (or, on the
+// slow path, the bitmap of the keys equal to the threshold).
+// Bitmaps keep word w at w + w / 32, so that the runs of 32 words that the
+// lanes scan fall in different banks.
+__host__ __device__ inline int cand_padded(int words) { return (words + words / 32 + 4) & ~3; }
+__device__ __forceinline__ int bmw(uint32_t w) { return (int)(w + (w >> 5)); }
+__host__ __device__ inline size_t cand_aside_bytes(int words)
+{
+    const size_t a = (size_t)kCandBin * 8, b = (size_t)cand_padded(words) * 4;
+    return a > b ? a : b;
+}
+// (every part a multiple of 16 bytes: the histogram is read as 16-byte words)
 __host__ __device__ inline size_t cand_warp_bytes(int words)
 {
-    return sizeof(CandWarp) + (size_t)2 * words * 4;
+    static_assert(sizeof(CandWarp) % 16 == 0, "CandWarp must keep 16-byte alignment");
+    return sizeof(CandWarp) + (size_t)cand_padded(words) * 4 + cand_aside_bytes(words);
+}
+
+// Bin of the warp's 256-bin histogram (descending) where the count from the
+// top reaches `need`: g.bin, g.need (what is still needed inside it), g.bcnt.
+__device__ __forceinline__ void warp_find(CandWarp &g, unsigned need)
+{
+    // lane l owns bins 255 - 8 l down to 248 - 8 l, read as two 16-byte words
+    const int lane = threadIdx.x & 31;
+    const uint4 lo4 = *reinterpret_cast<const uint4 *>(g.hist + 248 - 8 * lane);
+    const uint4 hi4 = *reinterpret_cast<const uint4 *>(g.hist + 252 - 8 * lane);
+    const unsigned h[8] = {hi4.w, hi4.z, hi4.y, hi4.x, lo4.w, lo4.z, lo4.y, lo4.x};  // descending
+    unsigned local = 0;
+#pragma unroll
+    for (int j = 0; j < 8; j++)
+        local += h[j];
+    unsigned incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += y;
+    }
+    const unsigned ex = incl - local;
+    if (ex < need && need <= incl) {
+        unsigned cum = ex;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            if (cum < need && cum + h[j] >= need) {
+                g.bin = 255u - 8u * lane - j;
+                g.need = need - cum;
+                g.bcnt = h[j];
+            }
+            cum += h[j];
+        }
+    }
+    __syncwarp();
+}
+
+__device__ __forceinline__ unsigned warp_excl(unsigned v)
+{
+    const int lane = threadIdx.x & 31;
+    unsigned incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += y;
+    }
+    return incl - v;
 }
 
 __global__ void __launch_bounds__(32 * kCandRows)
@@ -1037,7 +1102,10 @@ topk_cand_kernel(const TopkCandArgs a, int words)
     uint8_t *gbase = cdyn + (size_t)wid * cand_warp_bytes(words);
     CandWarp &g = *reinterpret_cast<CandWarp *>(gbase);
     uint32_t *bm_gt = (uint32_t *)(gbase + sizeof(CandWarp));
-    uint32_t *bm_eq = bm_gt + words;
+    uint8_t *aside = (uint8_t *)(bm_gt + cand_padded(words));
+    uint32_t *akey = (uint32_t *)aside;                 // threshold bin: keys
+    uint32_t *aidx = akey + kCandBin;                   //                indices
+    uint32_t *bm_eq = (uint32_t *)aside;                // slow path: keys equal to T
     const int64_t row = (int64_t)blockIdx.x * kCandRows + wid;
     if (row >= a.rows)
         return;
@@ -1051,133 +1119,210 @@ topk_cand_kernel(const TopkCandArgs a, int words)
             a.flag[row] = 0;
         return;
     }
-    // 1. the lists: counts, prefixes (the same on every lane)
+    // 1. the lists: counts (the same on every lane)
     const int L = a.lists;
     const unsigned room = (unsigned)(a.E / 2 / L);
     const uint32_t *ccnt = a.cnt + row * L;
     const uint2 *crow = a.cand + row * a.cand_ld;
-    unsigned nx[kCandMaxLists];
     unsigned total = 0;
     bool over = false;
 #pragma unroll
     for (int x = 0; x < kCandMaxLists; x++) {
-        nx[x] = x < L ? ccnt[x] : 0u;
-        over |= nx[x] > room;
-        total += nx[x];
+        const unsigned n = x < L ? ccnt[x] : 0u;
+        over |= n > room;
+        total += n;
     }
     if (over || total < (unsigned)k) {
         if (lane == 0)
             a.flag[row] = 1;
         return;
     }
-    // f(pair) for every pair of every list, eight loads in flight per lane
+    // f(key, index, valid) for every pair of every list, eight loads in
+    // flight per lane
     auto each = [&](auto &&f) {
-#pragma unroll
-        for (int x = 0; x < kCandMaxLists; x++) {
+#pragma unroll 1
+        for (int x = 0; x < L; x++) {
             const uint2 *lp = crow + (int64_t)x * room;
-            for (unsigned f0 = 0; f0 < nx[x]; f0 += 256) {
+            const unsigned n = __ldg(ccnt + x);
+            for (unsigned f0 = 0; f0 < n; f0 += 256) {
                 uint2 p[8];
 #pragma unroll
                 for (int i = 0; i < 8; i++) {
                     const unsigned j = f0 + i * 32 + lane;
-                    p[i] = j < nx[x] ? lp[j] : make_uint2(0u, 0xffffffffu);
+                    p[i] = j < n ? lp[j] : make_uint2(0u, 0xffffffffu);
                 }
 #pragma unroll
                 for (int i = 0; i < 8; i++)
-                    f(p[i], f0 + i * 32 + lane < nx[x]);
+                    f(float_key(__uint_as_float(p[i].x)), p[i].y, f0 + i * 32 + lane < n);
             }
         }
     };
-    // 2. the k-th largest key T, and how many keys equal to T are taken
-    uint32_t prefix = 0, pmask = 0;
-    unsigned need = (unsigned)k, bcnt = 0;
-#pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    const int W = (int)((V + 31) / 32);
+    for (int w = lane; w < W; w += 32)
+        bm_gt[bmw(w)] = 0u;
+    // 2. smallest and largest key: the bits above their highest differing
+    // bit are common to every pair, so the first digit starts below them
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    each([&](uint32_t u, uint32_t, bool v) {
+        if (v) {
+            kmin = u < kmin ? u : kmin;
+            kmax = u > kmax ? u : kmax;
+        }
+    });
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    const int d = kmin == kmax ? 0 : 32 - __clz(kmin ^ kmax);   // differing low bits
+    const int shift = d > 8 ? d - 8 : 0;
+    // bits common to every key above the first digit [shift, shift + 8)
+    const uint32_t hi = shift + 8 >= 32 ? 0u : (kmin & ~((1u << (shift + 8)) - 1u));
+    // 3. histogram of the first digit, the bin b that holds the k-th largest
+    uint32_t T = kmin;
+    unsigned need = (unsigned)k, bcnt = total;
+    bool fast = true;
+    if (d > 0) {
         for (int b = lane; b < 256; b += 32)
             g.hist[b] = 0;
         __syncwarp();
-        each([&](const uint2 &p, bool valid) {
-            const uint32_t u = float_key(__uint_as_float(p.x));
-            hist_add(g.hist, (u >> shift) & 255u, valid && (u & pmask) == prefix);
+        // (keys spread over many bins here: one shared atomic per key)
+        each([&](uint32_t u, uint32_t, bool v) {
+            if (v)
+                atomicAdd(&g.hist[(u >> shift) & 255u], 1u);
         });
         __syncwarp();
-        {
-            // bin where the count from the top reaches `need`
-            unsigned local = 0;
-#pragma unroll
-            for (int j = 0; j < 8; j++)
-                local += g.hist[255 - 8 * lane - j];
-            unsigned incl = local;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o)
-                    incl += y;
-            }
-            const unsigned ex = incl - local;
-            if (ex < need && need <= incl) {
-                unsigned cum = ex;
-                for (int j = 0; j < 8; j++) {
-                    const unsigned hb = g.hist[255 - 8 * lane - j];
-                    if (cum + hb >= need) {
-                        g.bin = 255u - 8u * lane - j;
-                        g.need = need - cum;
-                        g.bcnt = hb;
-                        break;
-                    }
-                    cum += hb;
-                }
-            }
-        }
-        __syncwarp();
-        prefix |= g.bin << shift;
-        pmask |= 255u << shift;
+        warp_find(g, need);
+        const uint32_t bin = g.bin;
         need = g.need;
         bcnt = g.bcnt;
-        __syncwarp();                             // hist and the results reused
-    }
-    const uint32_t T = prefix;
-    // 3. bitmaps of the chosen indices: keys above T, and keys equal to T
-    // (straight into the first when all of them are taken)
-    const int W = (int)((V + 31) / 32);
-    for (int w = lane; w < W; w += 32) {
-        bm_gt[w] = 0u;
-        bm_eq[w] = 0u;
-    }
-    __syncwarp();
-    const bool cut = need < bcnt;
-    each([&](const uint2 &p, bool valid) {
-        const uint32_t s = p.y;
-        if (valid && (int64_t)s < V) {
-            const uint32_t u = float_key(__uint_as_float(p.x));
-            const uint32_t bit = 1u << (s & 31u);
-            if (u > T)
-                atomicOr(&bm_gt[s >> 5], bit);
-            else if (u == T)
-                atomicOr(cut ? &bm_eq[s >> 5] : &bm_gt[s >> 5], bit);
+        // 4. keys above bin b are chosen; the pairs of bin b are set aside
+        // (when they fit)
+        fast = bcnt <= (unsigned)kCandBin;
+        unsigned nb = 0;
+        each([&](uint32_t u, uint32_t s, bool v) {
+            const uint32_t dg = (u >> shift) & 255u;
+            if (v && dg > bin && (int64_t)s < V)
+                atomicOr(&bm_gt[bmw(s >> 5)], 1u << (s & 31u));
+            const bool in = v && dg == bin;
+            const unsigned bal = __ballot_sync(0xffffffffu, in);
+            const unsigned at = nb + (unsigned)__popc(bal & ((1u << lane) - 1u));
+            if (fast && in && at < (unsigned)kCandBin) {
+                akey[at] = u;
+                aidx[at] = s;
+            }
+            nb += (unsigned)__popc(bal);
+        });
+        __syncwarp();
+        if (fast) {
+            // 5. the digits below the first one, over the pairs set aside
+            // (they all agree on the bits from `shift` up)
+            uint32_t sp = 0u, sm = 0u;
+            for (int sh = shift - 8; sh > -8; sh -= 8) {
+                const int s0 = sh > 0 ? sh : 0;
+                const uint32_t dm = 255u >> (sh < 0 ? -sh : 0);
+                for (int b = lane; b < 256; b += 32)
+                    g.hist[b] = 0;
+                __syncwarp();
+                for (unsigned j = lane; j < bcnt; j += 32) {
+                    const uint32_t u = akey[j];
+                    if ((u & sm) == sp)
+                        atomicAdd(&g.hist[(u >> s0) & dm], 1u);
+                }
+                __syncwarp();
+                warp_find(g, need);
+                sp |= g.bin << s0;
+                sm |= dm << s0;
+                need = g.need;
+                __syncwarp();
+            }
+            T = hi | (bin << shift) | sp;
+            // 6. within the bin: keys above T chosen, keys equal to T by index
+            unsigned neq = 0;
+            for (unsigned j0 = 0; j0 < bcnt; j0 += 32) {
+                const unsigned j = j0 + lane;
+                neq += (unsigned)__popc(__ballot_sync(0xffffffffu, j < bcnt && akey[j] == T));
+            }
+            for (unsigned j0 = 0; j0 < bcnt; j0 += 32) {
+                const unsigned j = j0 + lane;
+                if (j < bcnt) {
+                    const uint32_t u = akey[j], s = aidx[j];
+                    bool take = u > T;
+                    if (u == T) {
+                        if (need >= neq) {
+                            take = true;
+                        } else {
+                            unsigned rank = 0;                  // equal keys at lower indices
+                            for (unsigned i = 0; i < bcnt; i++)
+                                rank += (akey[i] == T && aidx[i] < s) ? 1u : 0u;
+                            take = rank < need;
+                        }
+                    }
+                    if (take && (int64_t)s < V)
+                        atomicOr(&bm_gt[bmw(s >> 5)], 1u << (s & 31u));
+                }
+            }
+            __syncwarp();
         }
-    });
-    __syncwarp();
+    }
+    if (d == 0) {
+        // every pair has the same key: the k lowest indices
+        for (int w = lane; w < W; w += 32)
+            bm_eq[bmw(w)] = 0u;
+        __syncwarp();
+        each([&](uint32_t, uint32_t s, bool v) {
+            if (v && (int64_t)s < V)
+                atomicOr(&bm_eq[bmw(s >> 5)], 1u << (s & 31u));
+        });
+        __syncwarp();
+        fast = false;
+        need = (unsigned)k;
+        bcnt = total;
+        T = kmin;
+    } else if (!fast) {
+        // slow path (a threshold bin of more than kCandBin pairs): the
+        // digits below the first one over all the pairs of bin b, then the
+        // keys equal to T in a second bitmap
+        const uint32_t bin = g.bin;
+        uint32_t sp = 0u, sm = 0u;
+        for (int sh = shift - 8; sh > -8; sh -= 8) {
+            const int s0 = sh > 0 ? sh : 0;
+            const uint32_t dm = 255u >> (sh < 0 ? -sh : 0);
+            for (int b = lane; b < 256; b += 32)
+                g.hist[b] = 0;
+            __syncwarp();
+            each([&](uint32_t u, uint32_t, bool v) {
+                hist_add(g.hist, (u >> s0) & dm,
+                         v && ((u >> shift) & 255u) == bin && (u & sm) == sp);
+            });
+            __syncwarp();
+            warp_find(g, need);
+            sp |= g.bin << s0;
+            sm |= dm << s0;
+            need = g.need;
+            __syncwarp();
+        }
+        T = hi | (bin << shift) | sp;
+        for (int w = lane; w < W; w += 32)
+            bm_eq[bmw(w)] = 0u;
+        __syncwarp();
+        each([&](uint32_t u, uint32_t s, bool v) {
+            if (v && (int64_t)s < V) {
+                if (u > T && (u >> shift) == (T >> shift))   // above T inside bin b
+                    atomicOr(&bm_gt[bmw(s >> 5)], 1u << (s & 31u));
+                else if (u == T)
+                    atomicOr(&bm_eq[bmw(s >> 5)], 1u << (s & 31u));
+            }
+        });
+        __syncwarp();
+    }
     const int wper = (W + 31) / 32;
     const int w0 = lane * wper, w1 = w0 + wper < W ? w0 + wper : W;
-    auto warp_excl = [&](unsigned v) -> unsigned {
-        unsigned incl = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o)
-                incl += y;
-        }
-        return incl - v;
-    };
-    if (cut) {
+    if (!fast) {
         // the `need` lowest indices among the keys equal to T
         unsigned c = 0;
         for (int w = w0; w < w1; w++)
-            c += (unsigned)__popc(bm_eq[w]);
+            c += (unsigned)__popc(bm_eq[bmw(w)]);
         unsigned e = warp_excl(c);
         for (int w = w0; w < w1 && e < need; w++) {
-            uint32_t x = bm_eq[w];
+            uint32_t x = bm_eq[bmw(w)];
             const unsigned pc = (unsigned)__popc(x);
             if (e + pc > need) {
                 unsigned keep = need - e;
@@ -1189,19 +1334,19 @@ topk_cand_kernel(const TopkCandArgs a, int words)
                 }
                 x = y;
             }
-            bm_gt[w] |= x;
+            bm_gt[bmw(w)] |= x;
             e += (unsigned)__popc(x);
         }
         __syncwarp();
     }
-    // 4. the chosen indices in ascending order
+    // 7. the chosen indices in ascending order
     unsigned c = 0;
     for (int w = w0; w < w1; w++)
-        c += (unsigned)__popc(bm_gt[w]);
+        c += (unsigned)__popc(bm_gt[bmw(w)]);
     unsigned e = warp_excl(c);
     const unsigned tot = __reduce_add_sync(0xffffffffu, c);
     for (int w = w0; w < w1; w++) {
-        uint32_t x = bm_gt[w];
+        uint32_t x = bm_gt[bmw(w)];
         while (x) {
             const int b = __ffs(x) - 1;
             x &= x - 1u;

@@ -227,3 +227,22 @@ def test_fused_misleading_sample_is_recomputed():
     np.testing.assert_array_equal(got, two)
     qv, kv64, wv = _values(qI, qs, kI, ks, wI, B, E, cI)
     _check_rows(got, qv, kv64, wv, pos, m, k, _some(n_q, 397), "planted sample")
+
+
+def test_fused_few_distinct_scores():
+    # every key is one of 6 vectors, so a query's scores take at most 6
+    # values: the threshold value is shared by thousands of candidates (the
+    # select's path for a crowded threshold bin, cut among equal scores by
+    # index)
+    B, n_q, E, hI, cI, m, k = 1, 4800, 16384, 64, 128, 4, 1024
+    assert abi.csa_indexer_topk_launches(B, n_q, E, hI, cI, k, abi.CSA_E4M3) == 6
+    g = np.random.default_rng(41)
+    base = g.normal(0.0, 1.0, size=(6, cI))
+    kI = _e4m3(base[g.integers(0, 6, size=E)])
+    ks = torch.ones(E, dtype=torch.float32)
+    qI, qs, _, _, wI = _operands(B, n_q, E, hI, cI, "e4m3", 42)
+    pos = _spread(n_q, E, m, 10)
+    got, two = _run(qI, qs, kI, ks, wI, pos, m, k, E)
+    np.testing.assert_array_equal(got, two)
+    qv, kv, wv = _values(qI, qs, kI, ks, wI, B, E, cI)
+    _check_rows(got, qv, kv, wv, pos, m, k, _some(n_q, 397), "six key vectors")
