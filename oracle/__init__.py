@@ -60,6 +60,12 @@ def lib():
             L.oracle_e4m3_code.argtypes = [ctypes.c_double]
             L.oracle_quantize_e4m3.argtypes = [_d, _I64, _I, _I, _u8, _f]
             L.oracle_dequantize.argtypes = [_u8, _f, _I64, _I, _I, _d]
+            L.oracle_e2m1_value.restype = ctypes.c_double
+            L.oracle_e2m1_value.argtypes = [ctypes.c_uint8]
+            L.oracle_e2m1_code.restype = ctypes.c_uint8
+            L.oracle_e2m1_code.argtypes = [ctypes.c_double]
+            L.oracle_quantize_e2m1.argtypes = [_d, _I64, _I, _u8, _u8]
+            L.oracle_dequantize_e2m1.argtypes = [_u8, _u8, _I64, _I, _d]
             L.oracle_compress.argtypes = [_d, _d, _d, _d, _d, _d, _I64, _I, _I, _I, _d]
             L.oracle_indexer.argtypes = [_d, _d, _d, _i64, _I, _I64, _I64, _I, _I, _I, _d]
             L.oracle_topk.argtypes = [_d, _I64, _I64, _I64, _i64, _I, _I, _i32]
@@ -128,6 +134,38 @@ def dequantize(codes, scales, group: int) -> np.ndarray:
     cols = c.shape[-1]
     out = np.empty(c.shape, dtype=np.float64)
     lib().oracle_dequantize(_p(c, _u8), _p(s, _f), c.size // cols, cols, group, _p(out, _d))
+    return out
+
+
+def e2m1_value(code: int) -> float:
+    return float(lib().oracle_e2m1_value(int(code)))
+
+
+def e2m1_code(x: float) -> int:
+    return int(lib().oracle_e2m1_code(float(x)))
+
+
+def quantize_e2m1(x) -> Tuple[np.ndarray, np.ndarray]:
+    """FP4 indexer-key storage of rows x [..., cols] (cols % 32 == 0): packed
+    codes uint8 [..., cols / 2] (even channel in the low nibble) and block
+    exponents uint8 [..., cols / 32] (block scale 2^(e - 127))."""
+    a = f64(x)
+    cols = a.shape[-1]
+    rows = a.size // cols
+    packed = np.zeros(a.shape[:-1] + (cols // 2,), dtype=np.uint8)
+    exps = np.empty(a.shape[:-1] + (cols // 32,), dtype=np.uint8)
+    lib().oracle_quantize_e2m1(_p(a, _d), rows, cols, _p(packed, _u8), _p(exps, _u8))
+    return packed, exps
+
+
+def dequantize_e2m1(packed, exps) -> np.ndarray:
+    """Values [..., 2 * packed cols] of FP4 rows."""
+    c = _codes(packed)
+    e = _codes(exps)
+    cols = 2 * c.shape[-1]
+    out = np.empty(c.shape[:-1] + (cols,), dtype=np.float64)
+    lib().oracle_dequantize_e2m1(_p(c, _u8), _p(e, _u8), c.size // c.shape[-1], cols,
+                                 _p(out, _d))
     return out
 
 

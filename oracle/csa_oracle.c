@@ -17,7 +17,8 @@
  *   top-k selection ........ Module B step 2, Eq. 17
  *   shared-KV attention .... Module B step 3, Eq. 18-19, with the sliding
  *                            window branch and the attention sink of Module D
- *   low-precision storage .. Module F (fp8 body, bf16 RoPE dims)
+ *   low-precision storage .. Module F (fp8 body, bf16 RoPE dims; FP4
+ *                            indexer keys)
  * Readings where the pages are silent are listed beside each function.
  *
  * Every function takes inputs already decoded exactly to double and computes
@@ -118,6 +119,117 @@ void oracle_dequantize(const uint8_t *codes, const float *scales, int64_t rows,
         for (int j = 0; j < cols; j++)
             out[r * cols + j] = oracle_e4m3_value(codes[r * cols + j]) *
                                 (double)scales[r * groups + j / group];
+}
+
+/* ------------------------------------------------- fp4 indexer keys --- */
+
+/* Value of a 4-bit e2m1 code (1 sign bit, 2 exponent bits with bias 1, 1
+ * mantissa bit; no infinities or NaN): the FP4 of the indexer path (Module F:
+ * "the indexer's QK path runs in FP4"). Magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+double oracle_e2m1_value(uint8_t code)
+{
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, f = code & 1;
+    double v = e == 0 ? 0.5 * f : ldexp(1.0 + 0.5 * f, e - 1);
+    return s ? -v : v;
+}
+
+/* Nearest e2m1 code to x, ties to the code with the even (zero) mantissa
+ * bit, magnitudes beyond 6 saturate to 6; the sign bit is the sign of x. */
+uint8_t oracle_e2m1_code(double x)
+{
+    uint8_t sign = (x < 0 || (x == 0 && signbit(x))) ? 8 : 0;
+    double a = fabs(x);
+    if (a >= 6.0)
+        return sign | 7;
+    int lo = 0, hi = 7;                   /* magnitudes increase with code */
+    while (hi - lo > 1) {                 /* value(lo) <= a < value(hi) */
+        int mid = (lo + hi) / 2;
+        if (oracle_e2m1_value((uint8_t)mid) <= a)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    double dl = a - oracle_e2m1_value((uint8_t)lo);
+    double dh = oracle_e2m1_value((uint8_t)hi) - a;
+    int code = (dl < dh) ? lo : (dh < dl) ? hi : ((lo & 1) ? hi : lo);
+    return (uint8_t)(sign | code);
+}
+
+/* FP4 storage of indexer-key rows. Readings adopted for what the pages leave
+ * open (they name FP4 only):
+ *  - blocks of 32 consecutive channels share a power-of-two scale 2^E, the
+ *    smallest one with 6 * 2^E >= the block's largest magnitude (so no value
+ *    saturates), taken on the float32 values;
+ *  - within a row the block exponents span at most 8 binades (a block whose
+ *    exponent would be lower takes max_E - 8), so that a row can be brought
+ *    to one scale exactly in 8-bit floats;
+ *  - an all-zero block takes the row's lowest allowed exponent; an all-zero
+ *    row takes exponent 0;
+ *  - codes are the nearest e2m1 values of x / 2^E (float32 quotient).
+ * Layout: packed[r][j / 2] holds channel j in its low nibble when j is even,
+ * in its high nibble when odd; exps[r][b] = E_b + 127 (the block scale is
+ * 2^(exps - 127)). cols must be a multiple of 32. */
+void oracle_quantize_e2m1(const double *x, int64_t rows, int cols, uint8_t *packed,
+                          uint8_t *exps)
+{
+    int blocks = cols / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        int E[64];
+        int any = 0, emax = -100000;
+        for (int b = 0; b < blocks; b++) {
+            float amax = 0.0f;
+            for (int j = 0; j < 32; j++) {
+                float v = (float)x[r * cols + b * 32 + j];
+                if (fabsf(v) > amax)
+                    amax = fabsf(v);
+            }
+            if (amax > 0.0f) {
+                int e = -160;                       /* smallest e: 6 * 2^e >= amax */
+                while (ldexp(6.0, e) < (double)amax)
+                    e++;
+                while (ldexp(6.0, e - 1) >= (double)amax)
+                    e--;
+                E[b] = e;
+                any = 1;
+                if (e > emax)
+                    emax = e;
+            } else {
+                E[b] = -100000;
+            }
+        }
+        for (int b = 0; b < blocks; b++) {
+            int e = any ? (E[b] < emax - 8 ? emax - 8 : E[b]) : 0;
+            exps[r * blocks + b] = (uint8_t)(e + 127);
+            for (int j = 0; j < 32; j++) {
+                int ch = b * 32 + j;
+                float v = (float)x[r * cols + ch];
+                float y = ldexpf(v, -e);
+                uint8_t q = oracle_e2m1_code((double)y);
+                uint8_t *dst = &packed[r * (cols / 2) + ch / 2];
+                if (ch & 1)
+                    *dst = (uint8_t)((*dst & 0x0F) | (q << 4));
+                else
+                    *dst = (uint8_t)((*dst & 0xF0) | q);
+            }
+        }
+    }
+}
+
+/* Stored value of an FP4 key channel: its code's value times its block's
+ * scale 2^(exps - 127). */
+void oracle_dequantize_e2m1(const uint8_t *packed, const uint8_t *exps, int64_t rows, int cols,
+                            double *out)
+{
+    int blocks = cols / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++)
+        for (int j = 0; j < cols; j++) {
+            uint8_t byte = packed[r * (cols / 2) + j / 2];
+            uint8_t q = (j & 1) ? (byte >> 4) : (byte & 15);
+            out[r * cols + j] =
+                ldexp(oracle_e2m1_value(q), (int)exps[r * blocks + j / 32] - 127);
+        }
 }
 
 /* --------------------------------------------------------- compression --- */
