@@ -44,7 +44,9 @@ extern "C" {
 typedef enum {
     CSA_F32 = 0,   /* IEEE binary32 */
     CSA_BF16 = 1,  /* bfloat16 */
-    CSA_E4M3 = 2   /* 8-bit float e4m3 (finite, max 448), always with scales */
+    CSA_E4M3 = 2,  /* 8-bit float e4m3 (finite, max 448), always with scales */
+    CSA_E2M1 = 3   /* 4-bit float e2m1 (max 6), two per byte, with block scales
+                      (indexer keys only) */
 } csa_dtype;
 
 typedef enum {
@@ -67,6 +69,14 @@ typedef enum {
  *     body[r][j] is code * scale[r][j / scale_group]; when rope_dims > 0 the
  *     trailing rope_dims channels are stored unscaled as bfloat16 in rope
  *     [rows, rope_dims].
+ *   fp4 layout (indexer keys: Module F, "the indexer's QK path runs in FP4"):
+ *     dt = CSA_E2M1, scale_group = 32, rope_dims = 0, rope = NULL, c a
+ *     multiple of 32; body is [rows, c / 2] bytes, channel j in the low
+ *     nibble of byte j / 2 when j is even, in the high nibble when odd; the
+ *     `scale` pointer holds [rows, c / 32] uint8 block exponents (not
+ *     floats): the value of channel j is e2m1(code) * 2^(e[r][j / 32] - 127).
+ *     Within a row the exponents span at most 8 (max - min <= 8), which the
+ *     compressor guarantees; larger spans read wrong values.
  * The same struct describes inputs (read) and outputs (written); `body`,
  * `scale` and `rope` are cast to const by readers.
  */
@@ -107,7 +117,12 @@ const char *csa_last_message(void);
  *   out             [E, c] entries: plain F32/BF16, or the fp8 layout with
  *                   scale_group dividing c - rope_dims (per-group scale =
  *                   max(amax / 448, 2^-126), codes rounded to nearest even
- *                   and saturated; rope channels stored as bf16).
+ *                   and saturated; rope channels stored as bf16), or the fp4
+ *                   layout (indexer keys; c / 32 blocks per row, 32 / vector
+ *                   width lanes each: each block takes the smallest scale
+ *                   2^E with 6 * 2^E >= its largest magnitude, raised to the
+ *                   row's largest E - 8 when below it; an all-zero row takes
+ *                   E = 0; codes rounded to nearest even).
  * Requirements: c / 8 (bf16) or c / 4 (f32) a power of two of at most 256,
  *   1 <= m <= 1024,
  *   all buffers 16-byte aligned.
@@ -127,7 +142,10 @@ csa_status csa_compress_kv(const void *Ca, const void *Cb, const void *Za, const
  *             [B, n_q, hI] float32 > 0 (one scale per query head), else NULL.
  *   wI        [B, n_q, hI] float32 head weights.
  *   kI        keys, rows = B * E (batch b owns rows b*E .. b*E+E-1), c = cI;
- *             kI.dt must equal dt; for CSA_E4M3, scale_group == cI (one
+ *             kI.dt must equal dt, or be CSA_E2M1 (FP4 keys) with dt =
+ *             CSA_E4M3 (FP4 keys against e4m3 queries: the products are
+ *             exact in the 8-bit tensor-core path, FP4 saving half of the
+ *             key bytes); for CSA_E4M3, scale_group == cI (one
  *             positive scale per key) and rope_dims == 0.
  *   q_pos     [B, n_q] int64 query positions.
  *   m         compression ratio used for visibility.

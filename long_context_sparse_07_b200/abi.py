@@ -20,7 +20,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libcsa.so")
 
-CSA_F32, CSA_BF16, CSA_E4M3 = 0, 1, 2
+CSA_F32, CSA_BF16, CSA_E4M3, CSA_E2M1 = 0, 1, 2, 3
 STATUS = {0: "CSA_OK", -1: "CSA_ERR_INVALID_ARG", -2: "CSA_ERR_UNSUPPORTED",
           -3: "CSA_ERR_CUDA", -4: "CSA_ERR_TIMEOUT", -5: "CSA_ERR_BOUNDS"}
 
@@ -140,17 +140,21 @@ def _check(st: int):
 class Entries:
     """A table of KV entries (``csa_entries``): plain [rows, c] f32/bf16, or
     the fp8 layout (e4m3 body [rows, c - rope_dims] with per-group float32
-    scales, optional bf16 rope part [rows, rope_dims])."""
+    scales, optional bf16 rope part [rows, rope_dims]), or the fp4 layout of
+    indexer keys (fp4=True: uint8 body [rows, c / 2] of packed e2m1 codes,
+    uint8 block exponents [rows, c / 32] in ``scale``, scale_group 32)."""
     body: torch.Tensor
     c: int
     scale: Optional[torch.Tensor] = None
     rope: Optional[torch.Tensor] = None
     rope_dims: int = 0
     scale_group: int = 0
+    fp4: bool = False
 
     def struct(self) -> _Entries:
+        dt = CSA_E2M1 if self.fp4 else dtype_code(self.body)
         return _Entries(_ptr(self.body), _ptr(self.scale), _ptr(self.rope), self.c,
-                        self.rope_dims, self.scale_group, dtype_code(self.body))
+                        self.rope_dims, self.scale_group, dt)
 
 
 def csa_abi_version() -> int:

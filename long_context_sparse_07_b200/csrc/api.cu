@@ -57,11 +57,22 @@ csa_status launched(cudaError_t e, const char *what)
             return fail(st, __VA_ARGS__);                                                \
     } while (0)
 
-csa_status check_entries(const csa_entries &t, int c, bool allow_fp8, const char *what)
+csa_status check_entries(const csa_entries &t, int c, bool allow_fp8, const char *what,
+                         bool allow_fp4 = false)
 {
     REQUIRE(t.body, CSA_ERR_INVALID_ARG, "%s: body is NULL", what);
     REQUIRE(t.c == c, CSA_ERR_INVALID_ARG, "%s: c = %d, expected %d", what, t.c, c);
     REQUIRE(aligned16(t.body), CSA_ERR_INVALID_ARG, "%s: body not 16-byte aligned", what);
+    if (t.dt == CSA_E2M1) {
+        REQUIRE(allow_fp4, CSA_ERR_UNSUPPORTED, "%s: e2m1 entries are for indexer keys only",
+                what);
+        REQUIRE(c % 32 == 0, CSA_ERR_UNSUPPORTED, "%s: e2m1 entries need c %% 32 == 0", what);
+        REQUIRE(t.scale && ((uintptr_t)t.scale & 3u) == 0, CSA_ERR_INVALID_ARG,
+                "%s: e2m1 entries need 4-byte aligned block exponents in `scale`", what);
+        REQUIRE(t.scale_group == 32 && t.rope_dims == 0 && !t.rope, CSA_ERR_INVALID_ARG,
+                "%s: e2m1 entries need scale_group 32 and no rope part", what);
+        return CSA_OK;
+    }
     if (t.dt == CSA_E4M3) {
         REQUIRE(allow_fp8, CSA_ERR_UNSUPPORTED, "%s: e4m3 entries not supported here", what);
         REQUIRE(t.scale && aligned16(t.scale), CSA_ERR_INVALID_ARG,
@@ -133,7 +144,7 @@ csa_status csa_compress_kv(const void *Ca, const void *Cb, const void *Za, const
     REQUIRE(aligned16(Ca) && aligned16(Za) && aligned16(Ba) && (!overlap ||
             (aligned16(Cb) && aligned16(Zb) && aligned16(Bb))), CSA_ERR_INVALID_ARG,
             "%s: inputs must be 16-byte aligned", w);
-    csa_status st = check_entries(out, c, true, "csa_compress_kv(out)");
+    csa_status st = check_entries(out, c, true, "csa_compress_kv(out)", true);
     if (st != CSA_OK)
         return st;
     if (out.dt == CSA_E4M3) {
@@ -141,6 +152,9 @@ csa_status csa_compress_kv(const void *Ca, const void *Cb, const void *Za, const
                 out.scale_group / vec <= 32, CSA_ERR_UNSUPPORTED,
                 "%s: scale_group %d unsupported for this input dtype", w, out.scale_group);
     }
+    if (out.dt == CSA_E2M1)
+        REQUIRE(c / vec <= 32, CSA_ERR_UNSUPPORTED,
+                "%s: e2m1 output needs a row within one warp (c / %d <= 32)", w, vec);
     unsigned *err = err_word();
     REQUIRE(err, CSA_ERR_CUDA, "%s: no CUDA device", w);
     csa::CompressArgs a{Ca, Cb, Za, Zb, Ba, Bb, n, c, m, overlap ? 1 : 0, in_dt, out};
@@ -165,17 +179,18 @@ csa_status check_indexer(const char *w, const void *qI, const float *qI_scale, c
     REQUIRE(m >= 1, CSA_ERR_INVALID_ARG, "%s: m must be >= 1", w);
     REQUIRE(dt == CSA_F32 || dt == CSA_BF16 || dt == CSA_E4M3, CSA_ERR_INVALID_ARG,
             "%s: unknown dtype", w);
-    REQUIRE(kI.dt == dt, CSA_ERR_INVALID_ARG, "%s: kI dtype differs from qI dtype", w);
+    REQUIRE(kI.dt == dt || (kI.dt == CSA_E2M1 && dt == CSA_E4M3), CSA_ERR_INVALID_ARG,
+            "%s: kI dtype must equal the qI dtype (or be e2m1 with e4m3 queries)", w);
     char what[64];
     snprintf(what, sizeof what, "%s(kI)", w);
-    csa_status st = check_entries(kI, cI, true, what);
+    csa_status st = check_entries(kI, cI, true, what, true);
     if (st != CSA_OK)
         return st;
-    if (dt == CSA_E4M3) {
+    if (dt == CSA_E4M3)
         REQUIRE(qI_scale, CSA_ERR_INVALID_ARG, "%s: e4m3 queries need qI_scale", w);
+    if (kI.dt == CSA_E4M3)
         REQUIRE(kI.scale_group == cI && kI.rope_dims == 0, CSA_ERR_UNSUPPORTED,
                 "%s: e4m3 keys need one scale per key and no rope part", w);
-    }
     REQUIRE(aligned16(qI), CSA_ERR_INVALID_ARG, "%s: qI not 16-byte aligned", w);
     return CSA_OK;
 }

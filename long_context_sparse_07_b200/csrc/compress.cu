@@ -9,6 +9,7 @@
 // into `split` interleaved slices handled by different warps; the slices are
 // merged through shared memory with the usual max-rescaled combination.
 // Each row of Ca / Za / Cb / Zb is read exactly once from HBM.
+#include <cuda_fp4.h>
 #include <float.h>
 
 #include "common.cuh"
@@ -169,6 +170,48 @@ compress_kernel(const T *__restrict__ Ca, const T *__restrict__ Cb, const T *__r
     }
 
     const bool writer = live && slice == 0;
+    if (out.dt == CSA_E2M1) {
+        // fp4 indexer keys: per block of 32 channels (32 / VEC lanes) the
+        // smallest 2^E with 6 * 2^E >= the block's largest magnitude, raised
+        // to the row's largest E - 8 when below it (the row's lanes are the
+        // entry's tpe consecutive lanes); an all-zero row takes E = 0
+        float amax = 0.f;
+#pragma unroll
+        for (int v = 0; v < VEC; v++)
+            amax = fmaxf(amax, fabsf(res[v]));
+        const int glanes = 32 / VEC;
+        for (int off = 1; off < glanes; off <<= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        constexpr int kNone = -100000;
+        int e = kNone;
+        if (amax > 0.f) {
+            int x;
+            const float f = frexpf(amax, &x);       // amax = f 2^x, f in [0.5, 1)
+            e = f <= 0.75f ? x - 3 : x - 2;
+        }
+        int emax = e;
+        for (int off = glanes; off < tpe; off <<= 1)
+            emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, off));
+        if (!writer)
+            return;
+        e = emax == kNone ? 0 : max(e, emax - 8);
+        e = min(max(e, -127), 128);
+        uint32_t packed = 0;                          // channel ch + v at byte v / 2
+#pragma unroll
+        for (int v = 0; v < VEC; v += 2)
+            packed |= (uint32_t)(uint8_t)__nv_cvt_float2_to_fp4x2(
+                          make_float2(ldexpf(res[v], -e), ldexpf(res[v + 1], -e)), __NV_E2M1,
+                          cudaRoundNearest)
+                      << (4 * v);
+        uint8_t *dst = (uint8_t *)out.body + i * (c / 2) + ch / 2;
+        if (VEC == 8)
+            *reinterpret_cast<uint32_t *>(dst) = packed;
+        else
+            *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
+        if (ch % 32 == 0)
+            ((uint8_t *)out.scale)[i * (c / 32) + ch / 32] = (uint8_t)(e + 127);
+        return;
+    }
     if (out.dt == CSA_E4M3) {
         // group amax across the group's lanes (aligned, power-of-two lanes);
         // every thread takes part in the shuffles, only slice 0 writes.

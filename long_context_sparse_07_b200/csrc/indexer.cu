@@ -6,7 +6,11 @@
 // query tile is staged in turn. Key tiles past the causal bound of every
 // query of the tile are skipped; score entries s >= V_t are not written.
 // This path serves float32 operands and any shape; the tensor-core path in
-// indexer_tc.cu takes bf16 / e4m3 operands of the supported shapes.
+// indexer_tc.cu takes bf16 / e4m3 operands of the supported shapes. FP4 keys
+// (e2m1 codes with a power-of-two scale per 32 channels) are decoded here
+// to float.
+#include <cuda_fp4.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -34,9 +38,9 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 indexer_kernel(const T *__restrict__ qI, const float *__restrict__ qI_scale,
                const float *__restrict__ wI, const T *__restrict__ kI,
-               const float *__restrict__ kI_scale, const int64_t *__restrict__ q_pos,
-               int64_t n_q, int64_t E, int hI, int cI, int m, float *__restrict__ scores,
-               int64_t ld)
+               const float *__restrict__ kI_scale, const uint8_t *__restrict__ kI_exp,
+               const int64_t *__restrict__ q_pos, int64_t n_q, int64_t E, int hI, int cI, int m,
+               float *__restrict__ scores, int64_t ld)
 {
     extern __shared__ float sm[];
     float *ks = sm;                       // [TS][cI + 1]
@@ -70,9 +74,18 @@ indexer_kernel(const T *__restrict__ qI, const float *__restrict__ qI_scale,
         const int64_t s = s0 + r;
         float v = 0.f;
         if (s < E) {
-            v = ld_val<T>(kI, ((int64_t)b * E + s) * cI + x);
-            if (kI_scale)
-                v *= kI_scale[(int64_t)b * E + s];
+            const int64_t row = (int64_t)b * E + s;
+            if (kI_exp) {
+                // fp4 key: nibble x % 2 of byte x / 2, scaled by 2^(e - 127)
+                const uint8_t byte = ((const uint8_t *)kI)[row * (cI / 2) + x / 2];
+                const __half_raw h = __nv_cvt_fp4_to_halfraw(
+                    (__nv_fp4_storage_t)((x & 1) ? byte >> 4 : byte & 15), __NV_E2M1);
+                v = ldexpf(__half2float(__half(h)), (int)kI_exp[row * (cI / 32) + x / 32] - 127);
+            } else {
+                v = ld_val<T>(kI, row * cI + x);
+                if (kI_scale)
+                    v *= kI_scale[row];
+            }
         }
         ks[r * (cI + 1) + x] = v;
     }
@@ -143,21 +156,22 @@ cudaError_t launch_indexer(const IndexerArgs &a, unsigned *err, cudaStream_t s)
         attr_set = true;
     }
     const float *ksc = a.kI.dt == CSA_E4M3 ? a.kI.scale : nullptr;
+    const uint8_t *kex = a.kI.dt == CSA_E2M1 ? (const uint8_t *)a.kI.scale : nullptr;
     const float *qsc = a.dt == CSA_E4M3 ? a.qI_scale : nullptr;
     switch (a.dt) {
     case CSA_F32:
         indexer_kernel<float><<<grid, kThreads, smem, s>>>(
-            (const float *)a.qI, qsc, a.wI, (const float *)a.kI.body, ksc, a.q_pos, a.n_q, a.E,
+            (const float *)a.qI, qsc, a.wI, (const float *)a.kI.body, ksc, kex, a.q_pos, a.n_q, a.E,
             a.hI, a.cI, a.m, a.scores, a.ld);
         break;
     case CSA_BF16:
         indexer_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(
             (const __nv_bfloat16 *)a.qI, qsc, a.wI, (const __nv_bfloat16 *)a.kI.body, ksc,
-            a.q_pos, a.n_q, a.E, a.hI, a.cI, a.m, a.scores, a.ld);
+            kex, a.q_pos, a.n_q, a.E, a.hI, a.cI, a.m, a.scores, a.ld);
         break;
     case CSA_E4M3:
         indexer_kernel<uint8_t><<<grid, kThreads, smem, s>>>(
-            (const uint8_t *)a.qI, qsc, a.wI, (const uint8_t *)a.kI.body, ksc, a.q_pos, a.n_q,
+            (const uint8_t *)a.qI, qsc, a.wI, (const uint8_t *)a.kI.body, ksc, kex, a.q_pos, a.n_q,
             a.E, a.hI, a.cI, a.m, a.scores, a.ld);
         break;
     }

@@ -27,6 +27,16 @@
 // (the causal triangle makes the last tokens' rows the longest). Every wait
 // is bounded; on expiry the block records CSA_ERR_TIMEOUT, drains its own
 // copies and returns.
+//
+// FP4 keys (K4; e2m1 codes with a power-of-two scale 2^(e - 127) per 32
+// channels, against e4m3 queries): the key tiles arrive packed (64 bytes per
+// key) in a ring of their own, and added warps turn each key into e4m3 codes
+// in the swizzled layout the MMA reads: channel value e2m1 * 2^-(emax - e)
+// (e4m3 holds every such value exactly for emax - e <= 8), the key's largest
+// block scale 2^(emax - 127) being applied in the epilogue like an e4m3
+// key's scale. The products are then exact in the e4m3 MMA.
+#include <cuda_fp4.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -46,6 +56,8 @@ struct TcArgs {
     float *scores;
     int64_t ld;
     int64_t ks_stride;    // key s has its scale at kI_scale[s * ks_stride]
+                          // (FP4: its 4 block exponents at kI_exp[4 * s * ks_stride])
+    const uint8_t *kI_exp;
     const int *row_flag;  // when set: blocks none of whose tokens is flagged exit
     // candidate mode (FUSE): every visible key of row r scoring at or above
     // bound[r] is kept as a (score bits, index) pair in cand; rows of at most
@@ -59,7 +71,7 @@ struct TcArgs {
     unsigned *err;
 };
 
-template <bool FP8, int HI, int NT, int NSUB>
+template <bool FP8, int HI, int NT, int NSUB, bool K4 = false>
 struct Cfg {
     static constexpr int N = NT * HI;          // columns of one accumulator
     static constexpr int TT = NT * NSUB;       // tokens of a block
@@ -74,14 +86,20 @@ struct Cfg {
     static constexpr int TPW = NT / SPLIT;
     static constexpr int CW = HI < 32 ? HI : 32;
     static constexpr int CPT = HI / CW;
-    static constexpr int THREADS = 32 * (2 + 4 * NSET * SPLIT);
-    static constexpr int STAGES = FP8 ? (NSUB > 1 ? 4 : 6) : 4;
+    static constexpr int NE = 4 * NSET * SPLIT;         // epilogue warps
+    static constexpr int UW = K4 ? (NT == 1 ? 4 : 2) : 0;  // FP4 unpack warps
+    static constexpr int THREADS = 32 * (2 + NE + UW);
+    // FP4 keys (c_I = 128): a 16 KB e4m3 stage and an 8 KB packed stage each
+    static constexpr int K4_STAGES_FIT =
+        (227 * 1024 - 2048 - QROWS * 128 - QROWS * 4 - TT * 16 - 256) / (16384 + 8192);
+    static constexpr int STAGES =
+        K4 ? (K4_STAGES_FIT > 6 ? 6 : K4_STAGES_FIT) : (FP8 ? (NSUB > 1 ? 4 : 6) : 4);
     static constexpr int TMEM_COLS = (2 * N) < 32 ? 32 : 2 * N;
     static constexpr uint32_t IDESC = FP8 ? tc::idesc_e4m3(128, N) : tc::idesc_bf16(128, N);
     static size_t smem_bytes(int kb)
     {
-        return 1024 + (size_t)kb * QROWS * 128 + (size_t)STAGES * kb * 16384 + 256 + QROWS * 4 +
-               TT * 16;
+        return 1024 + (size_t)kb * QROWS * 128 + (size_t)STAGES * kb * 16384 +
+               (K4 ? (size_t)STAGES * 8192 : 0) + 256 + QROWS * 4 + TT * 16;
     }
 };
 
@@ -105,12 +123,12 @@ __device__ __forceinline__ float relu_dot(const uint32_t *x, const float *w)
     return acc0.x + acc0.y;
 }
 
-template <bool FP8, int HI, int NT, int NSUB, bool FUSE>
-__global__ void __launch_bounds__(Cfg<FP8, HI, NT, NSUB>::THREADS, 1)
+template <bool FP8, int HI, int NT, int NSUB, bool FUSE, bool K4>
+__global__ void __launch_bounds__(Cfg<FP8, HI, NT, NSUB, K4>::THREADS, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmq,
                   const TcArgs a)
 {
-    using C = Cfg<FP8, HI, NT, NSUB>;
+    using C = Cfg<FP8, HI, NT, NSUB, K4>;
     constexpr int N = C::N;
     constexpr int TT = C::TT;
     constexpr int S = C::STAGES;
@@ -119,10 +137,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     const int KB = a.kb;
     uint8_t *sB = smem;
     uint8_t *sA = sB + (size_t)KB * C::QROWS * 128;
-    uint64_t *bars = (uint64_t *)(sA + (size_t)S * KB * 16384);
+    uint8_t *sR = sA + (size_t)S * KB * 16384;               // K4: packed key tiles
+    uint64_t *bars = (uint64_t *)(sR + (K4 ? (size_t)S * 8192 : 0));
     uint64_t *full = bars, *empty = bars + S, *bfull = bars + 2 * S;
     uint64_t *accf = bfull + 1, *acce = accf + 2, *done = acce + 2;
-    uint32_t *tmem_slot = (uint32_t *)(done + 1);
+    uint64_t *rfull = bars + 18, *rempty = bars + 24;          // K4 (S <= 6)
+    uint32_t *tmem_slot = (uint32_t *)(bars + 30);
     int *abort_flag = (int *)(tmem_slot + 1);
     float *wsm = (float *)(bars + 32);
     int64_t *vt = (int64_t *)(wsm + C::QROWS);
@@ -160,8 +180,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 
     if (warp == 0 && lane == 0) {
         for (int i = 0; i < S; i++) {
-            tc::mbar_init(&full[i], 1);
+            tc::mbar_init(&full[i], K4 ? C::UW : 1);
             tc::mbar_init(&empty[i], 1);
+            if (K4) {
+                tc::mbar_init(&rfull[i], 1);
+                tc::mbar_init(&rempty[i], C::UW);
+            }
         }
         tc::mbar_init(bfull, 1);
         for (int i = 0; i < 2; i++) {
@@ -177,8 +201,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
         tc::tmem_relinquish();
     }
-    if (warp >= 2) {
-        for (int col = threadIdx.x - 64; col < C::QROWS; col += C::THREADS - 64) {
+    if (warp >= 2 && warp < 2 + C::NE) {
+        for (int col = threadIdx.x - 64; col < C::QROWS; col += 32 * C::NE) {
             const int tt = col / HI, hh = col % HI;
             const int64_t t = t0 + tt;
             float wv = 0.f;
@@ -193,7 +217,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         if constexpr (FUSE) {
             // each token's bound (NaN: the row keeps nothing here, all of its
             // visible keys being the selection)
-            for (int tt = threadIdx.x - 64; tt < TT; tt += C::THREADS - 64) {
+            for (int tt = threadIdx.x - 64; tt < TT; tt += 32 * C::NE) {
                 const int64_t t = t0 + tt;
                 lbound[tt] = t < a.n_q && vt[tt] > a.k ? a.bound[(int64_t)b * a.n_q + t]
                                                         : __int_as_float(0x7fc00000);
@@ -217,16 +241,25 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 for (int r0 = 0; r0 < C::QROWS; r0 += QBOX)
                     tc::tma_load_2d(sB + ((size_t)kb * C::QROWS + r0) * 128, &tmq, bfull,
                                     kb * xstep, (int)(((int64_t)b * a.n_q + t0) * HI + r0));
+            // K4: the packed tiles go to their own ring, freed by the unpack
+            // warps; otherwise the e4m3 / bf16 tiles straight to the MMA ring
+            uint64_t *lfull = K4 ? rfull : full, *lempty = K4 ? rempty : empty;
             for (int i = 0; i < ntiles && ok; i++) {
                 const int st = i % S;
-                if (i >= S && !tc::mbar_wait(&empty[st], ((i / S) - 1) & 1, abort_flag)) {
+                if (i >= S && !tc::mbar_wait(&lempty[st], ((i / S) - 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                tc::mbar_arrive_expect_tx(&full[st], (uint32_t)(KB * 16384));
-                for (int kb = 0; kb < KB; kb++)
-                    tc::tma_load_2d(sA + (size_t)(st * KB + kb) * 16384, &tmk, &full[st],
-                                    kb * xstep, (int)((int64_t)b * a.E + s_begin + (int64_t)i * 128));
+                const int row0 = (int)((int64_t)b * a.E + s_begin + (int64_t)i * 128);
+                if constexpr (K4) {
+                    tc::mbar_arrive_expect_tx(&rfull[st], 8192u);
+                    tc::tma_load_2d(sR + (size_t)st * 8192, &tmk, &rfull[st], 0, row0);
+                } else {
+                    tc::mbar_arrive_expect_tx(&full[st], (uint32_t)(KB * 16384));
+                    for (int kb = 0; kb < KB; kb++)
+                        tc::tma_load_2d(sA + (size_t)(st * KB + kb) * 16384, &tmk, &full[st],
+                                        kb * xstep, row0);
+                }
                 issued = i + 1;
             }
             if (!ok) {
@@ -236,7 +269,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 volatile int never = 0;
                 static_cast<void>(tc::mbar_wait(bfull, 0, &never, 200000000ull));
                 for (int i = issued - S < 0 ? 0 : issued - S; i < issued; i++)
-                    static_cast<void>(tc::mbar_wait(&full[i % S], (i / S) & 1, &never, 200000000ull));
+                    static_cast<void>(tc::mbar_wait(&lfull[i % S], (i / S) & 1, &never, 200000000ull));
             }
         }
     } else if (warp == 1) {
@@ -287,7 +320,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             volatile int never = 0;
             static_cast<void>(tc::mbar_wait(done, 0, &never, 200000000ull));
         }
-    } else {
+    } else if (warp < 2 + C::NE) {
         // ---------------- epilogue: warps 2..; set = which TMEM buffer (with
         // two sets), lane quarter = warp % 4; in each token group, tokens
         // part * TPW .. part * TPW + TPW - 1
@@ -330,8 +363,19 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             const int64_t s = s_begin + (int64_t)i * 128 + row;
             // the key's scale is requested before the wait for its accumulator
             float ks = 1.f;
-            if (FP8)
+            if constexpr (K4) {
+                // the key's largest block scale, 2^(emax - 127)
+                ks = 0.f;
+                if (s < a.E) {
+                    const uint32_t ex =
+                        __ldg((const uint32_t *)a.kI_exp + ((int64_t)b * a.E + s) * a.ks_stride);
+                    const uint32_t em = max(max(ex & 255u, (ex >> 8) & 255u),
+                                            max((ex >> 16) & 255u, ex >> 24));
+                    ks = em ? __uint_as_float(em << 23) : __uint_as_float(1u << 22);
+                }
+            } else if (FP8) {
                 ks = s < a.E ? __ldg(a.kI_scale + ((int64_t)b * a.E + s) * a.ks_stride) : 0.f;
+            }
             auto group = [&](const int j) {
                 const int g = i * NSUB + j, buf = g & 1;
                 if (C::NSET == 2 && buf != set)
@@ -416,6 +460,72 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     }
             }
         }
+    } else if constexpr (K4) {
+        // ---------------- FP4 unpack warps: packed key rows -> e4m3 rows in
+        // the 128-byte swizzled layout of the MMA's A tile
+        const int uw = warp - 2 - C::NE;
+        bool ok = true;
+        for (int i = 0; i < ntiles && ok; i++) {
+            const int st = i % S;
+            if (!tc::mbar_wait(&rfull[st], (i / S) & 1, abort_flag) ||
+                (i >= S && !tc::mbar_wait(&empty[st], ((i / S) - 1) & 1, abort_flag))) {
+                *abort_flag = 1;
+                report(a.err, CSA_ERR_TIMEOUT, K_INDEXER_TC, blockIdx.x, 3);
+                ok = false;
+                break;
+            }
+            for (int r = uw * 32 + lane; r < 128; r += 32 * C::UW) {
+                const int64_t s = s_begin + (int64_t)i * 128 + r;
+                // rows past the table (zero-filled) take j = 0
+                uint32_t ex = 0x7f7f7f7fu;
+                if (s < a.E)
+                    ex = __ldg((const uint32_t *)a.kI_exp + ((int64_t)b * a.E + s) * a.ks_stride);
+                const uint32_t em = max(max(ex & 255u, (ex >> 8) & 255u),
+                                        max((ex >> 16) & 255u, ex >> 24));
+                const uint8_t *src = sR + (size_t)st * 8192 + r * 64;
+                uint8_t *dst = sA + (size_t)st * 16384 + r * 128;
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                    const int blk = (q + (r >> 1)) & 3;           // spreads the banks
+                    const uint4 w = *(const uint4 *)(src + blk * 16);
+                    int j = (int)(em - ((ex >> (8 * blk)) & 255u));
+                    j = j > 8 ? 8 : j;
+                    const __half2 sc = __float2half2_rn(__uint_as_float((uint32_t)(127 - j) << 23));
+                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int u = 0; u < 4; u++) {
+                        uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+                        for (int bb = 0; bb < 4; bb++) {
+                            const __half2_raw hr = __nv_cvt_fp4x2_to_halfraw2(
+                                (__nv_fp4x2_storage_t)((wv[u] >> (8 * bb)) & 255u), __NV_E2M1);
+                            const __half2 hv = __hmul2(__half2(hr), sc);
+                            const uint32_t e8 = (uint32_t)__nv_cvt_halfraw2_to_fp8x2(
+                                __half2_raw(hv), __NV_SATFINITE, __NV_E4M3);
+                            if (bb < 2)
+                                lo |= e8 << (16 * bb);
+                            else
+                                hi |= e8 << (16 * (bb - 2));
+                        }
+                        o[2 * u] = lo;
+                        o[2 * u + 1] = hi;
+                    }
+                    // channels 32 blk .. 32 blk + 31: 16-byte chunks 2 blk and
+                    // 2 blk + 1 of the row, at chunk ^ (row % 8)
+                    *(uint4 *)(dst + (((2 * blk) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *(uint4 *)(dst + (((2 * blk + 1) ^ (r & 7)) << 4)) =
+                        make_uint4(o[4], o[5], o[6], o[7]);
+                }
+            }
+            // the tile's generic writes become visible to the tensor core
+            tc::fence_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(&full[st]);
+                tc::mbar_arrive(&rempty[st]);
+            }
+        }
     }
     tc::fence_before();
     __syncthreads();
@@ -425,15 +535,16 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     }
 }
 
-template <bool FP8, int HI, int NT, int NSUB, bool FUSE>
+template <bool FP8, int HI, int NT, int NSUB, bool FUSE, bool K4>
 cudaError_t launch_one(const IndexerArgs &a, const IndexerTcExtra &x, unsigned *err, cudaStream_t s)
 {
-    using C = Cfg<FP8, HI, NT, NSUB>;
+    using C = Cfg<FP8, HI, NT, NSUB, K4>;
     const int esize = FP8 ? 1 : 2;
     TcArgs t;
     t.wI = a.wI;
     t.qI_scale = a.qI_scale;
-    t.kI_scale = a.kI.scale;
+    t.kI_scale = K4 ? nullptr : a.kI.scale;
+    t.kI_exp = K4 ? (const uint8_t *)a.kI.scale : nullptr;
     t.q_pos = a.q_pos;
     t.n_q = a.n_q;
     t.E = a.E;
@@ -476,19 +587,22 @@ cudaError_t launch_one(const IndexerArgs &a, const IndexerTcExtra &x, unsigned *
     CUtensorMap tmk, tmq;
     const CUtensorMapDataType dt =
         FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    // key s of the table is row s * key_step of kI.body
-    if (!make_tmap_2d(&tmk, a.kI.body, dt, esize, (uint64_t)a.B * a.E, a.cI, 128,
-                      (uint64_t)x.key_step * a.cI * esize) ||
-        !make_tmap_2d(&tmq, a.qI, dt, esize, (uint64_t)a.B * a.n_q * HI, a.cI,
-                      C::QROWS < 256 ? C::QROWS : 256))
+    // key s of the table is row s * key_step of kI.body (FP4: packed rows
+    // of c_I / 2 bytes, unswizzled)
+    const bool km = K4 ? make_tmap_bytes(&tmk, a.kI.body, (uint64_t)a.B * a.E, (uint64_t)a.cI / 2,
+                                         (uint64_t)x.key_step * a.cI / 2, 128, a.cI / 2)
+                       : make_tmap_2d(&tmk, a.kI.body, dt, esize, (uint64_t)a.B * a.E, a.cI, 128,
+                                      (uint64_t)x.key_step * a.cI * esize);
+    if (!km || !make_tmap_2d(&tmq, a.qI, dt, esize, (uint64_t)a.B * a.n_q * HI, a.cI,
+                             C::QROWS < 256 ? C::QROWS : 256))
         return cudaErrorInvalidValue;
     const size_t smem = C::smem_bytes(t.kb);
-    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<FP8, HI, NT, NSUB, FUSE>,
+    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<FP8, HI, NT, NSUB, FUSE, K4>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
     dim3 grid((unsigned)(ttiles * t.nchunks), (unsigned)a.B);
-    indexer_tc_kernel<FP8, HI, NT, NSUB, FUSE><<<grid, C::THREADS, smem, s>>>(tmk, tmq, t);
+    indexer_tc_kernel<FP8, HI, NT, NSUB, FUSE, K4><<<grid, C::THREADS, smem, s>>>(tmk, tmq, t);
     return cudaGetLastError();
 }
 
@@ -496,8 +610,13 @@ template <bool FP8, int HI, int NT, int NSUB>
 cudaError_t launch_mode(const IndexerArgs &a, const IndexerTcExtra &x, unsigned *err,
                         cudaStream_t s)
 {
-    return x.fuse ? launch_one<FP8, HI, NT, NSUB, true>(a, x, err, s)
-                  : launch_one<FP8, HI, NT, NSUB, false>(a, x, err, s);
+    if constexpr (FP8) {
+        if (a.kI.dt == CSA_E2M1)
+            return x.fuse ? launch_one<FP8, HI, NT, NSUB, true, true>(a, x, err, s)
+                          : launch_one<FP8, HI, NT, NSUB, false, true>(a, x, err, s);
+    }
+    return x.fuse ? launch_one<FP8, HI, NT, NSUB, true, false>(a, x, err, s)
+                  : launch_one<FP8, HI, NT, NSUB, false, false>(a, x, err, s);
 }
 
 template <bool FP8>
@@ -533,6 +652,9 @@ cudaError_t dispatch_heads(const IndexerArgs &a, const IndexerTcExtra &x, unsign
 bool indexer_tc_takes(const IndexerArgs &a)
 {
     if (a.dt == CSA_F32)
+        return false;
+    // FP4 keys: e4m3 queries, c_I = 128 (64-byte packed rows)
+    if (a.kI.dt == CSA_E2M1 && (a.dt != CSA_E4M3 || a.cI != 128))
         return false;
     if (a.hI != 16 && a.hI != 32 && a.hI != 64)
         return false;

@@ -43,4 +43,22 @@ inline bool make_tmap_2d(CUtensorMap *m, const void *base, CUtensorMapDataType d
     return r == CUDA_SUCCESS;
 }
 
+// Row-major [rows, row_bytes] bytes (rows `stride` bytes apart) read in
+// unswizzled boxes of box_rows x box_bytes; out-of-range rows read as zero.
+inline bool make_tmap_bytes(CUtensorMap *m, const void *base, uint64_t rows, uint64_t row_bytes,
+                            uint64_t stride, uint32_t box_rows, uint32_t box_bytes)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)stride};
+    cuuint32_t box[2] = {box_bytes, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace csa
