@@ -438,6 +438,86 @@ def time_out_proj(p, w, pk, stream, steps=3, g=8, dg=1024, d=4096):
             "shape": {"n": n, "h": w.h, "c": w.c, "g": g, "dg": dg, "d": d}}
 
 
+def _fp4_keys(rows, cI, seed):
+    """Random FP4 indexer keys on the device: packed e2m1 codes and block
+    exponents within a span of 8."""
+    from long_context_sparse_07_b200.abi import Entries
+    gen = torch.Generator(device="cuda").manual_seed(seed)
+    body = torch.randint(0, 256, (rows, cI // 2), device="cuda", dtype=torch.uint8, generator=gen)
+    exps = torch.randint(118, 127, (rows, cI // 32), device="cuda", dtype=torch.uint8,
+                         generator=gen)
+    return Entries(body, cI, scale=exps, scale_group=32, fp4=True)
+
+
+def _event_ms(f, stream, flush, steps):
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        f()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return sum(ts) / len(ts)
+
+
+def time_fp4_prefill(p, w, pk, stream, flush, steps=3):
+    """The step's indexer and top-k in one call with FP4 keys (random codes
+    of the same shape) in place of its e4m3 keys, L2 flushed in between."""
+    from long_context_sparse_07_b200 import abi
+    kI = _fp4_keys(w.E, w.cI, 11)
+    d = p.d
+    qs = d.get("qI_scale")
+    f = lambda: abi.csa_indexer_topk(d["qI"][None], qs[None], d["wI"][None], kI, p.q_pos[None],
+                                     w.m, w.k, p.idx, w.E, workspace=p.fused_ws)
+    f()
+    torch.cuda.synchronize()
+    ms = _event_ms(f, stream, flush, steps)
+    abi.csa_get_error()
+    fl = work.csa_prefill(w)["indexer_topk"]["flops"]
+    return {"ms": ms, "flops": fl, "achieved": fl / (ms * 1e-3) / 1e12, "peak": pk["fp8"],
+            "unit": "TFLOP/s", "frac": fl / (ms * 1e-3) / 1e12 / pk["fp8"],
+            "keys": "e2m1 + one power-of-two scale per 32 channels (68 bytes per key)"}
+
+
+def time_fp4_decode(pk, stream, flush, steps=20):
+    """Decode indexer over FP4 keys against the same call over e4m3 keys, on
+    the decode workload's queries and cache length (HBM-bound: the keys are
+    most of the bytes)."""
+    from long_context_sparse_07_b200 import abi
+    w = W.WORKLOADS["decode_b8_ctx1m"]
+    B, E, sd = w.batch, w.n // w.m, w.seed
+    # the decode workload's queries (the same generators and seeds)
+    qI = W.e4m3_codes(sd, "qI", B, w.hI * w.cI).view(B, 1, w.hI, w.cI).cuda()
+    qs = W.e4m3_scales(sd, "qI_scale", B, w.hI, w.std_q).view(B, 1, w.hI).cuda()
+    wI = W.to_storage(W.normal(sd, "wI", B, w.hI, w.std_w), "f32").view(B, 1, w.hI).cuda()
+    q_pos = torch.full((B, 1), w.n - 1, dtype=torch.int64, device="cuda")
+    scores = torch.empty(B, 1, E, device="cuda")
+    res = {}
+    for name, kI, kbytes in (("e4m3", None, w.cI + 4), ("e2m1", _fp4_keys(B * E, w.cI, 12),
+                                                         w.cI // 2 + w.cI // 32)):
+        if kI is None:
+            from long_context_sparse_07_b200.abi import Entries
+            body = torch.randint(-100, 100, (B * E, w.cI), device="cuda",
+                                 dtype=torch.int8).view(torch.float8_e4m3fn)
+            sc = torch.rand(B * E, device="cuda") + 0.5
+            kI = Entries(body, w.cI, scale=sc, scale_group=w.cI)
+        f = lambda: abi.csa_indexer_scores(qI, qs, wI, kI, q_pos, w.m, scores, E)
+        f()
+        torch.cuda.synchronize()
+        ms = _event_ms(f, stream, flush, steps)
+        by = B * E * kbytes + B * w.hI * (w.cI + 8) + B * E * 4
+        res[name] = {"ms": ms, "bytes": by, "achieved": by / (ms * 1e-3) / 1e9,
+                     "peak": pk["hbm"], "unit": "GB/s", "frac": by / (ms * 1e-3) / 1e9 / pk["hbm"],
+                     "key_bytes": kbytes}
+        del kI
+    abi.csa_get_error()
+    res["speedup"] = res["e4m3"]["ms"] / res["e2m1"]["ms"]
+    return res
+
+
 # --------------------------------------------------------------------------- CPU oracle
 
 
@@ -622,6 +702,9 @@ def run_ours(args, w):
         extras["norm_rope"] = time_norm_rope(p, w, pk, stream)
         if w.dtype == "bf16" and w.h % 8 == 0:
             extras["grouped_out_proj"] = time_out_proj(p, w, pk, stream)
+        if w.idx_dtype == "e4m3" and w.cI == 128 and p.fused:
+            extras["fp4_keys_prefill"] = time_fp4_prefill(p, w, pk, stream, flush)
+        extras["fp4_keys_decode"] = time_fp4_decode(pk, stream, flush)
 
     dom = summ["dominant"]
     roof = dict(summ["kernels"][dom])

@@ -87,11 +87,13 @@ struct Cfg {
     static constexpr int CW = HI < 32 ? HI : 32;
     static constexpr int CPT = HI / CW;
     static constexpr int NE = 4 * NSET * SPLIT;         // epilogue warps
-    static constexpr int UW = K4 ? (NT == 1 ? 4 : 2) : 0;  // FP4 unpack warps
+    static constexpr int UW = K4 ? (NT == 1 ? 8 : 2) : 0;  // FP4 unpack warps
     static constexpr int THREADS = 32 * (2 + NE + UW);
-    // FP4 keys (c_I = 128): a 16 KB e4m3 stage and an 8 KB packed stage each
+    // FP4 keys (c_I = 128): a 16 KB e4m3 stage and an 8 KB packed stage each;
+    // one-token blocks (decode) are sized for two blocks per SM
+    static constexpr int K4_BUDGET = NT == 1 ? 113 * 1024 : 227 * 1024;
     static constexpr int K4_STAGES_FIT =
-        (227 * 1024 - 2048 - QROWS * 128 - QROWS * 4 - TT * 16 - 256) / (16384 + 8192);
+        (K4_BUDGET - 2048 - QROWS * 128 - QROWS * 4 - TT * 16 - 256 - 128) / (16384 + 8192);
     static constexpr int STAGES =
         K4 ? (K4_STAGES_FIT > 6 ? 6 : K4_STAGES_FIT) : (FP8 ? (NSUB > 1 ? 4 : 6) : 4);
     static constexpr int TMEM_COLS = (2 * N) < 32 ? 32 : 2 * N;
@@ -99,9 +101,19 @@ struct Cfg {
     static size_t smem_bytes(int kb)
     {
         return 1024 + (size_t)kb * QROWS * 128 + (size_t)STAGES * kb * 16384 +
-               (K4 ? (size_t)STAGES * 8192 : 0) + 256 + QROWS * 4 + TT * 16;
+               (K4 ? (size_t)STAGES * 8192 + 128 : 0) + 256 + QROWS * 4 + TT * 16;
     }
 };
+
+// Byte permute (default mode): byte n of the result is byte (c >> 4n) & 7 of
+// {b, a} (a = bytes 0-3); with bit 3 of that selector set, the selected
+// byte's top bit is replicated over the result byte.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
 
 // sum_h w[h] * max(x[h], 0) over HI heads (x: raw TMEM words), two heads per
 // packed fp32 FMA, two independent accumulator pairs.
@@ -147,6 +159,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     float *wsm = (float *)(bars + 32);
     int64_t *vt = (int64_t *)(wsm + C::QROWS);
     float *lbound = (float *)(vt + TT);            // FUSE: per token
+    // K4: e4m3 byte of each e2m1 magnitude times 2^-j, j = 0..8 (2 words each)
+    uint32_t *lut = (uint32_t *)((uint8_t *)vt + TT * 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.y;
@@ -462,11 +476,52 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         }
     } else if constexpr (K4) {
         // ---------------- FP4 unpack warps: packed key rows -> e4m3 rows in
-        // the 128-byte swizzled layout of the MMA's A tile
+        // the 128-byte swizzled layout of the MMA's A tile. A block's 32
+        // channels share one j = emax - e; the e4m3 bytes of the 8 e2m1
+        // magnitudes times 2^-j come from a table of two words selected with
+        // byte permutes, the sign bits are moved in with a second permute.
         const int uw = warp - 2 - C::NE;
+        if (uw == 0 && lane < 9) {
+            uint32_t t[2] = {0u, 0u};
+#pragma unroll
+            for (int mag = 0; mag < 8; mag++) {
+                const __half_raw h = __nv_cvt_fp4_to_halfraw((__nv_fp4_storage_t)mag, __NV_E2M1);
+                const float v = __half2float(__half(h)) * __uint_as_float((uint32_t)(127 - lane) << 23);
+                const uint32_t e8 = (uint32_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+                t[mag >> 2] |= e8 << (8 * (mag & 3));
+            }
+            lut[2 * lane] = t[0];
+            lut[2 * lane + 1] = t[1];
+        }
+        tc::named_bar_sync(1, 32 * C::UW);
+        // thread ut takes RPT rows (or, with more threads than rows, BPT of
+        // a row's 4 channel blocks); the block exponents of its rows are
+        // loaded one tile ahead (rows past the table, zero-filled, take j = 0)
+        constexpr int UT = 32 * C::UW;
+        constexpr int TPR = UT > 128 ? UT / 128 : 1;         // threads per row
+        constexpr int RPT = UT >= 128 ? 1 : 128 / UT;        // rows per thread
+        constexpr int BPT = 4 / TPR;                         // blocks per thread
+        const int ut = uw * 32 + lane;
+        auto row_of = [&](int x) { return ut / TPR + x * (UT / TPR); };
+        auto exps_of = [&](int i, uint32_t(&e)[RPT]) {
+#pragma unroll
+            for (int x = 0; x < RPT; x++) {
+                const int64_t s = s_begin + (int64_t)i * 128 + row_of(x);
+                e[x] = (i < ntiles && s < a.E)
+                           ? __ldg((const uint32_t *)a.kI_exp + ((int64_t)b * a.E + s) * a.ks_stride)
+                           : 0x7f7f7f7fu;
+            }
+        };
+        uint32_t exn[RPT];
+        exps_of(0, exn);
         bool ok = true;
         for (int i = 0; i < ntiles && ok; i++) {
             const int st = i % S;
+            uint32_t exc[RPT];
+#pragma unroll
+            for (int x = 0; x < RPT; x++)
+                exc[x] = exn[x];
+            exps_of(i + 1, exn);
             if (!tc::mbar_wait(&rfull[st], (i / S) & 1, abort_flag) ||
                 (i >= S && !tc::mbar_wait(&empty[st], ((i / S) - 1) & 1, abort_flag))) {
                 *abort_flag = 1;
@@ -474,42 +529,38 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 ok = false;
                 break;
             }
-            for (int r = uw * 32 + lane; r < 128; r += 32 * C::UW) {
-                const int64_t s = s_begin + (int64_t)i * 128 + r;
-                // rows past the table (zero-filled) take j = 0
-                uint32_t ex = 0x7f7f7f7fu;
-                if (s < a.E)
-                    ex = __ldg((const uint32_t *)a.kI_exp + ((int64_t)b * a.E + s) * a.ks_stride);
+#pragma unroll
+            for (int x = 0; x < RPT; x++) {
+                const int r = row_of(x);
+                const uint32_t ex = exc[x];
                 const uint32_t em = max(max(ex & 255u, (ex >> 8) & 255u),
                                         max((ex >> 16) & 255u, ex >> 24));
                 const uint8_t *src = sR + (size_t)st * 8192 + r * 64;
                 uint8_t *dst = sA + (size_t)st * 16384 + r * 128;
 #pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    const int blk = (q + (r >> 1)) & 3;           // spreads the banks
+                for (int q = 0; q < BPT; q++) {
+                    // rotated by row: spreads the banks
+                    const int blk = (ut % TPR) * BPT + ((q + (r >> 1)) & (BPT - 1));
                     const uint4 w = *(const uint4 *)(src + blk * 16);
                     int j = (int)(em - ((ex >> (8 * blk)) & 255u));
                     j = j > 8 ? 8 : j;
-                    const __half2 sc = __float2half2_rn(__uint_as_float((uint32_t)(127 - j) << 23));
+                    const uint32_t t0 = lut[2 * j], t1 = lut[2 * j + 1];
                     const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
                     uint32_t o[8];
 #pragma unroll
                     for (int u = 0; u < 4; u++) {
-                        uint32_t lo = 0u, hi = 0u;
-#pragma unroll
-                        for (int bb = 0; bb < 4; bb++) {
-                            const __half2_raw hr = __nv_cvt_fp4x2_to_halfraw2(
-                                (__nv_fp4x2_storage_t)((wv[u] >> (8 * bb)) & 255u), __NV_E2M1);
-                            const __half2 hv = __hmul2(__half2(hr), sc);
-                            const uint32_t e8 = (uint32_t)__nv_cvt_halfraw2_to_fp8x2(
-                                __half2_raw(hv), __NV_SATFINITE, __NV_E4M3);
-                            if (bb < 2)
-                                lo |= e8 << (16 * bb);
-                            else
-                                hi |= e8 << (16 * (bb - 2));
-                        }
-                        o[2 * u] = lo;
-                        o[2 * u + 1] = hi;
+                        // word u: channels 8u .. 8u + 7 of the block, channel
+                        // 2c in the low nibble of byte c
+                        const uint32_t x = wv[u], xs = x << 4;
+                        const uint32_t m0 = prmt(t0, t1, x & 0x7777u);
+                        const uint32_t m1 = prmt(t0, t1, (x >> 16) & 0x7777u);
+                        // sign of channel 2c: top bit of byte c of x << 4;
+                        // of channel 2c + 1: top bit of byte c of x (the
+                        // selector's bit 3 replicates that bit over the byte)
+                        const uint32_t s0 = prmt(xs, x, 0xD9C8u) & 0x80808080u;
+                        const uint32_t s1 = prmt(xs, x, 0xFBEAu) & 0x80808080u;
+                        o[2 * u] = m0 | s0;
+                        o[2 * u + 1] = m1 | s1;
                     }
                     // channels 32 blk .. 32 blk + 31: 16-byte chunks 2 blk and
                     // 2 blk + 1 of the row, at chunk ^ (row % 8)
