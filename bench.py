@@ -157,20 +157,35 @@ def job_rate(local_ms, units_per_rank, world, dist, device):
 
 
 def units_per_step(w):
-    return w.batch if w.kind == "decode" else w.n
+    if w.kind == "decode":
+        return w.batch
+    return LAST_N if (LAST_N and w.kind == "csa") else w.n
 
 
 def unit_of(w):
     return "queries/s" if w.kind == "decode" else "tokens/s"
 
 
+# --fp4-keys: the indexer keys are stored in FP4 (e2m1 + a power-of-two scale
+# per 32 channels) instead of the workload's e4m3 keys
+FP4_KEYS = False
+# --last N: a CSA prefill step runs only the last N queries of the sequence
+# (its longest rows) over the whole sequence's entries (profiling cases)
+LAST_N = None
+
+
 def config_of(w, world=1):
     """The workload description both arms print (same keys, same values)."""
-    return {"workload": w.name, "n": w.n, "c": w.c, "m": w.m, "k": w.k, "h": w.h,
-            "hI": w.hI, "cI": w.cI, "n_win": w.n_win, "dtype": w.dtype,
-            "indexer_dtype": w.idx_dtype, "batch_per_gpu": w.batch,
-            "l2": "flushed between timed steps (512 MiB write)",
-            "parallelism": "dp%d (independent sequences)" % world}
+    cfg = {"workload": w.name, "n": w.n, "c": w.c, "m": w.m, "k": w.k, "h": w.h,
+           "hI": w.hI, "cI": w.cI, "n_win": w.n_win, "dtype": w.dtype,
+           "indexer_dtype": w.idx_dtype, "batch_per_gpu": w.batch,
+           "l2": "flushed between timed steps (512 MiB write)",
+           "parallelism": "dp%d (independent sequences)" % world}
+    if FP4_KEYS and w.hI:
+        cfg["indexer_keys"] = "e2m1, one power-of-two scale per 32 channels"
+    if LAST_N and w.kind == "csa":
+        cfg["queries"] = "the last %d positions" % LAST_N
+    return cfg
 
 
 def build_path(w, rank, keep_ops=False):
@@ -178,24 +193,33 @@ def build_path(w, rank, keep_ops=False):
     operands it was built from)."""
     from long_context_sparse_07_b200 import path
     wr = rank_workload(w, rank)
-    if w.kind == "csa":
+    if w.kind == "csa" and LAST_N:
+        q_lo = wr.n - LAST_N
+        ops = W.csa_operands(wr, parts=("kv", "indexer"))
+        for k in ("qI", "qI_scale", "wI"):
+            if k in ops:
+                ops[k] = ops[k][q_lo:].contiguous()
+        ops.update(W.csa_operands(wr, lo=q_lo, parts=("query",)))
+        p = path.CsaPrefill(wr, ops, fused=True, fp4_keys=FP4_KEYS and w.idx_dtype == "e4m3",
+                            q_lo=q_lo)
+    elif w.kind == "csa":
         ops = W.csa_operands(wr)
-        p = path.CsaPrefill(wr, ops, fused=True)
+        p = path.CsaPrefill(wr, ops, fused=True, fp4_keys=FP4_KEYS and w.idx_dtype == "e4m3")
     elif w.kind == "hca":
         ops = W.hca_operands(wr)
         p = path.HcaPrefill(wr, ops)
     else:
-        ops = W.decode_operands(wr)
+        ops = W.decode_operands(wr, fp4_keys=FP4_KEYS)
         p = path.Decode(wr, ops)
     return (p, ops) if keep_ops else p
 
 
 def algorithmic(w, p):
     if w.kind == "csa":
-        return work.csa_prefill(w)
+        return work.csa_prefill(w, fp4_keys=getattr(p, "fp4_keys", False), q_lo=w.n - p.nq)
     if w.kind == "hca":
         return work.hca_prefill(w)
-    return work.decode(w, p.E, p.E_hca)
+    return work.decode(w, p.E, p.E_hca, fp4_keys=getattr(p, "fp4_keys", False))
 
 
 def kernel_roofline(w, name, a, ms, pk):
@@ -709,7 +733,7 @@ def run_ours(args, w):
     dom = summ["dominant"]
     roof = dict(summ["kernels"][dom])
     roof.pop("ideal_ms", None)
-    roof["traffic"] = measured_traffic(w.name, dom)
+    roof["traffic"] = measured_traffic(w.name, dom) if not (LAST_N or FP4_KEYS) else None
     roof["kernel"] = dom
     roof["peak_source"] = pk["source"] if roof.get("peak_dtype") != "e4m3" else pk["fp8_source"]
     roof["kernel_ms"] = summ["kernel_ms"]
@@ -813,6 +837,12 @@ def main():
                     help="time only the selected workload")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the RMSNorm/RoPE and grouped-projection timings")
+    ap.add_argument("--fp4-keys", action="store_true",
+                    help="store the indexer keys in FP4 (e2m1 + a scale per 32 channels); "
+                         "no CPU baseline or reference arm in this mode")
+    ap.add_argument("--last", type=int, default=None,
+                    help="CSA prefill: run only the last N queries over the whole sequence's "
+                         "entries (profiling cases; no CPU baseline or reference arm)")
     ap.add_argument("--n", type=int, default=None,
                     help="run the workload on a shorter sequence of n tokens (small profiling cases)")
     ap.add_argument("--graph", default="auto", choices=["auto", "on", "off"],
@@ -826,6 +856,21 @@ def main():
         if args.n % w.m or args.n <= 0:
             sys.exit("--n must be a positive multiple of m = %d" % w.m)
         w = W.scaled(w, n=args.n, name="%s@n%d" % (w.name, args.n))
+    if args.last is not None:
+        if args.impl == "reference" or w.kind != "csa" or not 0 < args.last <= w.n:
+            sys.exit("--last takes 0 < N <= n on a CSA prefill workload, our arm only")
+        global LAST_N
+        LAST_N = args.last
+        args.no_cpu_baseline = True
+        args.no_extras = True
+        args.no_per_workload = True
+    if args.fp4_keys:
+        if args.impl == "reference":
+            sys.exit("--fp4-keys has no reference arm")
+        global FP4_KEYS
+        FP4_KEYS = True
+        args.no_cpu_baseline = True
+        args.no_extras = True
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -42,27 +42,38 @@ class CsaPrefill:
         """Kernels launched by one step (top-k of long rows takes four; the
         normalisation and RoPE add four)."""
         if self.fused:
-            sel = abi.csa_indexer_topk_launches(1, self.w.n, self.w.E, self.w.hI, self.w.cI,
+            sel = abi.csa_indexer_topk_launches(1, self.nq, self.w.E, self.w.hI, self.w.cI,
                                                 self.w.k, self.d["qI"])
         else:
             sel = 1 + (4 if self.topk_ws is not None else 1)
         return 3 + sel + (4 if self.rope_dims else 0)
 
     def __init__(self, w, ops: Dict[str, torch.Tensor], device="cuda", rope_dims: int = 0,
-                 fused: bool = False):
+                 fused: bool = False, fp4_keys: bool = False, q_lo: int = 0):
+        """`ops` as ``workloads.csa_operands``; with q_lo > 0 the queries (q,
+        qI, qI_scale, wI) are only those of positions q_lo .. n - 1 (the
+        sequence's longest rows), the KV side the whole sequence."""
         self.w = w
         self.fused = fused
+        self.fp4_keys = fp4_keys
         d = self.d = _dev(ops, device)
-        n, c, E = w.n, w.c, w.E
+        c, E = w.c, w.E
+        n = self.nq = w.n - q_lo
         # with rope_dims > 0 the step also applies Module D's RMSNorm and
         # partial RoPE to the entries, the window rows (a copy of C^a) and the
         # queries, and turns the output back by the query position
         self.rope_dims = rope_dims
         self.kwin = torch.empty_like(d["Ca"]) if rope_dims else d["Ca"]
-        self.q_pos = torch.arange(n, device=device, dtype=torch.int64)
+        self.q_pos = torch.arange(q_lo, w.n, device=device, dtype=torch.int64)
         self.win_pos0 = torch.zeros(1, device=device, dtype=torch.int64)
         self.entries = Entries(torch.empty(E, c, device=device, dtype=DT[w.dtype]), c)
-        if w.idx_dtype == "e4m3":
+        if fp4_keys:
+            # FP4 indexer keys (e2m1 + a power-of-two scale per 32 channels),
+            # written by the compressor; the queries stay e4m3
+            self.kI = Entries(torch.empty(E, w.cI // 2, device=device, dtype=torch.uint8), w.cI,
+                              scale=torch.empty(E, w.cI // 32, device=device, dtype=torch.uint8),
+                              scale_group=32, fp4=True)
+        elif w.idx_dtype == "e4m3":
             self.kI = Entries(torch.empty(E, w.cI, device=device, dtype=torch.float8_e4m3fn),
                               w.cI, scale=torch.empty(E, device=device, dtype=torch.float32),
                               scale_group=w.cI)
@@ -216,8 +227,14 @@ class Decode:
         B = w.batch
         self.E = d["kI"].shape[1]
         self.E_hca = d["hca_nope"].shape[1]
-        self.kI = Entries(d["kI"].view(B * self.E, w.cI), w.cI,
-                          scale=d["kI_scale"].view(B * self.E), scale_group=w.cI)
+        self.fp4_keys = "kI_exp" in d
+        if self.fp4_keys:
+            self.kI = Entries(d["kI"].view(B * self.E, w.cI // 2), w.cI,
+                              scale=d["kI_exp"].view(B * self.E, w.cI // 32), scale_group=32,
+                              fp4=True)
+        else:
+            self.kI = Entries(d["kI"].view(B * self.E, w.cI), w.cI,
+                              scale=d["kI_scale"].view(B * self.E), scale_group=w.cI)
         self.kv = Entries(d["kv_nope"].view(B * self.E, -1), w.c,
                           scale=d["kv_scale"].view(B * self.E, -1),
                           rope=d["kv_rope"].view(B * self.E, -1), rope_dims=w.rope_dims,

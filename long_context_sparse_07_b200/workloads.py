@@ -44,6 +44,7 @@ _TENSOR_IDS = {
     "kv_nope": 21, "kv_scale": 22, "kv_rope": 23, "kI": 24, "kI_scale": 25,
     "kwin": 26, "hca_nope": 27, "hca_scale": 28, "hca_rope": 29,
     "scores": 30, "idx_u": 31, "entries": 32, "kwin_step": 33,
+    "kI_fp4": 34, "kI_exp": 35,
     "H": 40, "W_aKV": 41, "W_bKV": 42, "W_aZ": 43, "W_bZ": 44, "W_aKI": 45, "W_bKI": 46,
     "W_aZI": 47, "W_bZI": 48, "W_DQ": 49, "W_IUQ": 50, "W_w": 51, "W_UQ": 52,
 }
@@ -256,6 +257,13 @@ def uniform(seed, name, rows, cols, lo=0, hi=None) -> np.ndarray:
     return _rows(seed, name, rows, cols, draw, lo, hi)
 
 
+def bytes_in(seed, name, rows, cols, lo_val, hi_val, lo=0, hi=None) -> torch.Tensor:
+    """Drawn uint8 values, uniform in [lo_val, hi_val]."""
+    def draw(g, shape):
+        return g.integers(lo_val, hi_val + 1, size=shape, dtype=np.uint8)
+    return torch.from_numpy(_rows(seed, name, rows, cols, draw, lo, hi, dtype=np.uint8))
+
+
 def to_storage(x: np.ndarray, dtype: str) -> torch.Tensor:
     """Cast drawn float32 values to a storage dtype ("f32" or "bf16")."""
     t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
@@ -341,7 +349,7 @@ def hca_operands(w: Workload, lo: int = 0, hi: Optional[int] = None,
 
 
 def decode_operands(w: Workload, E: Optional[int] = None,
-                    E_hca: Optional[int] = None) -> Dict[str, torch.Tensor]:
+                    E_hca: Optional[int] = None, fp4_keys: bool = False) -> Dict[str, torch.Tensor]:
     """Operands of one batched decode step.
 
     Every sequence b holds a context of ``n`` tokens and one query at position
@@ -350,7 +358,9 @@ def decode_operands(w: Workload, E: Optional[int] = None,
     HCA cache: hca_nope / hca_scale / hca_rope with E_hca entries. Queries:
     qI [B, 1, hI, cI] e4m3, qI_scale [B, 1, hI], wI [B, 1, hI], q [B, 1, h, c]
     bf16, kwin [B, n_win, c] bf16 holding positions n - n_win .. n - 1, sink
-    [h]; q_pos [B, 1] and win_pos0 [B] (int64).
+    [h]; q_pos [B, 1] and win_pos0 [B] (int64). With fp4_keys the indexer
+    keys are FP4 instead: kI [B, E, cI / 2] uniform packed e2m1 code bytes,
+    kI_exp [B, E, cI / 32] block exponents uniform in 118..126 (a span of 8).
     """
     B, s = w.batch, w.seed
     E = w.n // w.m if E is None else E
@@ -364,8 +374,12 @@ def decode_operands(w: Workload, E: Optional[int] = None,
                                           w.std_proj).view(B, En, G)
         out[pre + "_rope"] = to_storage(normal(s, pre + "_rope", B * En, w.rope_dims,
                                                w.std_proj), "bf16").view(B, En, w.rope_dims)
-    out["kI"] = e4m3_codes(s, "kI", B * E, w.cI).view(B, E, w.cI)
-    out["kI_scale"] = e4m3_scales(s, "kI_scale", B * E, 1, w.std_proj).view(B, E)
+    if fp4_keys:
+        out["kI"] = bytes_in(s, "kI_fp4", B * E, w.cI // 2, 0, 255).view(B, E, w.cI // 2)
+        out["kI_exp"] = bytes_in(s, "kI_exp", B * E, w.cI // 32, 118, 126).view(B, E, w.cI // 32)
+    else:
+        out["kI"] = e4m3_codes(s, "kI", B * E, w.cI).view(B, E, w.cI)
+        out["kI_scale"] = e4m3_scales(s, "kI_scale", B * E, 1, w.std_proj).view(B, E)
     out["qI"] = e4m3_codes(s, "qI", B, w.hI * w.cI).view(B, 1, w.hI, w.cI)
     out["qI_scale"] = e4m3_scales(s, "qI_scale", B, w.hI, w.std_q).view(B, 1, w.hI)
     out["wI"] = to_storage(normal(s, "wI", B, w.hI, w.std_w), "f32").view(B, 1, w.hI)
