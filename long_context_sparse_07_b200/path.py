@@ -166,6 +166,67 @@ class CsaPrefill:
         for _, f in self.phases():
             f(stream)
 
+    QUERY_SIDE = ("q", "qI", "qI_scale", "wI")
+
+    def step_from_host(self, host_in: Dict[str, torch.Tensor], host_out: torch.Tensor,
+                       stream=None, chunk: int = 16384):
+        """One step from pinned host operands (keys as ``inputs()``) to a
+        pinned host output (shaped like ``result()``), the copies overlapped
+        with the computation: the KV side arrives first and is compressed;
+        then the queries come in chunks, each chunk's selection and attention
+        running while the next chunk's queries arrive and the previous chunk's
+        output leaves on a second copy stream (host-to-device and
+        device-to-host copies run at the same time). The result equals
+        ``step()``'s: every query's work is the same, only grouped by chunk."""
+        cur = stream if stream is not None else torch.cuda.current_stream()
+        d, w = self.d, self.w
+        if self.rope_dims or not self.fused:
+            for k, v in host_in.items():
+                d[k].copy_(v, non_blocking=True)
+            self.step(cur)
+            host_out.copy_(self.out, non_blocking=True)
+            return
+        if not hasattr(self, "_h2d"):
+            self._h2d, self._d2h = torch.cuda.Stream(), torch.cuda.Stream()
+            self._chunk_ws = {}
+        h2d, d2h = self._h2d, self._d2h
+        h2d.wait_stream(cur)                      # earlier work on these buffers is done
+        d2h.wait_stream(cur)
+        qside = [k for k in self.QUERY_SIDE if k in d]
+        with torch.cuda.stream(h2d):
+            for k, v in host_in.items():
+                if k not in qside:
+                    d[k].copy_(v, non_blocking=True)
+        cur.wait_event(h2d.record_event())
+        self.compress_kv(cur)
+        self.compress_index(cur)
+        qs = d.get("qI_scale")
+        for lo in range(0, self.nq, chunk):
+            hi = min(self.nq, lo + chunk)
+            with torch.cuda.stream(h2d):
+                for k in qside:
+                    d[k][lo:hi].copy_(host_in[k][lo:hi], non_blocking=True)
+            cur.wait_event(h2d.record_event())
+            rows = hi - lo
+            if rows not in self._chunk_ws:
+                nf = abi.csa_indexer_topk_workspace_size(1, rows, w.E, w.hI, w.cI, w.k, d["qI"])
+                na = abi.csa_mqa_workspace_size(1, rows, w.h, w.c, w.k + w.n_win)
+                self._chunk_ws[rows] = (
+                    torch.empty(nf, device=self.out.device, dtype=torch.uint8) if nf else None,
+                    torch.empty(na, device=self.out.device, dtype=torch.uint8) if na else None)
+            fws, aws = self._chunk_ws[rows]
+            abi.csa_indexer_topk(d["qI"][lo:hi][None], qs[lo:hi][None] if qs is not None else None,
+                                 d["wI"][lo:hi][None], self.kI, self.q_pos[lo:hi][None], w.m, w.k,
+                                 self.idx[lo:hi], w.E, workspace=fws, stream=cur)
+            abi.csa_sparse_mqa(d["q"][lo:hi][None], self.entries, w.E, w.m, self.idx[lo:hi], w.k,
+                               self.kwin[None], self.win_pos0, w.n_win, self.q_pos[lo:hi][None],
+                               d["sink"], self.scale, self.out[:, lo:hi], self.lse[:, lo:hi],
+                               workspace=aws, stream=cur)
+            d2h.wait_event(cur.record_event())
+            with torch.cuda.stream(d2h):
+                host_out[:, lo:hi].copy_(self.out[:, lo:hi], non_blocking=True)
+        cur.wait_stream(d2h)
+
 
 class HcaPrefill:
     """One causal HCA prefill of a single sequence (batch 1)."""
