@@ -170,7 +170,9 @@ csa_status csa_indexer_scores(const void *qI, const float *qI_scale, const float
  *   workspace, ws_bytes   device scratch of at least
  *             csa_topk_workspace_size(rows, E, k) bytes, 256-byte aligned
  *             (may be NULL when that size is 0; it is nonzero for rows of
- *             65536 entries or more, which are split over many blocks).
+ *             more than 262144 entries, which are split over many blocks
+ *             in four launches; rows of 65536 .. 262144 entries take one
+ *             launch, a cluster of 8 blocks per row, and no workspace).
  *             The caller owns it; nothing in it must be initialised.
  * Requirements: 1 <= k <= 4096.
  */

@@ -12,10 +12,13 @@
 //    kept in shared memory and selected exactly with 8-bit digits; for larger
 //    k the keys are staged once in shared memory when they fit (re-read from
 //    L2 otherwise) and selected with 12 + 12 + 8-bit digits;
-//  * longer rows (decode): chunks of the row over many blocks, then one block
-//    per row over the candidates of the threshold bin.
+//  * longer rows (decode): rows of up to 256 K entries in one launch, a
+//    cluster of 8 blocks per row exchanging digit counts through distributed
+//    shared memory; past that, chunks of the row over many blocks, then one
+//    block per row over the candidates of the threshold bin.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace csa {
 
@@ -647,7 +650,7 @@ topk_mid_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
 }
 
 // ---------------------------------------------------------------------------
-// Long rows (many entries, few rows: decode): the row is cut into chunks of
+// Rows longer than the cluster path takes: the row is cut into chunks of
 // kChunk entries handled by separate blocks, in four launches:
 //   1. per-chunk histograms of the top 12 key bits;
 //   2. the row's bin totals, a slice of bins per block;
@@ -891,6 +894,652 @@ topk_final_kernel(const int64_t *__restrict__ q_pos, int64_t E, int m, int k, in
     __syncthreads();
     RowCandidates src{jk, ji};
     block_select(src, C, k, out, keys, C <= kResident, sh);
+}
+
+// ---------------------------------------------------------------------------
+// Long rows of up to kCluCtas * kCluChunk entries (decode over a 1 M-token
+// context: 262144 entries): one launch, each row taken by a cluster of
+// kCluCtas blocks, block c staging the keys of its contiguous share of the
+// row in shared memory. The blocks talk through distributed shared memory
+// and hardware cluster barriers only.
+//  1. Bound: every 32nd key of the row is a sample; with mu = k ns / V the
+//     samples expected at or above the row's k-th largest key, a bound with
+//     ks = 1.25 mu + 4 sqrt(mu) + 8 samples at or above it lies below that
+//     key unless the sample is off by many standard deviations. Each block
+//     takes the ceil(ks / kCluCtas)-th largest of its own samples (every
+//     warp's largest ones by repeated warp maxima, merged by one warp); the
+//     smallest of the blocks' values has at least ks samples at or above it.
+//  2. Candidates: each warp keeps the (key, index) pairs of its 1024 entries
+//     at or above the bound in its own region, in index order.
+//  3. When the candidates number at least k and every region held its own,
+//     block 0 gathers them in index order and selects exactly (digits from
+//     the first bit in which the candidates differ, ties to the lower index);
+//     the k-th largest key is at or above the bound, so every key that can
+//     be selected is a candidate.
+//  4. Otherwise (a bound that turned out too high, or candidates crowding one
+//     part of the row) the cluster selects over all keys: three radix rounds
+//     (11, 11, 10 bits) in which every block counts the digits of its keys
+//     that match the prefix so far and reads the other blocks' counts, then
+//     one more exchange of the counts above the threshold key and equal to it,
+//     after which each block writes its own elements in index order.
+constexpr int kCluCtas = 8;
+constexpr int kCluThreads = 1024;
+constexpr int kCluWarps = kCluThreads / 32;
+constexpr int kCluChunk = 32768;                  // keys per block (128 KB of shared memory)
+constexpr int kCluBins = 2048;
+constexpr int kCluCopies = 4;
+constexpr int kCluStep = 32;                      // sample spacing
+constexpr int kCluRegion = 128;                   // candidate pairs per warp
+constexpr int kCluGather = kCluChunk / 2;         // pairs block 0 gathers (in its key area)
+constexpr int kCluSel = 256;                      // threads of block 0 that select among them
+constexpr size_t kCluSmem =
+    (size_t)(kCluChunk + kCluCopies * kCluBins + 2 * kCluBins + kCluBins) * sizeof(uint32_t);
+static_assert(kCluWarps * kCluRegion * 2 <= kCluCopies * kCluBins, "regions alias the counters");
+static_assert(kCluChunk / kCluStep <= kCluThreads, "one sample per thread");
+
+__host__ __device__ inline bool cluster_takes(int64_t rows, int64_t E)
+{
+    return rows > 0 && rows <= 65535 && E >= kMultiMinE && E <= (int64_t)kCluCtas * kCluChunk;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_arrive()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_map(const void *local, uint32_t rank)
+{
+    const uint32_t a = (uint32_t)__cvta_generic_to_shared(local);
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    return ra;
+}
+
+// A 32-bit word of block `rank`'s shared memory, at the place `local` has in ours.
+__device__ __forceinline__ uint32_t cluster_ld(const uint32_t *local, uint32_t rank)
+{
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_map(local, rank))
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint2 cluster_ld2(const uint2 *local, uint32_t rank)
+{
+    uint2 v;
+    asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "r"(cluster_map(local, rank))
+                 : "memory");
+    return v;
+}
+
+struct CluShared {
+    uint32_t wa[kCluWarps], wb[kCluWarps];
+    uint32_t wcnt[kCluWarps];                     // candidates of each warp (read by block 0)
+    uint32_t pre[kCluCtas][kCluWarps + 1];        // block 0: where each region's pairs go
+    uint32_t samp[kCluThreads];
+    uint32_t tl[kCluWarps][32];                   // each warp's largest samples
+    uint32_t bin, above, off, take, x, L, nc, ovf, fast;
+    uint32_t cnt[2];                              // published: keys > T, keys == T
+    uint64_t staged;                              // the bulk copies of the share landed
+    int never;                                    // an abort flag nothing sets
+};
+
+// Barrier of the first NT threads of the block (all of them: barrier 0;
+// fewer: named barrier 1, which nothing else uses).
+template <int NT>
+__device__ __forceinline__ void team_sync()
+{
+    if (NT == kCluThreads)
+        __syncthreads();
+    else
+        asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
+
+// Of the counts cnt[0 .. kCluBins) (digits), the digit holding the need-th
+// largest element counted from the top, and how many lie above it, worked out
+// by the first NT threads. Call with cnt complete and visible to them; the
+// result is in sh.bin / sh.above after the closing barrier. Thread i owns the
+// PER digits below 2047 - PER i.
+template <int NT>
+__device__ __forceinline__ void clu_find(const uint32_t *cnt, uint32_t need, CluShared &sh)
+{
+    constexpr int PER = kCluBins / NT;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int top = kCluBins - 1 - PER * tid;
+    uint32_t t[PER], loc = 0;
+#pragma unroll
+    for (int u = 0; u < PER; u++) {
+        t[u] = cnt[top - u];
+        loc += t[u];
+    }
+    uint32_t v = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o)
+            v += x;
+    }
+    if (lane == 31)
+        sh.wa[warp] = v;
+    team_sync<NT>();
+    uint32_t before = 0;
+    if (lane < warp)
+        before = sh.wa[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        before += __shfl_xor_sync(0xffffffffu, before, o);
+    const uint32_t incl = v + before, excl = incl - loc;
+    if (excl < need && need <= incl) {
+        uint32_t cum = excl;
+#pragma unroll
+        for (int u = 0; u < PER; u++) {
+            if (cum + t[u] >= need) {
+                sh.bin = (uint32_t)(top - u);
+                sh.above = cum;
+                break;
+            }
+            cum += t[u];
+        }
+    }
+    team_sync<NT>();
+}
+
+// Exclusive prefix over the first NT threads of two per-thread counts, and
+// their totals.
+template <int NT>
+__device__ __forceinline__ void clu_scan2(uint32_t a, uint32_t b, CluShared &sh, uint32_t *a_before,
+                                          uint32_t *b_before, uint32_t *a_tot, uint32_t *b_tot)
+{
+    constexpr int NW = NT / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t va = a, vb = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t xa = __shfl_up_sync(0xffffffffu, va, o);
+        const uint32_t xb = __shfl_up_sync(0xffffffffu, vb, o);
+        if (lane >= o) {
+            va += xa;
+            vb += xb;
+        }
+    }
+    if (lane == 31) {
+        sh.wa[warp] = va;
+        sh.wb[warp] = vb;
+    }
+    team_sync<NT>();
+    const uint32_t wa = lane < NW ? sh.wa[lane] : 0u, wb = lane < NW ? sh.wb[lane] : 0u;
+    uint32_t pa = lane < warp ? wa : 0u, pb = lane < warp ? wb : 0u, ta = wa, tb = wb;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        pa += __shfl_xor_sync(0xffffffffu, pa, o);
+        pb += __shfl_xor_sync(0xffffffffu, pb, o);
+        ta += __shfl_xor_sync(0xffffffffu, ta, o);
+        tb += __shfl_xor_sync(0xffffffffu, tb, o);
+    }
+    *a_before = pa + va - a;
+    *b_before = pb + vb - b;
+    *a_tot = ta;
+    *b_tot = tb;
+    team_sync<NT>();                                       // wa / wb are reused
+}
+
+// The exact top-k of C (key, index) pairs in index order (gk, gi), ties to
+// the lower index, by the first kCluSel threads: the pairs' common top bits
+// (from the smallest and largest key), then digits of up to 11 bits, the
+// digit counts alternating between h0 and h1 (the next one cleared while the
+// current one is filled); then an ordered write, each thread owning a run of
+// consecutive pairs.
+__device__ __forceinline__ void clu_select_team(const uint32_t *gk, const uint32_t *gi, uint32_t C,
+                                                int k, uint32_t *h0, uint32_t *h1, int32_t *out,
+                                                CluShared &sh)
+{
+    constexpr int NT = kCluSel, NW = NT / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t mn = 0xffffffffu, mx = 0u;
+    for (uint32_t e = (uint32_t)tid; e < C; e += NT) {
+        mn = min(mn, gk[e]);
+        mx = max(mx, gk[e]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (lane == 0) {
+        sh.wa[warp] = mn;
+        sh.wb[warp] = mx;
+    }
+    for (int b = tid; b < kCluBins; b += NT)
+        h0[b] = 0;
+    team_sync<NT>();
+    mn = lane < NW ? sh.wa[lane] : 0xffffffffu;
+    mx = lane < NW ? sh.wb[lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    team_sync<NT>();                                     // wa / wb reused by clu_find
+    int bits = mn == mx ? 0 : 32 - __clz(mn ^ mx);
+    uint32_t pmask = bits == 32 ? 0u : ~((1u << bits) - 1u);
+    uint32_t prefix = mn & pmask, need = (uint32_t)k;
+    for (int r = 0; bits > 0; r++) {
+        const int w = bits < 11 ? bits : 11;
+        const int shift = bits - w;
+        const uint32_t dm = (1u << w) - 1u;
+        uint32_t *h = (r & 1) ? h1 : h0, *hn = (r & 1) ? h0 : h1;
+        for (uint32_t e = (uint32_t)tid; e < C; e += NT) {
+            const uint32_t kk = gk[e];
+            if ((kk & pmask) == prefix)
+                atomicAdd(&h[(kk >> shift) & dm], 1u);
+        }
+        for (int b = tid; b < kCluBins; b += NT)
+            hn[b] = 0;
+        team_sync<NT>();
+        clu_find<NT>(h, need, sh);
+        prefix |= sh.bin << shift;
+        need -= sh.above;
+        pmask |= dm << shift;
+        bits = shift;
+    }
+    const uint32_t T = prefix;
+    const uint32_t per = (C + NT - 1) / NT;
+    const uint32_t e0 = (uint32_t)tid * per, e1 = min(C, e0 + per);
+    uint32_t ng = 0, ne = 0;
+    for (uint32_t e = e0; e < e1; e++) {
+        ng += gk[e] > T ? 1u : 0u;
+        ne += gk[e] == T ? 1u : 0u;
+    }
+    uint32_t g_b, e_b, g_t, e_t;
+    clu_scan2<NT>(ng, ne, sh, &g_b, &e_b, &g_t, &e_t);
+    uint32_t pos = g_b + min(e_b, need), er = e_b;
+    for (uint32_t e = e0; e < e1; e++) {
+        const uint32_t kk = gk[e];
+        const bool sel = kk > T || (kk == T && er < need);
+        er += kk == T ? 1u : 0u;
+        if (sel && pos < (uint32_t)k)
+            out[pos] = (int32_t)gi[e];
+        pos += sel ? 1u : 0u;
+    }
+}
+
+__global__ void __cluster_dims__(kCluCtas, 1, 1) __launch_bounds__(kCluThreads, 1)
+topk_cluster_kernel(const float *__restrict__ scores, int64_t E, int64_t ld,
+                    const int64_t *__restrict__ q_pos, int m, int k, int32_t *__restrict__ idx,
+                    unsigned *err)
+{
+    extern __shared__ uint4 clu_smem[];
+    uint32_t *keys = (uint32_t *)clu_smem;                  // [kCluChunk]
+    uint32_t *hc = keys + kCluChunk;                        // [kCluCopies][kCluBins]
+    uint2 *cand = (uint2 *)hc;                              //   or [kCluWarps][kCluRegion] pairs
+    uint32_t *pub = hc + kCluCopies * kCluBins;             // [2][kCluBins] published counts
+    uint32_t *tot = pub + 2 * kCluBins;                     // [kCluBins]
+    __shared__ CluShared sh;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned lt = (1u << lane) - 1u;
+    const uint32_t c = cluster_rank();
+    const int64_t row = blockIdx.y;
+    const int64_t V = visible(q_pos[row], m, E);
+    int32_t *out = idx + row * k;
+    if (V <= k) {
+        // the same decision in every block of the cluster: no barrier follows
+        for (int64_t j = (int64_t)c * kCluThreads + tid; j < k; j += kCluCtas * kCluThreads)
+            out[j] = j < V ? (int32_t)j : -1;
+        return;
+    }
+    // this block's share [b0, b0 + n) of the row, a multiple of 4 entries long
+    const int64_t cs = (((V + kCluCtas - 1) / kCluCtas) + 3) & ~(int64_t)3;
+    const int64_t b0 = (int64_t)c * cs;
+    const int n = (int)(V - b0 < 0 ? 0 : (V - b0 < cs ? V - b0 : cs));
+    const int ns_own = (n + kCluStep - 1) / kCluStep;
+    const float *src = scores + row * ld + b0;
+    if ((((uintptr_t)src) & 15u) == 0) {
+        // the share's whole 16-byte words by bulk copies (pieces of 32 KB
+        // from one thread), the last n % 4 entries by plain loads; then every
+        // word turned into its key in place
+        const int n4 = n >> 2;
+        if (tid == 0) {
+            sh.never = 0;
+            tc::mbar_init(&sh.staged, 1);
+            tc::fence_mbar_init();
+        }
+        __syncthreads();
+        if (tid == 0) {
+            tc::mbar_arrive_expect_tx(&sh.staged, (uint32_t)n4 * 16u);
+            for (uint32_t off = 0; off < (uint32_t)n4 * 16u; off += 32768u) {
+                const uint32_t len = min(32768u, (uint32_t)n4 * 16u - off);
+                tc::bulk_load((uint8_t *)keys + off, (const uint8_t *)src + off, len, &sh.staged);
+            }
+        }
+        for (int j = 4 * n4 + tid; j < n; j += kCluThreads) {
+            keys[j] = float_key(__ldg(src + j));
+            if ((j & (kCluStep - 1)) == 0)
+                sh.samp[j / kCluStep] = keys[j];
+        }
+        if (!tc::mbar_wait(&sh.staged, 0, &sh.never, 100000000ull))
+            report(err, CSA_ERR_TIMEOUT, K_TOPK, (unsigned)row, c);   // carries on: every
+                                                                     // block keeps the
+                                                                     // cluster's barriers
+        uint4 *k4 = (uint4 *)keys;
+#pragma unroll 4
+        for (int i = tid; i < n4; i += kCluThreads) {
+            const uint4 f = k4[i];
+            const uint4 kk = make_uint4(float_key(__uint_as_float(f.x)), float_key(__uint_as_float(f.y)),
+                                        float_key(__uint_as_float(f.z)), float_key(__uint_as_float(f.w)));
+            k4[i] = kk;
+            if ((i & 7) == 0)
+                sh.samp[i >> 3] = kk.x;
+        }
+    } else {
+#pragma unroll 8
+        for (int j = tid; j < n; j += kCluThreads) {
+            const uint32_t kk = float_key(__ldg(src + j));
+            keys[j] = kk;
+            if ((j & (kCluStep - 1)) == 0)
+                sh.samp[j / kCluStep] = kk;
+        }
+    }
+    __syncthreads();                           // keys and samples complete
+
+    // ---- 1. the bound: the jl-th largest of this block's samples (each
+    // warp's jl largest by repeated warp maxima, merged by warp 0), then the
+    // smallest over the cluster
+    {
+        int64_t ns = 0;
+        for (int q = 0; q < kCluCtas; q++) {
+            const int64_t nq = V - q * cs < 0 ? 0 : (V - q * cs < cs ? V - q * cs : cs);
+            ns += (nq + kCluStep - 1) / kCluStep;
+        }
+        const float mu = (float)k * (float)ns / (float)V;
+        const int ks = (int)ceilf(1.25f * mu + 4.f * sqrtf(mu) + 8.f);
+        const int jl = min((ks + kCluCtas - 1) / kCluCtas, 32);
+        uint32_t v = tid < ns_own ? sh.samp[tid] : 0u;
+        for (int it = 0; it < jl; it++) {
+            uint32_t mx = v;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const unsigned who = __ballot_sync(0xffffffffu, v == mx);
+            if (lane == __ffs(who) - 1)
+                v = 0u;
+            if (lane == 0)
+                sh.tl[warp][it] = mx;
+        }
+        __syncthreads();
+        uint32_t x = 0;
+        if (warp == 0) {
+            // lane l walks warp l's list (descending)
+            int head = 0;
+            uint32_t cur = sh.tl[lane][0];
+            for (int it = 0; it < jl; it++) {
+                uint32_t mx = cur;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+                    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                x = mx;
+                const unsigned who = __ballot_sync(0xffffffffu, cur == mx);
+                if (lane == __ffs(who) - 1) {
+                    head++;
+                    cur = head < jl ? sh.tl[lane][head] : 0u;
+                }
+            }
+        }
+        if (tid == 0)
+            sh.x = x;
+        // idle warps wait at the block barrier, not at the cluster barrier
+        // (warps waiting there slow the ones still working)
+        __syncthreads();
+        cluster_arrive();
+        cluster_wait();
+        if (warp == 0) {
+            uint32_t v = lane < kCluCtas ? cluster_ld(&sh.x, (uint32_t)lane) : 0xffffffffu;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (lane == 0)
+                sh.L = v;
+        }
+        __syncthreads();
+    }
+    const uint32_t L = sh.L;
+
+    // ---- 2. candidates: warp w keeps its entries [1024 w, +1024) at or above L
+    {
+        const int wbase = warp * 1024;
+        uint2 *reg = cand + warp * kCluRegion;
+        uint32_t cnt = 0;
+#pragma unroll 4
+        for (int i = 0; i < 32; i++) {
+            const int j = wbase + 32 * i + lane;
+            const bool v = j < n;
+            const uint32_t kk = v ? keys[j] : 0u;
+            const bool on = v && kk >= L;
+            const unsigned bal = __ballot_sync(0xffffffffu, on);
+            const uint32_t at = cnt + __popc(bal & lt);
+            if (on && at < (uint32_t)kCluRegion)
+                reg[at] = make_uint2(kk, (uint32_t)(b0 + j));
+            cnt += __popc(bal);
+        }
+        if (lane == 0)
+            sh.wcnt[warp] = cnt;
+        __syncthreads();
+        if (warp == 0) {
+            const uint32_t wc = sh.wcnt[lane];
+            uint32_t tot_c = wc, ovf = wc > (uint32_t)kCluRegion ? 1u : 0u;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                tot_c += __shfl_xor_sync(0xffffffffu, tot_c, o);
+                ovf |= __shfl_xor_sync(0xffffffffu, ovf, o);
+            }
+            if (lane == 0) {
+                sh.nc = tot_c;
+                sh.ovf = ovf;
+            }
+        }
+        __syncthreads();
+    }
+    cluster_arrive();
+    cluster_wait();
+    if (warp == 0) {
+        const bool on = lane < kCluCtas;
+        const uint32_t nq = on ? cluster_ld(&sh.nc, (uint32_t)lane) : 0u;
+        uint32_t ov = on ? cluster_ld(&sh.ovf, (uint32_t)lane) : 0u;
+        uint32_t ni = nq;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xffffffffu, ni, o);
+            if (lane >= o)
+                ni += x;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            ov |= __shfl_xor_sync(0xffffffffu, ov, o);
+        const uint32_t C = __shfl_sync(0xffffffffu, ni, 31);
+        if (lane < kCluCtas)
+            sh.pre[lane][kCluWarps] = ni - nq;           // first pair of block `lane`
+        if (lane == 0)
+            sh.fast = (ov == 0u && C >= (uint32_t)k && C <= (uint32_t)kCluGather) ? C : 0u;
+    }
+    __syncthreads();
+    const uint32_t C = sh.fast;
+
+    if (C > 0) {
+        // ---- 3. block 0 gathers the pairs in index order and selects
+        uint32_t *gk = keys, *gi = keys + kCluGather;
+        if (c == 0) {
+            // group g of 128 threads copies block g's regions
+            const int g = tid >> 7, gt = tid & 127;
+            if ((gt >> 5) == 0) {
+                const uint32_t wc = cluster_ld(&sh.wcnt[gt], (uint32_t)g);
+                uint32_t v = wc;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t x = __shfl_up_sync(0xffffffffu, v, o);
+                    if (gt >= o)
+                        v += x;
+                }
+                sh.pre[g][gt] = v - wc;                  // region offsets inside block g
+                if (gt == 31)
+                    sh.wa[g] = v;                        // block g's pair count
+            }
+            __syncthreads();
+            const uint32_t base = sh.pre[g][kCluWarps], ng = sh.wa[g];
+            for (uint32_t f = (uint32_t)gt; f < ng; f += 128) {
+                // the region holding pair f of block g: the last w with pre[g][w] <= f
+                int lo = 0, hi = kCluWarps - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (sh.pre[g][mid] <= f)
+                        lo = mid;
+                    else
+                        hi = mid - 1;
+                }
+                const uint2 pr = cluster_ld2(cand + lo * kCluRegion + (f - sh.pre[g][lo]), (uint32_t)g);
+                gk[base + f] = pr.x;
+                gi[base + f] = pr.y;
+            }
+        }
+        // the other blocks may leave once block 0 has read their pairs
+        cluster_arrive();
+        if (c == 0) {
+            __syncthreads();                             // the gathered pairs
+            if (tid < kCluSel)
+                clu_select_team(gk, gi, C, k, tot, pub, out, sh);
+            __syncthreads();
+        }
+        cluster_wait();
+        return;
+    }
+
+    // ---- 4. every key: three radix rounds over the whole row
+    uint32_t prefix = 0, pmask = 0, need = (uint32_t)k;
+#pragma unroll 1
+    for (int r = 0; r < 3; r++) {
+        const int shift = r == 0 ? 21 : (r == 1 ? 10 : 0);
+        const uint32_t dmask = r == 2 ? 1023u : 2047u;
+        for (int b = tid; b < kCluCopies * kCluBins; b += kCluThreads)
+            hc[b] = 0;
+        __syncthreads();
+        uint32_t *h = hc + (lane & (kCluCopies - 1)) * kCluBins;
+#pragma unroll 4
+        for (int j = tid; j < n; j += kCluThreads) {
+            const uint32_t kk = keys[j];
+            if ((kk & pmask) == prefix)
+                atomicAdd(&h[(kk >> shift) & dmask], 1u);
+        }
+        __syncthreads();
+        uint32_t *pr = pub + (r & 1) * kCluBins;
+        for (int b = tid; b < kCluBins; b += kCluThreads)
+            pr[b] = hc[b] + hc[kCluBins + b] + hc[2 * kCluBins + b] + hc[3 * kCluBins + b];
+        // every block's counts of this round are published; the buffer of the
+        // round before the last is free again (its readers have passed the
+        // previous barrier)
+        cluster_arrive();
+        cluster_wait();
+        for (int b = tid; b < kCluBins; b += kCluThreads) {
+            uint32_t t = 0;
+#pragma unroll
+            for (int q = 0; q < kCluCtas; q++)
+                t += cluster_ld(pr + b, (uint32_t)q);
+            tot[b] = t;
+        }
+        __syncthreads();
+        clu_find<kCluThreads>(tot, need, sh);
+        prefix |= sh.bin << shift;
+        pmask |= dmask << shift;
+        need -= sh.above;
+        __syncthreads();                       // sh.bin and sh.above are rewritten next round
+    }
+    const uint32_t T = prefix;
+
+    // counts above T and equal to T: warp w covers entries [1024 w, +1024)
+    const int wbase = warp * 1024;
+    uint32_t gt = 0, eq = 0;
+#pragma unroll 4
+    for (int i = 0; i < 32; i++) {
+        const int j = wbase + 32 * i + lane;
+        const bool v = j < n;
+        const uint32_t kk = v ? keys[j] : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, v && kk > T));
+        eq += __popc(__ballot_sync(0xffffffffu, v && kk == T));
+    }
+    // per-warp prefix (one lane per warp contributes the warp's counts)
+    uint32_t gt_b, eq_b, gt_c, eq_c;
+    clu_scan2<kCluThreads>(lane == 0 ? gt : 0u, lane == 0 ? eq : 0u, sh, &gt_b, &eq_b, &gt_c, &eq_c);
+    gt_b = __shfl_sync(0xffffffffu, gt_b, 0);
+    eq_b = __shfl_sync(0xffffffffu, eq_b, 0);
+    if (tid == 0) {
+        sh.cnt[0] = gt_c;
+        sh.cnt[1] = eq_c;
+    }
+    cluster_arrive();
+    cluster_wait();
+    if (warp == 0) {
+        // lane q < kCluCtas: block q's counts; ties go to the lowest blocks first
+        const bool on = lane < kCluCtas;
+        const uint32_t g = on ? cluster_ld(&sh.cnt[0], (uint32_t)lane) : 0u;
+        const uint32_t e = on ? cluster_ld(&sh.cnt[1], (uint32_t)lane) : 0u;
+        uint32_t ei = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xffffffffu, ei, o);
+            if (lane >= o)
+                ei += x;
+        }
+        const uint32_t ebefore = ei - e;
+        const uint32_t take = need > ebefore ? (need - ebefore < e ? need - ebefore : e) : 0u;
+        const uint32_t sel = g + take;
+        uint32_t si = sel;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xffffffffu, si, o);
+            if (lane >= o)
+                si += x;
+        }
+        if (lane == (int)c) {
+            sh.off = si - sel;
+            sh.take = take;
+        }
+    }
+    // the other blocks' shared memory is not read past this point
+    cluster_arrive();
+    __syncthreads();
+    const uint32_t take = sh.take;
+    uint32_t eqrun = eq_b;
+    uint32_t pos = sh.off + gt_b + (eq_b < take ? eq_b : take);
+#pragma unroll 4
+    for (int i = 0; i < 32; i++) {
+        const int j = wbase + 32 * i + lane;
+        const bool v = j < n;
+        const uint32_t kk = v ? keys[j] : 0u;
+        const bool ise = v && kk == T;
+        const unsigned be = __ballot_sync(0xffffffffu, ise);
+        const bool sel = (v && kk > T) || (ise && eqrun + __popc(be & lt) < take);
+        const unsigned bs = __ballot_sync(0xffffffffu, sel);
+        const uint32_t at = pos + __popc(bs & lt);
+        if (sel && at < (uint32_t)k)
+            out[at] = (int32_t)(b0 + j);
+        eqrun += __popc(be);
+        pos += __popc(bs);
+    }
+    // a block leaves only when no other block of its cluster can still read
+    // its shared memory
+    cluster_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -1387,14 +2036,13 @@ cudaError_t launch_topk_cand(const TopkCandArgs &a, cudaStream_t s)
 size_t topk_workspace_size(int64_t rows, int64_t E, int k)
 {
     (void)k;
-    if (E < kMultiMinE || rows > 65535 || rows <= 0 || (E + kChunk - 1) / kChunk > 1024)
+    if (cluster_takes(rows, E) || E < kMultiMinE || rows > 65535 || rows <= 0 || (E + kChunk - 1) / kChunk > 1024)
         return 0;
     return multi_ws_bytes(rows, E);
 }
 
 cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s)
 {
-    (void)err;
     if (a.rows == 0)
         return cudaSuccess;
     if (a.E <= 32 * kPerLane) {
@@ -1412,6 +2060,15 @@ cudaError_t launch_topk(const TopkArgs &a, unsigned *err, cudaStream_t s)
     }
     cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kResident * (int)sizeof(uint32_t));
+    if (cluster_takes(a.rows, a.E)) {
+        cudaError_t e = cudaFuncSetAttribute(
+            topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCluSmem);
+        if (e != cudaSuccess)
+            return e;
+        topk_cluster_kernel<<<dim3(kCluCtas, (unsigned)a.rows), kCluThreads, kCluSmem, s>>>(
+            a.scores, a.E, a.ld, a.q_pos, a.m, a.k, a.idx, err);
+        return cudaGetLastError();
+    }
     if (topk_workspace_size(a.rows, a.E, a.k) > 0) {
         const int nchunks = (int)((a.E + kChunk - 1) / kChunk);
         const MultiWs w = multi_ws(a.ws, a.rows, a.E);

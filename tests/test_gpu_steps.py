@@ -224,10 +224,11 @@ def test_topk_mid_rows_clustered_sorted_and_sparse():
 
 
 def test_topk_long_rows_split_over_blocks():
-    # rows past 65536 entries go through the four-launch chunked path with a
-    # caller workspace: candidates of the threshold bin across chunk borders,
+    # rows of 65536 .. 262144 entries: one cluster of blocks per row, each
+    # block a share of the row; the threshold key's ties across block borders,
     # short rows (V <= k) mixed in, and a row with massive ties
     rows, E, k = 5, 100000, 700
+    assert abi.csa_topk_workspace_size(rows, E, k) == 0
     pos = [E - 1, 70000, 500, E - 1, 80000]
     _topk_case(rows, E, k, 1, pos, 24)
     sc = torch.zeros(2, E)
@@ -239,6 +240,34 @@ def test_topk_long_rows_split_over_blocks():
     abi.csa_get_error()
     ref = oracle.topk(sc.double().numpy(), q_pos.numpy(), 1, k)
     np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_cluster_rows_unaligned_and_tied():
+    # decode-width rows (262144 entries) whose starts are not 16-byte aligned
+    # (row stride E + 1: the shares are read element by element), the largest
+    # k, and rows whose k-th value is tied across every block of the row
+    rows, E, k = 6, 262144, 4096
+    rng = np.random.default_rng(28)
+    full = rng.standard_normal((rows, E + 1)).astype(np.float32)
+    full[1, :E] = np.where(rng.random(E) < 0.02, 2.0, -1.0)     # ~5200 tied at the top
+    full[2, :E] = 0.0
+    full[2, 100:E:50] = -0.0                                    # -0 and +0 are one value
+    full[3, :E] = np.round(full[3, :E] * 4) / 4                 # many ties in every digit
+    q_pos = torch.tensor([E - 1, E - 1, E - 1, 4000, 200000, E - 2], dtype=torch.int64)
+    sc = torch.as_tensor(full)
+    idx = torch.full((rows, k), -7, device=DEV, dtype=torch.int32)
+    abi.csa_topk(sc.to(DEV), q_pos.to(DEV), 1, k, idx, E)      # row stride E + 1
+    abi.csa_get_error()
+    ref = oracle.topk(full[:, :E].astype(np.float64), q_pos.numpy(), 1, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_rows_past_cluster_reach():
+    # rows longer than 262144 entries: the four-launch chunked path with a
+    # caller workspace
+    rows, E, k = 3, 300000, 1024
+    assert abi.csa_topk_workspace_size(rows, E, k) > 0
+    _topk_case(rows, E, k, 1, [E - 1, 290000, 262145], 29)
 
 
 def test_topk_all_equal_scores_prefers_low_indices():
