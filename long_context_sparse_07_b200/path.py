@@ -168,16 +168,38 @@ class CsaPrefill:
 
     QUERY_SIDE = ("q", "qI", "qI_scale", "wI")
 
+    @staticmethod
+    def chunk_plan(nq: int, chunk: int, small: int = 2048):
+        """Query chunk sizes for ``step_from_host``: doubling from ``small`` up
+        to ``chunk`` at the start (the first output leaves early, so the
+        device-to-host copies run beside the host-to-device ones for most of
+        the step), full chunks in the middle, and halving back to ``small`` at
+        the end (little computation and output are left once the last queries
+        have arrived)."""
+        ramp = []
+        s = small
+        while s < chunk:
+            ramp.append(s)
+            s *= 2
+        mid = nq - 2 * sum(ramp)
+        if not ramp or mid < chunk:
+            return [min(chunk, nq - lo) for lo in range(0, nq, chunk)]
+        sizes = list(ramp) + [chunk] * (mid // chunk)
+        if mid % chunk:
+            sizes.append(mid % chunk)
+        return sizes + ramp[::-1]
+
     def step_from_host(self, host_in: Dict[str, torch.Tensor], host_out: torch.Tensor,
-                       stream=None, chunk: int = 16384):
+                       stream=None, chunk: int = 8192):
         """One step from pinned host operands (keys as ``inputs()``) to a
         pinned host output (shaped like ``result()``), the copies overlapped
         with the computation: the KV side arrives first and is compressed;
-        then the queries come in chunks, each chunk's selection and attention
-        running while the next chunk's queries arrive and the previous chunk's
-        output leaves on a second copy stream (host-to-device and
-        device-to-host copies run at the same time). The result equals
-        ``step()``'s: every query's work is the same, only grouped by chunk."""
+        then the queries come in chunks (``chunk_plan``), each chunk's
+        selection and attention running while the next chunk's queries arrive
+        and the previous chunk's output leaves on a second copy stream
+        (host-to-device and device-to-host copies run at the same time). The
+        result equals ``step()``'s: every query's work is the same, only
+        grouped by chunk."""
         cur = stream if stream is not None else torch.cuda.current_stream()
         d, w = self.d, self.w
         if self.rope_dims or not self.fused:
@@ -201,20 +223,25 @@ class CsaPrefill:
         self.compress_kv(cur)
         self.compress_index(cur)
         qs = d.get("qI_scale")
-        for lo in range(0, self.nq, chunk):
-            hi = min(self.nq, lo + chunk)
+        plan = self.chunk_plan(self.nq, chunk)
+        # one workspace pair, for the largest chunk (the chunks run one after
+        # another on one stream)
+        big = max(plan)
+        if big not in self._chunk_ws:
+            nf = max(abi.csa_indexer_topk_workspace_size(1, r, w.E, w.hI, w.cI, w.k, d["qI"])
+                     for r in set(plan))
+            na = max(abi.csa_mqa_workspace_size(1, r, w.h, w.c, w.k + w.n_win) for r in set(plan))
+            self._chunk_ws = {big: (
+                torch.empty(nf, device=self.out.device, dtype=torch.uint8) if nf else None,
+                torch.empty(na, device=self.out.device, dtype=torch.uint8) if na else None)}
+        fws, aws = self._chunk_ws[big]
+        lo = 0
+        for rows in plan:
+            hi = lo + rows
             with torch.cuda.stream(h2d):
                 for k in qside:
                     d[k][lo:hi].copy_(host_in[k][lo:hi], non_blocking=True)
             cur.wait_event(h2d.record_event())
-            rows = hi - lo
-            if rows not in self._chunk_ws:
-                nf = abi.csa_indexer_topk_workspace_size(1, rows, w.E, w.hI, w.cI, w.k, d["qI"])
-                na = abi.csa_mqa_workspace_size(1, rows, w.h, w.c, w.k + w.n_win)
-                self._chunk_ws[rows] = (
-                    torch.empty(nf, device=self.out.device, dtype=torch.uint8) if nf else None,
-                    torch.empty(na, device=self.out.device, dtype=torch.uint8) if na else None)
-            fws, aws = self._chunk_ws[rows]
             abi.csa_indexer_topk(d["qI"][lo:hi][None], qs[lo:hi][None] if qs is not None else None,
                                  d["wI"][lo:hi][None], self.kI, self.q_pos[lo:hi][None], w.m, w.k,
                                  self.idx[lo:hi], w.E, workspace=fws, stream=cur)
@@ -225,6 +252,7 @@ class CsaPrefill:
             d2h.wait_event(cur.record_event())
             with torch.cuda.stream(d2h):
                 host_out[:, lo:hi].copy_(self.out[:, lo:hi], non_blocking=True)
+            lo = hi
         cur.wait_stream(d2h)
 
 
