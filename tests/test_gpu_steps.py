@@ -262,6 +262,27 @@ def test_topk_cluster_rows_unaligned_and_tied():
     np.testing.assert_array_equal(idx.cpu().numpy(), ref)
 
 
+def test_topk_cluster_rows_mixed_lengths_and_orders():
+    # 40 rows of a 131072-wide table: lengths from k + 1 up to the full row,
+    # normal, exponential, sorted and grid-valued rows (the candidate path and
+    # the all-keys path both taken), k = 1000
+    rows, E, k = 40, 131072, 1000
+    rng = np.random.default_rng(30)
+    sc = rng.standard_normal((rows, E)).astype(np.float32)
+    sc[1::5] = rng.exponential(1.0, size=(len(range(1, rows, 5)), E))
+    sc[2] = np.arange(E, dtype=np.float32)                 # ascending
+    sc[3] = -np.arange(E, dtype=np.float32)                # descending
+    sc[4::5] = np.round(sc[4::5] * 8) / 8                  # many ties near every digit
+    V = np.concatenate([[k + 1, k + 2, 2 * k, 32 * k + 7, E, E - 1, 65537, 100001],
+                        rng.integers(k + 1, E + 1, size=rows - 8)])
+    q_pos = torch.as_tensor(V - 1, dtype=torch.int64)
+    idx = torch.full((rows, k), -7, device=DEV, dtype=torch.int32)
+    abi.csa_topk(torch.as_tensor(sc).to(DEV), q_pos.to(DEV), 1, k, idx, E)
+    abi.csa_get_error()
+    ref = oracle.topk(sc.astype(np.float64), q_pos.numpy(), 1, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+
+
 def test_topk_rows_past_cluster_reach():
     # rows longer than 262144 entries: the four-launch chunked path with a
     # caller workspace
