@@ -900,8 +900,9 @@ topk_final_kernel(const int64_t *__restrict__ q_pos, int64_t E, int m, int k, in
 // Long rows of up to kCluCtas * kCluChunk entries (decode over a 1 M-token
 // context: 262144 entries): one launch, each row taken by a cluster of
 // kCluCtas blocks, block c staging the keys of its contiguous share of the
-// row in shared memory. The blocks talk through distributed shared memory
-// and hardware cluster barriers only.
+// row in shared memory (bulk copies; plain loads when the share does not
+// start on a 16-byte boundary). The blocks talk through distributed shared
+// memory and hardware cluster barriers only.
 //  1. Bound: every 32nd key of the row is a sample; with mu = k ns / V the
 //     samples expected at or above the row's k-th largest key, a bound with
 //     ks = 1.25 mu + 4 sqrt(mu) + 8 samples at or above it lies below that
