@@ -120,3 +120,17 @@ def test_no_alloc_validates_before_touching_the_device(lib):
     st = lib.csa_sparse_mqa_noalloc(P, abi.CSA_BF16, kv, 10, 4, None, 5, P, 10, None, 4, P, P, 1,
                                     4, 8, 0.1, P, None, None)
     assert st == -1 and b"idx" in lib.csa_last_message()
+
+
+def test_topk_workspace_contract(lib):
+    # rows up to 2048 .. 64 K entries and rows of 64 K .. 256 K entries (one
+    # cluster of blocks per row) need no workspace; longer rows are split over
+    # many blocks in four launches and need one that grows with rows * E
+    for E in (1024, 40000, 65535, 65536, 100000, 262144):
+        assert abi.csa_topk_workspace_size(8, E, 1024) == 0, E
+    small = abi.csa_topk_workspace_size(2, 300000, 1024)
+    assert small >= 2 * 300000 * 16
+    assert abi.csa_topk_workspace_size(4, 300000, 1024) > small
+    # decode through the one-call entry: the indexer, then one top-k launch
+    assert abi.csa_indexer_topk_launches(8, 1, 262144, 64, 128, 1024, abi.CSA_E4M3) == 2
+    assert abi.csa_indexer_topk_launches(2, 1, 300000, 64, 128, 1024, abi.CSA_E4M3) == 5
